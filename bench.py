@@ -1,0 +1,379 @@
+"""Throughput of the routed MoE layer forward on B200.
+
+One step = one whole forward of the layer (router GEMM + grouped top-k,
+permute, grouped fc1+SwiGLU / fc2, combine) over one batch of T synthetic
+tokens of the mid-size bf16 workload (T=2048, H=2048, I=1024, E=64, groups
+8/4, top-6, shared expert I=1024), weights resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun) every rank runs an independent replica on its own batch
+(tokens are independent, so the layer shards by batch with no exchange): weak
+scaling, whole-job tokens/s = N*T*K / max-over-ranks time.
+
+--impl reference times the CPU oracle (fp64 numpy) on a bounded token sample
+of the same workload, on rank 0 only.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+from synth.configs import BENCH_CONFIG  # noqa: E402
+
+METRIC = "MoE layer fwd tokens/s at 1 B200; % of roofline (tensor peak or HBM GB/s)"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _workload(cfg, l2_note):
+    return {
+        "workload": f"routed MoE layer forward, {cfg.name}",
+        "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "n_group": cfg.n_group,
+        "topk_group": cfg.topk_group, "top_k": cfg.top_k, "I_shared": cfg.I_shared,
+        "routed_scaling_factor": cfg.rsf, "pad_multiple": cfg.pad_multiple,
+        "global_batch": None, "seq_len": None, "l2": l2_note,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            parts = [x.strip() for x in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+
+def _oracle_inputs(cfg, T):
+    from oracle import moe_oracle as O
+    x = O.from_bf16(synth.gen_x(cfg, "cpu", T=T))
+    wr, bias = synth.gen_router(cfg, "cpu")
+    w1 = np.empty((cfg.E, cfg.I, cfg.H))
+    w3 = np.empty_like(w1)
+    w2 = np.empty((cfg.E, cfg.H, cfg.I))
+    for e in range(cfg.E):
+        a, b, c = synth.gen_expert_weights(cfg, e, "cpu")
+        w1[e], w3[e], w2[e] = O.from_bf16(a), O.from_bf16(b), O.from_bf16(c)
+    sh = synth.gen_shared_weights(cfg, "cpu")
+    sh = tuple(O.from_bf16(t) for t in sh) if sh is not None else None
+    return x, O.from_bf16(wr), bias.numpy().astype(np.float64), w1, w3, w2, sh
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(cfg, sample_tokens, steps, warmup):
+    """Oracle forward on a token sample; returns (tokens/s, seconds per step)."""
+    from oracle import moe_oracle as O
+    x, wr, bias, w1, w3, w2, sh = _oracle_inputs(cfg, sample_tokens)
+    scfg = cfg.scaled(T=sample_tokens)
+    for _ in range(warmup):
+        O.forward(scfg, x, wr, bias, w1, w3, w2, shared=sh)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        O.forward(scfg, x, wr, bias, w1, w3, w2, shared=sh)
+    dt = (time.perf_counter() - t0) / max(steps, 1)
+    return sample_tokens / dt, dt
+
+
+def run_reference(args, cfg):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    tokens = args.ref_tokens
+    tps, dt = time_oracle(cfg, tokens, args.steps, args.warmup)
+    cores = _blas_threads()
+    sample = (f"oracle forward (fp64 numpy) on a {tokens}-token sample of the workload "
+              f"(all {cfg.E} experts' weights), per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _workload(cfg, "host oracle; no GPU"),
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def grouped_mlp_algorithmic(cfg, touched):
+    """Bytes and FLOPs the grouped MLP call cannot avoid: every touched routed
+    expert's and the shared expert's weights read once; 6*H*I per row."""
+    wbytes = 2 * 3 * cfg.H * (touched * cfg.I + cfg.I_shared)
+    flops = 6 * cfg.H * (cfg.T * cfg.top_k * cfg.I + cfg.T * cfg.I_shared)
+    return wbytes, flops
+
+
+def layer_algorithmic(cfg, touched):
+    """Whole-layer algorithmic bytes / FLOPs: weights touched + shared + router,
+    x in and y out (bf16)."""
+    wb, fl = grouped_mlp_algorithmic(cfg, touched)
+    b = wb + 2 * cfg.E * cfg.H + 2 * 2 * cfg.T * cfg.H
+    f = fl + 2 * cfg.T * cfg.H * cfg.E
+    return b, f
+
+
+def run_ours(args, cfg):
+    import mixture_experts_layer_grouped_b200 as M
+    ws_n, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws_n > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    c = M.config_from_shape(cfg)
+    d = synth.gen_all(cfg, dev)
+    # each rank its own batch of tokens
+    if rank:
+        d["x"] = synth.gen_x(cfg.scaled(seed=rank), dev)
+    w = {k: d[k] for k in ("w1", "w3", "w2", "ws1", "ws3", "ws2") if k in d}
+    layer = M.MoELayer(c, w, d["w_router"], d["bias"])
+    x, y = d["x"], torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # warm-up (eager), then capture one forward into a CUDA graph
+    for _ in range(args.warmup):
+        layer.forward(x, out=y)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.forward(x, out=y)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    status = layer.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    # ---- timed region: device-resident inputs, graph replay
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    barrier()
+    ms_max = ms
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    value = ws_n * cfg.T / (ms_max * 1e-3)
+
+    # ---- e2e: host (pinned) buffers through the same C call, eager
+    x_h = x.cpu().pin_memory()
+    y_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, pin_memory=True)
+    for _ in range(args.warmup):
+        layer.forward(x_h, out=y_h)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        layer.forward(x_h, out=y_h)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1) / args.steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = ws_n * cfg.T / (e2e_ms * 1e-3)
+
+    # ---- roofline of the dominant call (grouped MLP: fc1+SwiGLU and fc2)
+    nbytes, r_cap = M.moe_workspace_size(c)
+    wsp = M.binding.new_workspace(nbytes, dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    logits = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
+    idx = torch.empty(cfg.T, cfg.top_k, **i32)
+    tw = torch.empty(cfg.T, cfg.top_k, dtype=torch.float32, device=dev)
+    counts, offsets = torch.empty(cfg.E, **i32), torch.empty(cfg.E + 1, **i32)
+    row_token, token_row = torch.empty(r_cap, **i32), torch.empty(cfg.T * cfg.top_k, **i32)
+    rows = torch.empty(r_cap, cfg.H, dtype=torch.bfloat16, device=dev)
+    out_rows = torch.empty(r_cap, cfg.H, dtype=torch.bfloat16, device=dev)
+    shared_out = (torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+                  if cfg.I_shared else None)
+    steps_ms = {"route": [], "permute": [], "grouped_mlp": [], "combine": []}
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    for it in range(args.warmup + args.steps):
+        evs[0].record(stream)
+        M.moe_route(c, x, d["w_router"], d["bias"], idx, tw, wsp, logits_out=logits)
+        evs[1].record(stream)
+        M.moe_permute(c, idx, x, counts, offsets, row_token, token_row, rows, wsp)
+        evs[2].record(stream)
+        M.moe_grouped_mlp(c, w, rows, counts, offsets, out_rows, wsp, x=x, shared_out=shared_out)
+        evs[3].record(stream)
+        M.moe_combine(c, out_rows, token_row, tw, y, shared_out=shared_out)
+        evs[4].record(stream)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            for i, k in enumerate(steps_ms):
+                steps_ms[k].append(evs[i].elapsed_time(evs[i + 1]))
+    touched = int((counts > 0).sum().item())
+    mlp_ms = statistics.mean(steps_ms["grouped_mlp"])
+    wbytes, flops = grouped_mlp_algorithmic(cfg, touched)
+    hbm, tf_burst, tf_sus, peak_kind = _peaks()
+    achieved_gbs = wbytes / (mlp_ms * 1e-3) / 1e9
+    lb, lf = layer_algorithmic(cfg, touched)
+    roof_ms = max(lb / (hbm * 1e9), lf / (tf_burst * 1e12)) * 1e3
+
+    if dist is not None:
+        dist.barrier()
+        del graph
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    cpu = None
+    if ws_n == 1 and not args.no_cpu_baseline:
+        tps, _ = time_oracle(cfg, args.ref_tokens, 1, 0)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+               "sample": f"oracle forward (fp64 numpy) on a {args.ref_tokens}-token sample of "
+                         f"the workload, one pass"}
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normal inputs and random-init weights of the workload)",
+        "config": dict(_workload(cfg, "inputs larger than L2: %.0f MB of expert weights per step"
+                                 % (2 * 3 * cfg.H * cfg.I * cfg.E / 1e6)),
+                       launch="CUDA graph of the one-call forward", parallelism=f"replicas{ws_n}"),
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm, "traffic": None,
+                     "kernel": "moe_grouped_mlp (fc1+SwiGLU and fc2 tcgen05 kernels)",
+                     "algorithmic_bytes_per_launch": wbytes, "ms_per_launch": mlp_ms,
+                     "tensor_tflops": flops / (mlp_ms * 1e-3) / 1e12,
+                     "tensor_frac": flops / (mlp_ms * 1e-3) / 1e12 / tf_burst,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs / bf16_tflops)"},
+        "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_max,
+                           "bytes": lb, "flops": lf, "experts_touched": touched},
+        "step_ms": {k: statistics.mean(v) for k, v in steps_ms.items()},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
+        "gpu_launches": 9 * args.steps,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"]},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=BENCH_CONFIG, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--ref-tokens", type=int, default=128)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = synth.get_config(args.config)
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * moe_b200.h -- C ABI of the routed Mixture-of-Experts layer forward on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (TransformerEngine PR "DeepSeekV3Layer: full MoE transformer
+ * layer", Description, DeepSeekV3MoE bullet): a sigmoid router with an
+ * aux-loss-free bias and grouped top-k selection, tokens permuted into
+ * expert-major order, per-expert fc1 -> SwiGLU -> fc2 as a grouped GEMM, and a
+ * gate-weighted combine back to token order, with an optional shared expert.
+ * Block-scaled variants: MXFP8 (same PR, Performance, MXFP8 rows) and NVFP4
+ * W4A4 (sglang PR "Mistral Large 3 NVFP4 TRTLLM MoE support", Modifications).
+ *
+ * Conventions for every call:
+ *   - All pointer arguments are DEVICE pointers unless stated otherwise.  The
+ *     caller allocates every buffer; no call allocates or frees memory.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream) and never synchronizes the host,
+ *     except moe_get_device_status.
+ *   - Matrices are row-major.  "bf16" is IEEE bfloat16 stored as uint16.
+ *   - Arguments are validated on the host before any launch; a bad argument
+ *     returns an error code and launches nothing.  Errors found on the device
+ *     (an expert index out of range, a wait that timed out) are written to a
+ *     status word at the start of the workspace and read back with
+ *     moe_get_device_status.  No kernel traps.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad enum       */
+  MOE_ERR_UNSUPPORTED = 2,  /* shape the kernels do not handle (see moe_config) */
+  MOE_ERR_WORKSPACE = 3,    /* workspace smaller than the size query returned  */
+  MOE_ERR_CAPACITY = 4,     /* device: expert index out of [0, E)             */
+  MOE_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up                  */
+  MOE_ERR_CUDA = 6          /* a CUDA runtime/driver call failed              */
+} moe_status;
+
+typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1, MOE_NVFP4 = 2 } moe_dtype;
+
+/*
+ * Layer shape.  T tokens of hidden size H; E routed experts of intermediate
+ * size I, in n_group contiguous groups of E/n_group; each token keeps the
+ * topk_group best groups and the top_k best experts inside them; gates are
+ * normalised and multiplied by routed_scaling_factor.  I_shared > 0 adds a
+ * shared expert of intermediate size I_shared applied to every token with
+ * weight 1.  Each expert's segment of the expert-major layout is padded to a
+ * multiple of pad_multiple rows.
+ *
+ * Supported: 1 <= T; H, I, I_shared multiples of 128; 1 <= E <= 1024;
+ * E % n_group == 0 with E/n_group >= 2 and n_group <= 32; 1 <= topk_group <=
+ * n_group; 1 <= top_k <= min(32, topk_group*E/n_group); pad_multiple >= 1
+ * (MXFP8/NVFP4: pad_multiple == 128).
+ */
+typedef struct moe_config {
+  int32_t T, H, I, E;
+  int32_t n_group, topk_group, top_k;
+  int32_t I_shared;
+  float routed_scaling_factor;
+  int32_t dtype;          /* moe_dtype */
+  int32_t pad_multiple;
+} moe_config;
+
+/*
+ * Expert weights as the grouped GEMM consumes them.
+ *   bf16 : w1, w3 [E, I, H]; w2 [E, H, I] (K-major: the contraction dim is
+ *          contiguous); ws1, ws3 [I_shared, H]; ws2 [H, I_shared].
+ *   The *_scales and *_global fields are used by MXFP8/NVFP4 only and are
+ *   written by moe_prepare_weights.
+ * Shared-expert fields are ignored when I_shared == 0.
+ */
+typedef struct moe_weights {
+  void* w1; void* w3; void* w2;
+  void* w1_scales; void* w3_scales; void* w2_scales;
+  float* w13_global; float* w2_global;
+  void* ws1; void* ws3; void* ws2;
+  void* ws1_scales; void* ws3_scales; void* ws2_scales;
+  float* ws13_global; float* ws2_global;
+} moe_weights;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(moe_status s);
+
+/*
+ * Sizes.  *bytes = scratch the step calls (moe_route .. moe_combine) need in
+ * `workspace`; *r_cap = rows of the expert-major buffers (row_token, the
+ * permuted rows, the grouped-GEMM outputs): T*top_k + E*(pad_multiple-1)
+ * rounded up to pad_multiple.  Either output pointer may be NULL.
+ */
+moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes, int32_t* r_cap);
+
+/*
+ * Router (DeepSeekV3MoE bullet: "fused sigmoid router with aux-loss-free bias
+ * and grouped top-k").
+ *   x [T, H] bf16, w_router [E, H] bf16, bias [E] fp32.
+ *   logits_in  [T, E] fp32 or NULL.  When given, the router GEMM is skipped
+ *              and selection runs on these logits.
+ *   logits_out [T, E] fp32: x . W_r^T with fp32 accumulation; required when
+ *              logits_in is NULL, ignored otherwise.
+ *   topk_idx [T, top_k] int32: selected experts, biased score descending,
+ *              ties to the lower index.  topk_w [T, top_k] fp32: gates
+ *              sigmoid(logit) / sum * routed_scaling_factor.
+ */
+moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
+                     const float* bias, const float* logits_in, float* logits_out,
+                     int32_t* topk_idx, float* topk_w, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/*
+ * Permute into padded expert-major order (Performance, "NCCL EP local
+ * permute": staging buffer to expert-major layout, zero-filled padding).
+ *   topk_idx [T, top_k] int32 (values outside [0, E) set MOE_ERR_CAPACITY on
+ *   the device and are skipped).
+ *   counts [E] int32: rows per expert.  offsets [E+1] int32: exclusive scan of
+ *   counts rounded up to pad_multiple.  row_token [r_cap] int32: token of each
+ *   row, -1 for pad rows and rows past offsets[E].  token_row [T*top_k] int32:
+ *   row of (t, j).  Within a segment tokens ascend.
+ *   src_rows: bf16 x [T, H] (BF16), e4m3 codes [T, H] (MXFP8), packed e2m1
+ *   codes [T, H/2] (NVFP4).  dst_rows [r_cap, same row bytes]; pad rows zero.
+ *   src_scales / dst_scales: block scales (MXFP8/NVFP4) in the MMA scale
+ *   layout of moe_quantize, for T and r_cap rows; NULL for BF16.
+ */
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx,
+                       const void* src_rows, const void* src_scales,
+                       int32_t* counts, int32_t* offsets, int32_t* row_token,
+                       int32_t* token_row, void* dst_rows, void* dst_scales,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Grouped expert MLP (DeepSeekV3MoE bullet: GroupedLinear -> ScaledSwiGLU ->
+ * GroupedLinear): for every expert e and its rows X_e,
+ *   h = bf16(silu(X_e W1_e^T) * (X_e W3_e^T));  out = bf16(h W2_e^T),
+ * and the same for the shared expert on all T tokens of x.
+ *   rows [r_cap, H] (as moe_permute's dst_rows), counts/offsets from
+ *   moe_permute; x [T, H] in token order (shared expert input; may be NULL
+ *   when I_shared == 0).
+ *   out_rows [r_cap, H] bf16: fc2 output per row (rows of pads untouched).
+ *   shared_out [T, H] bf16 or NULL when I_shared == 0.
+ * Tensor-core kernels: tcgen05 MMA with TMEM accumulators fed by TMA.
+ */
+moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w,
+                           const void* rows, const void* row_scales,
+                           const void* x, const void* x_scales, const float* x_global,
+                           const int32_t* counts, const int32_t* offsets,
+                           void* out_rows, void* shared_out,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Combine (gate-weighted scatter-add, written as a per-token gather-reduce):
+ *   y[t] = bf16( sum_{j<top_k} topk_w[t,j] * out_rows[token_row[t*top_k+j]]
+ *                + shared_out[t] ), fp32 accumulation in j order.
+ *   shared_out may be NULL.  y [T, H] bf16.
+ */
+moe_status moe_combine(const moe_config* cfg, const void* out_rows,
+                       const int32_t* token_row, const float* topk_w,
+                       const void* shared_out, void* y, void* stream);
+
+/*
+ * Whole layer: route -> (quantize) -> permute -> grouped MLP -> combine, with
+ * every intermediate in `workspace` (size from moe_forward_workspace_size).
+ * If xy_on_host != 0, x and y are HOST pointers (pinned memory recommended):
+ * x is copied to the device and y back, on `stream`, inside the call.
+ */
+moe_status moe_forward_workspace_size(const moe_config* cfg, size_t* bytes);
+moe_status moe_forward(const moe_config* cfg, const moe_weights* w,
+                       const void* w_router, const float* bias,
+                       const void* x, void* y, int32_t xy_on_host,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Reads (and clears) the device status word at the start of `workspace`.
+ * Synchronizes `stream`.  *device_status receives a moe_status value.
+ */
+moe_status moe_get_device_status(void* workspace, int32_t* device_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,25 @@
+"""Routed Mixture-of-Experts layer forward on one B200 (sm_100a).
+
+A thin ctypes binding over ``libmoe_b200.so``: the functions below marshal
+torch tensors into device pointers and call the C ABI of include/moe_b200.h
+with the same names.  Every step runs in the library's CUDA kernels; there is
+no fallback path, and importing the binding fails loudly when the library has
+not been built.
+"""
+
+from .binding import (  # noqa: F401
+    MoEConfig,
+    MoEWeights,
+    MoEError,
+    config_from_shape,
+    lib,
+    moe_workspace_size,
+    moe_forward_workspace_size,
+    moe_route,
+    moe_permute,
+    moe_grouped_mlp,
+    moe_combine,
+    moe_forward,
+    moe_get_device_status,
+    MoELayer,
+)

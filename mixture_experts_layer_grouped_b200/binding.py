@@ -1,0 +1,228 @@
+"""ctypes binding of libmoe_b200.so (argument marshalling only).
+
+Each ``moe_*`` function takes torch tensors, checks device/dtype/contiguity,
+and passes raw pointers, sizes and the current CUDA stream to the C function of
+the same name.  Nothing here computes any part of the layer.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+DTYPES = {"bf16": 0, "mxfp8": 1, "nvfp4": 2}
+
+STATUS = {
+    0: "ok", 1: "invalid argument", 2: "unsupported shape or dtype",
+    3: "workspace too small", 4: "expert index out of range (device)",
+    5: "bounded wait timed out (device)", 6: "CUDA error",
+}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)} ({code})")
+
+
+class MoEConfig(ctypes.Structure):
+    _fields_ = [
+        ("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+        ("E", ctypes.c_int32), ("n_group", ctypes.c_int32),
+        ("topk_group", ctypes.c_int32), ("top_k", ctypes.c_int32),
+        ("I_shared", ctypes.c_int32), ("routed_scaling_factor", ctypes.c_float),
+        ("dtype", ctypes.c_int32), ("pad_multiple", ctypes.c_int32),
+    ]
+
+
+_WEIGHT_FIELDS = [
+    "w1", "w3", "w2", "w1_scales", "w3_scales", "w2_scales", "w13_global", "w2_global",
+    "ws1", "ws3", "ws2", "ws1_scales", "ws3_scales", "ws2_scales", "ws13_global", "ws2_global",
+]
+
+
+class MoEWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _WEIGHT_FIELDS]
+
+
+def config_from_shape(s, T=None) -> MoEConfig:
+    """MoEConfig from any object with the layer's shape attributes."""
+    return MoEConfig(
+        T=s.T if T is None else T, H=s.H, I=s.I, E=s.E, n_group=s.n_group,
+        topk_group=s.topk_group, top_k=s.top_k, I_shared=s.I_shared,
+        routed_scaling_factor=s.rsf, dtype=DTYPES[s.dtype], pad_multiple=s.pad_multiple)
+
+
+_lib = None
+_VP = ctypes.c_void_p
+_CFG = ctypes.POINTER(MoEConfig)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m mixture_experts_layer_grouped_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        sig = {
+            "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "moe_workspace_size": ([_CFG, ctypes.POINTER(ctypes.c_size_t),
+                                    ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
+            "moe_forward_workspace_size": ([_CFG, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+            "moe_route": ([_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP],
+                          ctypes.c_int),
+            "moe_permute": ([_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                             ctypes.c_size_t, _VP], ctypes.c_int),
+            "moe_grouped_mlp": ([_CFG, ctypes.POINTER(MoEWeights), _VP, _VP, _VP, _VP, _VP,
+                                 _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
+            "moe_combine": ([_CFG, _VP, _VP, _VP, _VP, _VP, _VP], ctypes.c_int),
+            "moe_forward": ([_CFG, ctypes.POINTER(MoEWeights), _VP, _VP, _VP, _VP,
+                             ctypes.c_int32, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
+            "moe_get_device_status": ([_VP, ctypes.POINTER(ctypes.c_int32), _VP], ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _cuda(t, dtype, name):
+    if t is None:
+        return None
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got "
+                         f"{t.dtype} on {t.device} (contiguous={t.is_contiguous()})")
+    return t
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, code):
+    if code != 0:
+        raise MoEError(fn, code)
+
+
+def moe_workspace_size(cfg: MoEConfig):
+    b, r = ctypes.c_size_t(), ctypes.c_int32()
+    _check("moe_workspace_size", lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(b),
+                                                          ctypes.byref(r)))
+    return b.value, r.value
+
+
+def moe_forward_workspace_size(cfg: MoEConfig):
+    b = ctypes.c_size_t()
+    _check("moe_forward_workspace_size",
+           lib().moe_forward_workspace_size(ctypes.byref(cfg), ctypes.byref(b)))
+    return b.value
+
+
+def new_workspace(nbytes, device="cuda"):
+    """A zeroed byte buffer (the status word must start at zero)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def moe_route(cfg, x, w_router, bias, topk_idx, topk_w, workspace, logits_in=None,
+              logits_out=None, stream=None):
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    _check("moe_route", lib().moe_route(
+        ctypes.byref(cfg), _p(_cuda(x, bf, "x")), _p(_cuda(w_router, bf, "w_router")),
+        _p(_cuda(bias, f32, "bias")), _p(_cuda(logits_in, f32, "logits_in")),
+        _p(_cuda(logits_out, f32, "logits_out")), _p(_cuda(topk_idx, i32, "topk_idx")),
+        _p(_cuda(topk_w, f32, "topk_w")), _p(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_permute(cfg, topk_idx, src_rows, counts, offsets, row_token, token_row, dst_rows,
+                workspace, src_scales=None, dst_scales=None, stream=None):
+    i32 = torch.int32
+    _check("moe_permute", lib().moe_permute(
+        ctypes.byref(cfg), _p(_cuda(topk_idx, i32, "topk_idx")), _p(src_rows), _p(src_scales),
+        _p(_cuda(counts, i32, "counts")), _p(_cuda(offsets, i32, "offsets")),
+        _p(_cuda(row_token, i32, "row_token")), _p(_cuda(token_row, i32, "token_row")),
+        _p(dst_rows), _p(dst_scales), _p(workspace), workspace.numel(), _stream(stream)))
+
+
+def weights_struct(w: dict) -> MoEWeights:
+    return MoEWeights(**{k: (w[k].data_ptr() if w.get(k) is not None else None)
+                         for k in _WEIGHT_FIELDS})
+
+
+def moe_grouped_mlp(cfg, weights, rows, counts, offsets, out_rows, workspace, x=None,
+                    shared_out=None, row_scales=None, x_scales=None, x_global=None,
+                    stream=None):
+    ws = weights if isinstance(weights, MoEWeights) else weights_struct(weights)
+    i32 = torch.int32
+    _check("moe_grouped_mlp", lib().moe_grouped_mlp(
+        ctypes.byref(cfg), ctypes.byref(ws), _p(rows), _p(row_scales), _p(x), _p(x_scales),
+        _p(x_global), _p(_cuda(counts, i32, "counts")), _p(_cuda(offsets, i32, "offsets")),
+        _p(out_rows), _p(shared_out), _p(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_combine(cfg, out_rows, token_row, topk_w, y, shared_out=None, stream=None):
+    bf = torch.bfloat16
+    _check("moe_combine", lib().moe_combine(
+        ctypes.byref(cfg), _p(_cuda(out_rows, bf, "out_rows")),
+        _p(_cuda(token_row, torch.int32, "token_row")), _p(_cuda(topk_w, torch.float32, "topk_w")),
+        _p(_cuda(shared_out, bf, "shared_out")), _p(_cuda(y, bf, "y")), _stream(stream)))
+
+
+def moe_forward(cfg, weights, w_router, bias, x, y, workspace, stream=None):
+    """Whole layer.  If x and y are host tensors they are copied inside the call."""
+    ws = weights if isinstance(weights, MoEWeights) else weights_struct(weights)
+    on_host = not x.is_cuda
+    if on_host != (not y.is_cuda):
+        raise ValueError("x and y must both be host tensors or both device tensors")
+    _check("moe_forward", lib().moe_forward(
+        ctypes.byref(cfg), ctypes.byref(ws), _p(_cuda(w_router, torch.bfloat16, "w_router")),
+        _p(_cuda(bias, torch.float32, "bias")), _p(x), _p(y), 1 if on_host else 0,
+        _p(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_get_device_status(workspace, stream=None) -> int:
+    v = ctypes.c_int32()
+    _check("moe_get_device_status",
+           lib().moe_get_device_status(_p(workspace), ctypes.byref(v), _stream(stream)))
+    return v.value
+
+
+class MoELayer:
+    """A layer with its weights resident on the device.
+
+    ``weights`` maps the moe_weights field names (w1, w3, w2, ws1, ...) to
+    device tensors; ``forward(x)`` runs the whole layer through moe_forward.
+    """
+
+    def __init__(self, cfg: MoEConfig, weights: dict, w_router, bias, device="cuda"):
+        self.cfg = cfg
+        self.weights = dict(weights)
+        self._ws_struct = weights_struct(self.weights)
+        self.w_router = w_router
+        self.bias = bias
+        self.workspace = new_workspace(moe_forward_workspace_size(cfg), device)
+
+    def forward(self, x, out=None, stream=None):
+        if out is None:
+            out = torch.empty(self.cfg.T, self.cfg.H, dtype=torch.bfloat16, device=x.device,
+                              pin_memory=not x.is_cuda)
+        moe_forward(self.cfg, self._ws_struct, self.w_router, self.bias, x, out, self.workspace,
+                    stream)
+        return out
+
+    def device_status(self) -> int:
+        return moe_get_device_status(self.workspace)

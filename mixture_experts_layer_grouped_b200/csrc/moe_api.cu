@@ -1,0 +1,526 @@
+// C ABI entry points: argument checks, workspace layout, TMA descriptors and
+// kernel launches.  See include/moe_b200.h for the contract of each call.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "grouped_gemm.cuh"
+#include "route_permute_combine.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------
+// Workspace layout of the step calls.
+// ---------------------------------------------------------------------------
+struct StepLayout {
+  size_t status, hist, h, h_shared, total;
+  int32_t r_cap, ntiles;
+};
+
+int32_t r_cap_of(const moe_config& c) {
+  const int64_t P = c.pad_multiple;
+  const int64_t r = static_cast<int64_t>(c.T) * c.top_k + static_cast<int64_t>(c.E) * (P - 1);
+  return static_cast<int32_t>((r + P - 1) / P * P);
+}
+
+StepLayout step_layout(const moe_config& c) {
+  StepLayout L;
+  L.r_cap = r_cap_of(c);
+  L.ntiles = (c.T * c.top_k + kPermTile - 1) / kPermTile;
+  size_t o = 0;
+  L.status = o; o = align_up(o + 4);
+  L.hist = o; o = align_up(o + static_cast<size_t>(L.ntiles) * c.E * 4);
+  L.h = o; o = align_up(o + static_cast<size_t>(L.r_cap) * c.I * 2);
+  L.h_shared = o; o = align_up(o + static_cast<size_t>(c.T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
+  L.total = o;
+  return L;
+}
+
+struct FwdLayout {
+  StepLayout step;
+  size_t logits, topk_idx, topk_w, counts, offsets, row_token, token_row, rows, out_rows,
+      shared_out, x, y, total;
+};
+
+FwdLayout fwd_layout(const moe_config& c) {
+  FwdLayout F;
+  F.step = step_layout(c);
+  const size_t T = c.T, H = c.H, E = c.E, k = c.top_k, R = F.step.r_cap;
+  size_t o = F.step.total;
+  F.logits = o; o = align_up(o + T * E * 4);
+  F.topk_idx = o; o = align_up(o + T * k * 4);
+  F.topk_w = o; o = align_up(o + T * k * 4);
+  F.counts = o; o = align_up(o + E * 4);
+  F.offsets = o; o = align_up(o + (E + 1) * 4);
+  F.row_token = o; o = align_up(o + R * 4);
+  F.token_row = o; o = align_up(o + T * k * 4);
+  F.rows = o; o = align_up(o + R * H * 2);
+  F.out_rows = o; o = align_up(o + R * H * 2);
+  F.shared_out = o; o = align_up(o + (c.I_shared > 0 ? T * H * 2 : 0));
+  F.x = o; o = align_up(o + T * H * 2);
+  F.y = o; o = align_up(o + T * H * 2);
+  F.total = o;
+  return F;
+}
+
+moe_status check_config(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 1 || c->H < 1 || c->I < 1 || c->E < 1 || c->n_group < 1 || c->topk_group < 1 ||
+      c->top_k < 1 || c->pad_multiple < 1 || c->I_shared < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_BF16 && c->dtype != MOE_MXFP8 && c->dtype != MOE_NVFP4)
+    return MOE_ERR_INVALID_ARG;
+  if (c->H % 128 || c->I % 128 || (c->I_shared % 128)) return MOE_ERR_UNSUPPORTED;
+  if (c->E > kMaxExperts || c->E % c->n_group || c->E / c->n_group < 2 || c->n_group > 32)
+    return MOE_ERR_UNSUPPORTED;
+  if (c->topk_group > c->n_group) return MOE_ERR_UNSUPPORTED;
+  if (c->top_k > 32 || c->top_k > c->topk_group * (c->E / c->n_group)) return MOE_ERR_UNSUPPORTED;
+  const int64_t rcap = static_cast<int64_t>(c->T) * c->top_k +
+                       static_cast<int64_t>(c->E) * (c->pad_multiple - 1);
+  if (rcap > (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// Data paths built so far: bf16.
+moe_status check_dtype(const moe_config* c) {
+  return c->dtype == MOE_BF16 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+inline moe_status cuda_check(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  fprintf(stderr, "moe_b200: CUDA error %s\n", cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
+#define MOE_TRY(expr)                      \
+  do {                                     \
+    moe_status _s = (expr);                \
+    if (_s != MOE_OK) return _s;           \
+  } while (0)
+
+#define MOE_CUDA(expr) MOE_TRY(cuda_check(expr))
+
+inline moe_status launch_check() { return cuda_check(cudaGetLastError()); }
+
+// ---------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched through the runtime).
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D K-major tile map over [rows, inner] elements with a 128-byte swizzle.
+// The box is (128 bytes of K) x box_rows.
+moe_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                    uint64_t inner, uint64_t rows, uint64_t row_stride_bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MOE_ERR_CUDA;
+  if (reinterpret_cast<uintptr_t>(base) % 16 || row_stride_bytes % 16) return MOE_ERR_INVALID_ARG;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fprintf(stderr, "moe_b200: cuTensorMapEncodeTiled failed (%d)\n", static_cast<int>(r));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+template <int MODE>
+moe_status launch_gemm(const GemmParams& p, int max_units, cudaStream_t s) {
+  using C = GemmCfg<MODE>;
+  MOE_CUDA(cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  int grid = sm_count();
+  if (max_units < grid) grid = max_units;
+  if (grid < 1) return MOE_OK;
+  grouped_gemm_kernel<MODE><<<grid, kGemmThreads, C::SMEM_BYTES, s>>>(p);
+  return launch_check();
+}
+
+int32_t* status_ptr(void* ws) { return static_cast<int32_t*>(ws); }
+
+// ---------------------------------------------------------------------------
+// Step implementations (arguments already validated).
+// ---------------------------------------------------------------------------
+moe_status do_route(const moe_config& c, const void* x, const void* w_router, const float* bias,
+                    const float* logits_in, float* logits_out, int32_t* topk_idx, float* topk_w,
+                    void* ws, cudaStream_t s) {
+  const float* logits = logits_in;
+  if (!logits_in) {
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    MOE_TRY(make_map(&p.a0[1], w_router, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.H, c.E,
+                     static_cast<uint64_t>(c.H) * 2, kBM));
+    MOE_TRY(make_map(&p.b[1], x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.H, c.T,
+                     static_cast<uint64_t>(c.H) * 2, kBoxRows));
+    p.a0[0] = p.a0[1];
+    p.a1[0] = p.a1[1] = p.a0[1];
+    p.b[0] = p.b[1];
+    p.g[1].a_rows_per_expert = 0;
+    p.g[1].a_valid_rows = c.E;
+    p.g[1].n_slabs = (c.E + kBM - 1) / kBM;
+    p.g[1].k_tiles = c.H / kBK;
+    p.g[1].out = logits_out;
+    p.g[1].out_ld = c.E;
+    p.g[0] = p.g[1];
+    p.counts = nullptr;
+    p.offsets = nullptr;
+    p.E = 0;
+    p.dense_rows = c.T;
+    p.tile_n = 64;
+    p.status = status_ptr(ws);
+    const int units = ((c.T + 63) / 64) * p.g[1].n_slabs;
+    MOE_TRY(launch_gemm<kRouter>(p, units, s));
+    logits = logits_out;
+  }
+  SelArgs a;
+  a.logits = logits;
+  a.bias = bias;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.T = c.T;
+  a.E = c.E;
+  a.G = c.n_group;
+  a.g = c.topk_group;
+  a.k = c.top_k;
+  a.rsf = c.routed_scaling_factor;
+  const int per = (c.E + 31) / 32;
+  const dim3 grid((c.T + kSelWarps - 1) / kSelWarps), block(kSelWarps * 32);
+  if (per <= 1) route_select_kernel<1><<<grid, block, 0, s>>>(a);
+  else if (per <= 2) route_select_kernel<2><<<grid, block, 0, s>>>(a);
+  else if (per <= 4) route_select_kernel<4><<<grid, block, 0, s>>>(a);
+  else if (per <= 8) route_select_kernel<8><<<grid, block, 0, s>>>(a);
+  else if (per <= 12) route_select_kernel<12><<<grid, block, 0, s>>>(a);
+  else if (per <= 16) route_select_kernel<16><<<grid, block, 0, s>>>(a);
+  else route_select_kernel<32><<<grid, block, 0, s>>>(a);
+  return launch_check();
+}
+
+moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* src_rows,
+                      int32_t* counts, int32_t* offsets, int32_t* row_token, int32_t* token_row,
+                      void* dst_rows, void* ws, cudaStream_t s) {
+  const StepLayout L = step_layout(c);
+  PermArgs a;
+  a.topk_idx = topk_idx;
+  a.hist = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + L.hist);
+  a.counts = counts;
+  a.offsets = offsets;
+  a.row_token = row_token;
+  a.token_row = token_row;
+  a.status = status_ptr(ws);
+  a.n = c.T * c.top_k;
+  a.k = c.top_k;
+  a.E = c.E;
+  a.P = c.pad_multiple;
+  a.r_cap = L.r_cap;
+  a.ntiles = L.ntiles;
+  const size_t hsm = static_cast<size_t>(c.E) * 4;
+  permute_hist_kernel<<<L.ntiles, 256, hsm, s>>>(a);
+  MOE_TRY(launch_check());
+  permute_scan_kernel<<<1, 1024, 0, s>>>(a);
+  MOE_TRY(launch_check());
+  permute_rank_kernel<<<L.ntiles, 32, hsm, s>>>(a);
+  MOE_TRY(launch_check());
+  GatherArgs g;
+  g.src = static_cast<const uint8_t*>(src_rows);
+  g.dst = static_cast<uint8_t*>(dst_rows);
+  g.row_token = row_token;
+  g.offsets = offsets;
+  g.E = c.E;
+  g.row_bytes = c.H * 2;
+  permute_gather_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
+  return launch_check();
+}
+
+moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void* rows,
+                          const void* x, const int32_t* counts, const int32_t* offsets,
+                          void* out_rows, void* shared_out, void* ws, cudaStream_t s) {
+  const StepLayout L = step_layout(c);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  void* h = wsb + L.h;
+  void* hs = wsb + L.h_shared;
+  const bool sh = c.I_shared > 0;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
+  const int tile_n = 256;
+  // fc1 + SwiGLU
+  {
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    MOE_TRY(make_map(&p.a0[0], w.w1, BF, 2, H, E * I, H * 2, kBM));
+    MOE_TRY(make_map(&p.a1[0], w.w3, BF, 2, H, E * I, H * 2, kBM));
+    MOE_TRY(make_map(&p.b[0], rows, BF, 2, H, L.r_cap, H * 2, kBoxRows));
+    if (sh) {
+      MOE_TRY(make_map(&p.a0[1], w.ws1, BF, 2, H, Is, H * 2, kBM));
+      MOE_TRY(make_map(&p.a1[1], w.ws3, BF, 2, H, Is, H * 2, kBM));
+      MOE_TRY(make_map(&p.b[1], x, BF, 2, H, T, H * 2, kBoxRows));
+    } else {
+      p.a0[1] = p.a0[0];
+      p.a1[1] = p.a1[0];
+      p.b[1] = p.b[0];
+    }
+    p.g[0] = GemmGroup{c.I, c.I, c.I / kBM, c.H / kBK, h, c.I};
+    p.g[1] = GemmGroup{0, c.I_shared, c.I_shared / kBM, c.H / kBK, hs, c.I_shared};
+    p.counts = counts;
+    p.offsets = offsets;
+    p.E = c.E;
+    p.dense_rows = sh ? c.T : 0;
+    p.tile_n = tile_n;
+    p.status = status_ptr(ws);
+    const int max_chunks = c.E + (c.T * c.top_k) / tile_n + 1;
+    const int units = max_chunks * p.g[0].n_slabs +
+                      (sh ? ((c.T + tile_n - 1) / tile_n) * p.g[1].n_slabs : 0);
+    MOE_TRY(launch_gemm<kFc1>(p, units, s));
+  }
+  // fc2
+  {
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    MOE_TRY(make_map(&p.a0[0], w.w2, BF, 2, I, E * H, I * 2, kBM));
+    MOE_TRY(make_map(&p.b[0], h, BF, 2, I, L.r_cap, I * 2, kBoxRows));
+    if (sh) {
+      MOE_TRY(make_map(&p.a0[1], w.ws2, BF, 2, Is, H, Is * 2, kBM));
+      MOE_TRY(make_map(&p.b[1], hs, BF, 2, Is, T, Is * 2, kBoxRows));
+    } else {
+      p.a0[1] = p.a0[0];
+      p.b[1] = p.b[0];
+    }
+    p.a1[0] = p.a0[0];
+    p.a1[1] = p.a0[1];
+    p.g[0] = GemmGroup{c.H, c.H, c.H / kBM, c.I / kBK, out_rows, c.H};
+    p.g[1] = GemmGroup{0, c.H, c.H / kBM, (sh ? c.I_shared : 64) / kBK, shared_out, c.H};
+    p.counts = counts;
+    p.offsets = offsets;
+    p.E = c.E;
+    p.dense_rows = sh ? c.T : 0;
+    p.tile_n = tile_n;
+    p.status = status_ptr(ws);
+    const int max_chunks = c.E + (c.T * c.top_k) / tile_n + 1;
+    const int units = max_chunks * p.g[0].n_slabs +
+                      (sh ? ((c.T + tile_n - 1) / tile_n) * p.g[1].n_slabs : 0);
+    MOE_TRY(launch_gemm<kFc2>(p, units, s));
+  }
+  return MOE_OK;
+}
+
+moe_status do_combine(const moe_config& c, const void* out_rows, const int32_t* token_row,
+                      const float* topk_w, const void* shared_out, void* y, cudaStream_t s) {
+  CombineArgs a;
+  a.out_rows = static_cast<const __nv_bfloat16*>(out_rows);
+  a.token_row = token_row;
+  a.topk_w = topk_w;
+  a.shared = static_cast<const __nv_bfloat16*>(shared_out);
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.T = c.T;
+  a.H = c.H;
+  a.k = c.top_k;
+  combine_kernel<<<(c.T + 7) / 8, 256, 0, s>>>(a);
+  return launch_check();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+moe_status check_ws(const moe_config& c, void* ws, size_t bytes) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return MOE_ERR_INVALID_ARG;
+  if (bytes < step_layout(c).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+moe_status check_weights(const moe_config& c, const moe_weights* w) {
+  if (!w || !w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->w1) || !aligned16(w->w3) || !aligned16(w->w2)) return MOE_ERR_INVALID_ARG;
+  if (c.I_shared > 0) {
+    if (!w->ws1 || !w->ws3 || !w->ws2) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w->ws1) || !aligned16(w->ws3) || !aligned16(w->ws2)) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CAPACITY: return "expert index out of range (device)";
+    case MOE_ERR_TIMEOUT: return "bounded wait timed out (device)";
+    case MOE_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes, int32_t* r_cap) {
+  MOE_TRY(check_config(cfg));
+  const StepLayout L = step_layout(*cfg);
+  if (bytes) *bytes = L.total;
+  if (r_cap) *r_cap = L.r_cap;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
+                     const float* bias, const float* logits_in, float* logits_out,
+                     int32_t* topk_idx, float* topk_w, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  MOE_TRY(check_config(cfg));
+  MOE_TRY(check_ws(*cfg, workspace, workspace_bytes));
+  if (!bias || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!logits_in) {
+    if (!x || !w_router || !logits_out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+  }
+  return do_route(*cfg, x, w_router, bias, logits_in, logits_out, topk_idx, topk_w, workspace,
+                  static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* src_rows,
+                       const void* src_scales, int32_t* counts, int32_t* offsets,
+                       int32_t* row_token, int32_t* token_row, void* dst_rows, void* dst_scales,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  (void)src_scales;
+  (void)dst_scales;
+  MOE_TRY(check_config(cfg));
+  MOE_TRY(check_dtype(cfg));
+  MOE_TRY(check_ws(*cfg, workspace, workspace_bytes));
+  if (!topk_idx || !src_rows || !counts || !offsets || !row_token || !token_row || !dst_rows)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(src_rows) || !aligned16(dst_rows)) return MOE_ERR_INVALID_ARG;
+  return do_permute(*cfg, topk_idx, src_rows, counts, offsets, row_token, token_row, dst_rows,
+                    workspace, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w, const void* rows,
+                           const void* row_scales, const void* x, const void* x_scales,
+                           const float* x_global, const int32_t* counts, const int32_t* offsets,
+                           void* out_rows, void* shared_out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  (void)row_scales;
+  (void)x_scales;
+  (void)x_global;
+  MOE_TRY(check_config(cfg));
+  MOE_TRY(check_dtype(cfg));
+  MOE_TRY(check_ws(*cfg, workspace, workspace_bytes));
+  MOE_TRY(check_weights(*cfg, w));
+  if (!rows || !counts || !offsets || !out_rows) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(rows) || !aligned16(out_rows)) return MOE_ERR_INVALID_ARG;
+  if (cfg->I_shared > 0 && (!x || !shared_out || !aligned16(x) || !aligned16(shared_out)))
+    return MOE_ERR_INVALID_ARG;
+  return do_grouped_mlp(*cfg, *w, rows, x, counts, offsets, out_rows, shared_out, workspace,
+                        static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* out_rows, const int32_t* token_row,
+                       const float* topk_w, const void* shared_out, void* y, void* stream) {
+  MOE_TRY(check_config(cfg));
+  if (!out_rows || !token_row || !topk_w || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out_rows) || !aligned16(y) || (shared_out && !aligned16(shared_out)))
+    return MOE_ERR_INVALID_ARG;
+  return do_combine(*cfg, out_rows, token_row, topk_w, shared_out, y,
+                    static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_workspace_size(const moe_config* cfg, size_t* bytes) {
+  MOE_TRY(check_config(cfg));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = fwd_layout(*cfg).total;
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* w_router,
+                       const float* bias, const void* x, void* y, int32_t xy_on_host,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  MOE_TRY(check_config(cfg));
+  MOE_TRY(check_dtype(cfg));
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign) return MOE_ERR_INVALID_ARG;
+  const FwdLayout F = fwd_layout(*cfg);
+  if (workspace_bytes < F.total) return MOE_ERR_WORKSPACE;
+  MOE_TRY(check_weights(*cfg, w));
+  if (!w_router || !bias || !x || !y || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = *cfg;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* b = static_cast<uint8_t*>(workspace);
+  const size_t xbytes = static_cast<size_t>(c.T) * c.H * 2;
+  const void* xd = x;
+  void* yd = y;
+  if (xy_on_host) {
+    MOE_CUDA(cudaMemcpyAsync(b + F.x, x, xbytes, cudaMemcpyHostToDevice, s));
+    xd = b + F.x;
+    yd = b + F.y;
+  } else if (!aligned16(x) || !aligned16(y)) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  float* logits = reinterpret_cast<float*>(b + F.logits);
+  int32_t* topk_idx = reinterpret_cast<int32_t*>(b + F.topk_idx);
+  float* topk_w = reinterpret_cast<float*>(b + F.topk_w);
+  int32_t* counts = reinterpret_cast<int32_t*>(b + F.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(b + F.offsets);
+  int32_t* row_token = reinterpret_cast<int32_t*>(b + F.row_token);
+  int32_t* token_row = reinterpret_cast<int32_t*>(b + F.token_row);
+  void* rows = b + F.rows;
+  void* out_rows = b + F.out_rows;
+  void* shared_out = c.I_shared > 0 ? b + F.shared_out : nullptr;
+  MOE_TRY(do_route(c, xd, w_router, bias, nullptr, logits, topk_idx, topk_w, workspace, s));
+  MOE_TRY(do_permute(c, topk_idx, xd, counts, offsets, row_token, token_row, rows, workspace, s));
+  MOE_TRY(do_grouped_mlp(c, *w, rows, xd, counts, offsets, out_rows, shared_out, workspace, s));
+  MOE_TRY(do_combine(c, out_rows, token_row, topk_w, shared_out, yd, s));
+  if (xy_on_host) MOE_CUDA(cudaMemcpyAsync(y, yd, xbytes, cudaMemcpyDeviceToHost, s));
+  return MOE_OK;
+}
+
+moe_status moe_get_device_status(void* workspace, int32_t* device_status, void* stream) {
+  if (!workspace || !device_status) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  MOE_CUDA(cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, s));
+  MOE_CUDA(cudaStreamSynchronize(s));
+  MOE_CUDA(cudaMemsetAsync(workspace, 0, 4, s));
+  MOE_CUDA(cudaStreamSynchronize(s));
+  *device_status = v;
+  return MOE_OK;
+}
+
+}  // extern "C"

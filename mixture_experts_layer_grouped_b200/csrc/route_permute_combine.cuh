@@ -1,0 +1,317 @@
+// Memory-bound steps of the layer: grouped top-k selection, the permute into
+// padded expert-major order (histogram, scan, stable ranks, row gather) and
+// the gate-weighted combine.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kPermTile = 256;  // (t, j) entries per histogram / rank tile
+
+// ---------------------------------------------------------------------------
+// Selection: one warp per token.
+// s = sigmoid(logit), b = s + bias; group score = sum of the two largest b in
+// each contiguous group of E/G experts; keep the topk_group best groups; pick
+// the top_k largest b among their experts (ties to the lower index, listed by
+// b descending); gate_j = s_j / sum_j s_j * rsf.
+// (TransformerEngine PR "DeepSeekV3Layer", Description, DeepSeekV3MoE bullet.)
+// ---------------------------------------------------------------------------
+constexpr int kSelMaxPerLane = 32;  // E <= 1024
+constexpr int kSelWarps = 4;
+
+struct SelArgs {
+  const float* logits;  // [T, E]
+  const float* bias;    // [E]
+  int32_t* topk_idx;    // [T, k]
+  float* topk_w;        // [T, k]
+  int T, E, G, g, k;
+  float rsf;
+};
+
+// Warp arg-max of (v, i): larger v wins, ties to the smaller i.
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+    if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
+  }
+}
+
+template <int PER>
+__global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(SelArgs a) {
+  __shared__ float sb[kSelWarps][kSelMaxPerLane * 32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kSelWarps + w;
+  if (t >= a.T) return;
+  const int gs = a.E / a.G;
+  const float* lg = a.logits + static_cast<int64_t>(t) * a.E;
+
+  float s[PER], b[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    if (e < a.E) {
+      const float l = lg[e];
+      s[i] = 1.0f / (1.0f + expf(-l));
+      b[i] = s[i] + a.bias[e];
+      sb[w][e] = b[i];
+    } else {
+      s[i] = 0.f;
+      b[i] = -INFINITY;
+    }
+  }
+  __syncwarp();
+  // group scores (lane q handles group q)
+  float gscore = -INFINITY;
+  if (lane < a.G) {
+    float m1 = -INFINITY, m2 = -INFINITY;
+    for (int e = lane * gs; e < (lane + 1) * gs; ++e) {
+      const float v = sb[w][e];
+      if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
+    }
+    gscore = m1 + m2;
+  }
+  // keep the best g groups
+  uint32_t keep = 0;
+  float gv = gscore;
+  for (int r = 0; r < a.g; ++r) {
+    float v = gv;
+    int i = (lane < a.G) ? lane : 1 << 30;
+    warp_argmax(v, i);
+    keep |= 1u << i;
+    if (lane == i) gv = -INFINITY;
+  }
+  // eligible keys
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    if (e >= a.E || !((keep >> (e / gs)) & 1u)) b[i] = -INFINITY;
+  }
+  float sel_s = 0.f;
+  int sel_e = 0;
+  float ssum = 0.f;
+  for (int r = 0; r < a.k; ++r) {
+    float v = -INFINITY;
+    int idx = 1 << 30;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane + 32 * i;
+      if (b[i] > v || (b[i] == v && e < idx)) { v = b[i]; idx = e; }
+    }
+    warp_argmax(v, idx);
+    // the owner lane removes it and broadcasts s
+    float sv = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (lane + 32 * i == idx) { sv = s[i]; b[i] = -INFINITY; }
+    sv = __shfl_sync(0xffffffffu, sv, idx & 31);
+    ssum += sv;
+    if (lane == r) { sel_s = sv; sel_e = idx; }
+  }
+  if (lane < a.k) {
+    a.topk_idx[static_cast<int64_t>(t) * a.k + lane] = sel_e;
+    a.topk_w[static_cast<int64_t>(t) * a.k + lane] = sel_s / ssum * a.rsf;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Permute.
+//   hist:  per tile of kPermTile entries, per-expert counts;
+//   scan:  per-expert running bases across tiles, counts, padded offsets,
+//          -1 for pad rows and rows past the last segment;
+//   rank:  stable slot of every (t, j) (ascending t inside each expert);
+//   gather: dst[r] = src[row_token[r]] or zeros.
+// (TransformerEngine PR "DeepSeekV3Layer", Performance, "NCCL EP local
+//  permute": expert-major staging buffer with zero-filled padding.)
+// ---------------------------------------------------------------------------
+struct PermArgs {
+  const int32_t* topk_idx;  // [T*k]
+  int32_t* hist;            // [ntiles, E] workspace
+  int32_t* counts;          // [E]
+  int32_t* offsets;         // [E+1]
+  int32_t* row_token;       // [r_cap]
+  int32_t* token_row;       // [T*k]
+  int32_t* status;
+  int n, k, E, P, r_cap, ntiles;
+};
+
+__global__ void __launch_bounds__(256) permute_hist_kernel(PermArgs a) {
+  extern __shared__ int32_t h[];
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) h[e] = 0;
+  __syncthreads();
+  const int base = blockIdx.x * kPermTile;
+  for (int i = threadIdx.x; i < kPermTile; i += blockDim.x) {
+    const int f = base + i;
+    if (f < a.n) {
+      const int e = a.topk_idx[f];
+      if (e >= 0 && e < a.E) atomicAdd(&h[e], 1);
+      else set_status(a.status, MOE_ERR_CAPACITY);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+    a.hist[static_cast<int64_t>(blockIdx.x) * a.E + e] = h[e];
+}
+
+// One block of 1024 threads; thread e owns expert e.
+__global__ void __launch_bounds__(1024) permute_scan_kernel(PermArgs a) {
+  __shared__ int32_t warp_sums[32];
+  const int e = threadIdx.x;
+  int cnt = 0;
+  if (e < a.E) {
+    for (int b = 0; b < a.ntiles; ++b) {
+      int32_t* p = a.hist + static_cast<int64_t>(b) * a.E + e;
+      const int v = *p;
+      *p = cnt;  // becomes the tile's base rank for this expert
+      cnt += v;
+    }
+    a.counts[e] = cnt;
+  }
+  const int padded = (e < a.E) ? (cnt + a.P - 1) / a.P * a.P : 0;
+  // block exclusive scan of padded
+  const int lane = e & 31, w = e >> 5;
+  int incl = padded;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int ws = warp_sums[lane];
+    int wi = ws;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += v;
+    }
+    warp_sums[lane] = wi - ws;
+  }
+  __syncthreads();
+  const int off = warp_sums[w] + incl - padded;
+  if (e < a.E) {
+    a.offsets[e] = off;
+    for (int r = off + cnt; r < off + padded; ++r) a.row_token[r] = -1;
+  }
+  if (e == a.E - 1) a.offsets[a.E] = off + padded;
+  __syncthreads();
+  // rows past the last segment
+  const int total = (a.E > 0) ? a.offsets[a.E] : 0;
+  for (int r = total + e; r < a.r_cap; r += blockDim.x) a.row_token[r] = -1;
+}
+
+// One warp per tile, walking its entries in order.
+__global__ void __launch_bounds__(32) permute_rank_kernel(PermArgs a) {
+  extern __shared__ int32_t run[];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < a.E; e += 32) run[e] = a.hist[static_cast<int64_t>(blockIdx.x) * a.E + e];
+  __syncwarp();
+  const int base = blockIdx.x * kPermTile;
+  for (int c = 0; c < kPermTile; c += 32) {
+    const int f = base + c + lane;
+    int e = -1;
+    if (f < a.n) {
+      e = a.topk_idx[f];
+      if (e < 0 || e >= a.E) e = -1;
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int slot = a.offsets[e] + run[e] + rank;
+      a.token_row[f] = slot;
+      a.row_token[slot] = f / a.k;
+    } else if (f < a.n) {
+      a.token_row[f] = -1;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// Row gather: one warp per destination row, 16-byte vectors.
+struct GatherArgs {
+  const uint8_t* src;     // [T, row_bytes]
+  uint8_t* dst;           // [r_cap, row_bytes]
+  const int32_t* row_token;
+  const int32_t* offsets; // offsets[E] = rows in use
+  int E, row_bytes;       // row_bytes % 16 == 0
+};
+
+__global__ void __launch_bounds__(256) permute_gather_kernel(GatherArgs a) {
+  const int rows = a.offsets[a.E];
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int vecs = a.row_bytes >> 4;
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int t = a.row_token[r];
+    uint4* d = reinterpret_cast<uint4*>(a.dst + static_cast<int64_t>(r) * a.row_bytes);
+    if (t >= 0) {
+      const uint4* s = reinterpret_cast<const uint4*>(a.src + static_cast<int64_t>(t) * a.row_bytes);
+      for (int v = threadIdx.x & 31; v < vecs; v += 32) d[v] = __ldg(s + v);
+    } else {
+      for (int v = threadIdx.x & 31; v < vecs; v += 32) d[v] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Combine: y[t] = bf16(sum_j w[t,j] * out_rows[token_row[t*k+j]] + shared[t]),
+// fp32 accumulation in j order.  One warp per token, 8 bf16 per lane-vector.
+// ---------------------------------------------------------------------------
+struct CombineArgs {
+  const __nv_bfloat16* out_rows;  // [r_cap, H]
+  const int32_t* token_row;       // [T*k]
+  const float* topk_w;            // [T*k]
+  const __nv_bfloat16* shared;    // [T, H] or null
+  __nv_bfloat16* y;               // [T, H]
+  int T, H, k;
+};
+
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= a.T) return;
+  const int lane = threadIdx.x & 31;
+  const int vecs = a.H >> 3;
+  int rows[32];
+  float ws[32];
+  for (int j = 0; j < a.k; ++j) {
+    rows[j] = a.token_row[static_cast<int64_t>(t) * a.k + j];
+    ws[j] = a.topk_w[static_cast<int64_t>(t) * a.k + j];
+  }
+  for (int v = lane; v < vecs; v += 32) {
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    for (int j = 0; j < a.k; ++j) {
+      if (rows[j] < 0) continue;  // entry dropped by the permute (bad expert index)
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(a.out_rows + static_cast<int64_t>(rows[j]) * a.H) + v);
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(p2[q]);
+        acc[2 * q] = fmaf(ws[j], f.x, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(ws[j], f.y, acc[2 * q + 1]);
+      }
+    }
+    if (a.shared) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(a.shared + static_cast<int64_t>(t) * a.H) + v);
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(p2[q]);
+        acc[2 * q] += f.x;
+        acc[2 * q + 1] += f.y;
+      }
+    }
+    uint4 o;
+    __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) o2[q] = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+    reinterpret_cast<uint4*>(a.y + static_cast<int64_t>(t) * a.H)[v] = o;
+  }
+}
+
+}  // namespace moe

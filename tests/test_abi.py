@@ -1,0 +1,99 @@
+"""The C ABI on the host: the library loads, exports every function the header
+declares, and rejects bad arguments before launching anything (no GPU needed:
+every case below fails validation before the first CUDA call)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+@pytest.fixture(scope="module")
+def M():
+    import mixture_experts_layer_grouped_b200 as M
+    from mixture_experts_layer_grouped_b200 import build
+    build.build()
+    return M
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_five_steps():
+    names = declared_functions()
+    for f in ("moe_route", "moe_permute", "moe_grouped_mlp", "moe_combine", "moe_forward",
+              "moe_workspace_size", "moe_status_string", "moe_get_device_status"):
+        assert f in names
+
+
+def test_library_exports_every_declared_function(M):
+    lib = M.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", M.binding.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(l.split()[-1] for l in out.splitlines() if l.strip())
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings(M):
+    lib = M.lib()
+    for code in range(7):
+        assert lib.moe_status_string(code)
+    assert lib.moe_status_string(99) == b"unknown status"
+
+
+def _cfg(M, **kw):
+    s = synth.get_config("tiny_bf16_T64").scaled(**kw)
+    return M.config_from_shape(s)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=0), 1), (dict(E=15), 2), (dict(H=200), 2), (dict(I=96), 2),
+    (dict(n_group=5), 2), (dict(top_k=40), 2), (dict(topk_group=5), 2),
+    (dict(pad_multiple=0), 1), (dict(I_shared=100), 2),
+])
+def test_workspace_size_rejects_bad_shapes(M, kw, code):
+    c = _cfg(M, **kw)
+    b, r = ctypes.c_size_t(), ctypes.c_int32()
+    assert M.lib().moe_workspace_size(ctypes.byref(c), ctypes.byref(b), ctypes.byref(r)) == code
+
+
+def test_workspace_size_and_rcap(M):
+    s = synth.get_config("mid_bf16_shared_T2048")
+    nbytes, r_cap = M.moe_workspace_size(M.config_from_shape(s))
+    assert r_cap == s.r_cap == 2048 * 6 + 64 * 7
+    assert nbytes >= r_cap * s.I * 2 + s.T * s.I_shared * 2
+    assert M.moe_forward_workspace_size(M.config_from_shape(s)) > nbytes
+
+
+def test_calls_reject_null_and_small_workspace(M):
+    lib = M.lib()
+    c = _cfg(M)
+    nb, _ = M.moe_workspace_size(c)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    # null topk outputs
+    assert lib.moe_route(ctypes.byref(c), fake, fake, fake, None, fake, None, None, fake, nb,
+                         None) == 1
+    # workspace too small
+    assert lib.moe_route(ctypes.byref(c), fake, fake, fake, None, fake, fake, fake, fake, 16,
+                         None) == 3
+    # misaligned workspace
+    assert lib.moe_permute(ctypes.byref(c), fake, fake, None, fake, fake, fake, fake, fake, None,
+                           ctypes.c_void_p((1 << 20) + 8), nb, None) == 1
+    w = M.MoEWeights()
+    assert lib.moe_grouped_mlp(ctypes.byref(c), ctypes.byref(w), fake, None, fake, None, None,
+                               fake, fake, fake, None, fake, nb, None) == 1
+    assert lib.moe_combine(ctypes.byref(c), None, fake, fake, None, fake, None) == 1
+    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), fake, fake, fake, fake, 0, fake, 16,
+                           None) == 3
