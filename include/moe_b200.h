@@ -135,6 +135,36 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * moe_permute without a workspace.  The pages have no counterpart to this
+ * call; it exists for callers that cannot allocate device memory: code that
+ * runs under an engine or framework that owns every device allocation (a
+ * plugin handed only its input and output buffers), and code that must not
+ * call cudaMalloc because cudaMalloc can synchronize the device.
+ *
+ * Same arguments, outputs and results as moe_permute, minus the workspace.
+ * The histogram scratch is a fixed 1 MiB int32 array compiled into the
+ * library (static __device__ storage, held on every GPU that loads the
+ * library until the process exits), so ceil(T*top_k/256) * E must be at most
+ * 262144; larger shapes return MOE_ERR_WORKSPACE with a message on stderr and
+ * launch nothing.  The call allocates and frees nothing.
+ *
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - Every call on a device shares the one array.  Nothing in it needs to
+ *     start at zero (each call writes every entry before reading it), but
+ *     calls whose kernels overlap on the GPU -- on different streams, or from
+ *     different host threads -- race on it and give wrong results.
+ *   - There is no status word: an expert index outside [0, E) is dropped
+ *     (its token_row is -1), as in moe_permute, but is not reported.
+ */
+moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx,
+                               const void* src_rows, const void* src_scales,
+                               int32_t* counts, int32_t* offsets, int32_t* row_token,
+                               int32_t* token_row, void* dst_rows, void* dst_scales,
+                               void* stream);
+
+/*
  * Grouped expert MLP (DeepSeekV3MoE bullet: GroupedLinear -> ScaledSwiGLU ->
  * GroupedLinear): for every expert e and its rows X_e,
  *   h = bf16(silu(X_e W1_e^T) * (X_e W3_e^T));  out = bf16(h W2_e^T),

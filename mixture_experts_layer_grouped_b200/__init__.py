@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     moe_forward_workspace_size,
     moe_route,
     moe_permute,
+    moe_permute_noalloc,
     moe_grouped_mlp,
     moe_combine,
     moe_forward,

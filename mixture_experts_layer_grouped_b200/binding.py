@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
                           ctypes.c_int),
             "moe_permute": ([_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                              ctypes.c_size_t, _VP], ctypes.c_int),
+            "moe_permute_noalloc": ([_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
+                                    ctypes.c_int),
             "moe_grouped_mlp": ([_CFG, ctypes.POINTER(MoEWeights), _VP, _VP, _VP, _VP, _VP,
                                  _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
             "moe_combine": ([_CFG, _VP, _VP, _VP, _VP, _VP, _VP], ctypes.c_int),
@@ -156,6 +158,17 @@ def moe_permute(cfg, topk_idx, src_rows, counts, offsets, row_token, token_row, 
         _p(_cuda(counts, i32, "counts")), _p(_cuda(offsets, i32, "offsets")),
         _p(_cuda(row_token, i32, "row_token")), _p(_cuda(token_row, i32, "token_row")),
         _p(dst_rows), _p(dst_scales), _p(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_permute_noalloc(cfg, topk_idx, src_rows, counts, offsets, row_token, token_row,
+                        dst_rows, src_scales=None, dst_scales=None, stream=None):
+    """moe_permute without a workspace (scratch built into the library)."""
+    i32 = torch.int32
+    _check("moe_permute_noalloc", lib().moe_permute_noalloc(
+        ctypes.byref(cfg), _p(_cuda(topk_idx, i32, "topk_idx")), _p(src_rows), _p(src_scales),
+        _p(_cuda(counts, i32, "counts")), _p(_cuda(offsets, i32, "offsets")),
+        _p(_cuda(row_token, i32, "row_token")), _p(_cuda(token_row, i32, "token_row")),
+        _p(dst_rows), _p(dst_scales), _stream(stream)))
 
 
 def weights_struct(w: dict) -> MoEWeights:

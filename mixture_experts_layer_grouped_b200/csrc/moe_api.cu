@@ -6,6 +6,7 @@
 
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "grouped_gemm.cuh"
@@ -524,3 +525,100 @@ moe_status moe_get_device_status(void* workspace, int32_t* device_status, void* 
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// moe_permute_noalloc: the permute with its histogram scratch in a fixed
+// device array compiled into the library, for callers that cannot hand the
+// library a workspace.
+// ===========================================================================
+namespace {
+
+// Histogram scratch: one int32 per (tile of 256 (t, j) entries, expert).
+constexpr int kNoAllocScratchInts = 1 << 18;  // 1 MiB per device
+
+}  // namespace
+
+static __device__ __align__(256) int32_t moe_noalloc_permute_scratch[kNoAllocScratchInts];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+int32_t* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  Host code must
+// not use the array's name as a pointer: on the host it is only a stand-in
+// for the symbol.  The address is looked up once per device, with that device
+// current, and cached.
+moe_status noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    MOE_CUDA(cudaGetSymbolAddress(&p, moe_noalloc_permute_scratch));
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx,
+                                          const void* src_rows, const void* src_scales,
+                                          int32_t* counts, int32_t* offsets, int32_t* row_token,
+                                          int32_t* token_row, void* dst_rows, void* dst_scales,
+                                          void* stream) {
+  (void)src_scales;
+  (void)dst_scales;
+  MOE_TRY(check_config(cfg));
+  MOE_TRY(check_dtype(cfg));
+  if (!topk_idx || !src_rows || !counts || !offsets || !row_token || !token_row || !dst_rows)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(src_rows) || !aligned16(dst_rows)) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = *cfg;
+  const StepLayout L = step_layout(c);
+  const int64_t need = static_cast<int64_t>(L.ntiles) * c.E;
+  if (need > kNoAllocScratchInts) {
+    fprintf(stderr,
+            "moe_permute_noalloc: ceil(T*top_k/256)*E = %lld exceeds the built-in scratch of "
+            "%d entries; use moe_permute with a workspace\n",
+            static_cast<long long>(need), kNoAllocScratchInts);
+    return MOE_ERR_WORKSPACE;
+  }
+  int32_t* scratch = nullptr;
+  MOE_TRY(noalloc_scratch(&scratch));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PermArgs a;
+  a.topk_idx = topk_idx;
+  a.hist = scratch;  // every entry read is first written by this call's histogram kernel
+  a.counts = counts;
+  a.offsets = offsets;
+  a.row_token = row_token;
+  a.token_row = token_row;
+  a.status = nullptr;  // bad indices are dropped (token_row = -1) without a status word
+  a.n = c.T * c.top_k;
+  a.k = c.top_k;
+  a.E = c.E;
+  a.P = c.pad_multiple;
+  a.r_cap = L.r_cap;
+  a.ntiles = L.ntiles;
+  const size_t hsm = static_cast<size_t>(c.E) * 4;
+  permute_hist_kernel<<<L.ntiles, 256, hsm, s>>>(a);
+  MOE_TRY(launch_check());
+  permute_scan_kernel<<<1, 1024, 0, s>>>(a);
+  MOE_TRY(launch_check());
+  permute_rank_kernel<<<L.ntiles, 32, hsm, s>>>(a);
+  MOE_TRY(launch_check());
+  GatherArgs g;
+  g.src = static_cast<const uint8_t*>(src_rows);
+  g.dst = static_cast<uint8_t*>(dst_rows);
+  g.row_token = row_token;
+  g.offsets = offsets;
+  g.E = c.E;
+  g.row_bytes = c.H * 2;
+  permute_gather_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
+  return launch_check();
+}
