@@ -81,7 +81,10 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self):
+        return time.time()
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -91,10 +94,12 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, t0=0.0, t1=float("inf")):
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in self.lines:
+        for ts, l in self.lines:
+            if ts < t0 or ts > t1:
+                continue
             parts = [x.strip() for x in l.split(",")]
             if len(parts) < 9:
                 continue
@@ -229,6 +234,7 @@ def run_ours(args, cfg):
             dist.barrier()
         torch.cuda.synchronize()
 
+    clk = ClockSampler(local).__enter__()
     # warm-up (eager), then capture one forward into a CUDA graph
     for _ in range(args.warmup):
         layer.forward(x, out=y)
@@ -243,15 +249,23 @@ def run_ours(args, cfg):
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
 
+    # untimed soak so the clock sampler sees the GPU under this load
+    t_soak = time.time()
+    while time.time() - t_soak < args.soak_s:
+        for _ in range(20):
+            graph.replay()
+        torch.cuda.synchronize()
+
     # ---- timed region: device-resident inputs, graph replay
     barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        ev0.record(stream)
-        for _ in range(args.steps):
-            graph.replay()
-        ev1.record(stream)
-        torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t_timed_end = time.time()
+    clk.__exit__(None, None, None)
     ms = ev0.elapsed_time(ev1) / args.steps
     barrier()
     ms_max = ms
@@ -300,7 +314,8 @@ def run_ours(args, cfg):
         evs[1].record(stream)
         M.moe_permute(c, idx, x, counts, offsets, row_token, token_row, rows, wsp)
         evs[2].record(stream)
-        M.moe_grouped_mlp(c, w, rows, counts, offsets, out_rows, wsp, x=x, shared_out=shared_out)
+        M.moe_grouped_mlp(c, layer.weights, rows, counts, offsets, out_rows, wsp, x=x,
+                          shared_out=shared_out)
         evs[3].record(stream)
         M.moe_combine(c, out_rows, token_row, tw, y, shared_out=shared_out)
         evs[4].record(stream)
@@ -329,7 +344,7 @@ def run_ours(args, cfg):
         cpu = {"value": tps, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
                "sample": f"oracle forward (fp64 numpy) on a {args.ref_tokens}-token sample of "
                          f"the workload, one pass"}
-    clocks = clk.summary()
+    clocks = clk.summary(t_soak, t_timed_end)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
@@ -353,7 +368,8 @@ def run_ours(args, cfg):
                 "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
         "gpu_launches": 9 * args.steps,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
-                   "reasons": clocks["reasons"]},
+                   "reasons": clocks["reasons"], "samples": clocks["samples"]},
+        "tile_n": int(os.environ.get("MOE_GEMM_TILE_N", "256")),
     }
     print(json.dumps(line), flush=True)
 
@@ -367,6 +383,8 @@ def main():
     ap.add_argument("--config", default=BENCH_CONFIG, choices=sorted(synth.CONFIGS))
     ap.add_argument("--ref-tokens", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--soak-s", type=float, default=1.5,
+                    help="untimed graph replays before the timed region (clock sampling)")
     args = ap.parse_args()
     cfg = synth.get_config(args.config)
     if args.impl == "reference":

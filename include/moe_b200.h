@@ -70,11 +70,16 @@ typedef struct moe_config {
 } moe_config;
 
 /*
- * Expert weights as the grouped GEMM consumes them.
- *   bf16 : w1, w3 [E, I, H]; w2 [E, H, I] (K-major: the contraction dim is
- *          contiguous); ws1, ws3 [I_shared, H]; ws2 [H, I_shared].
- *   The *_scales and *_global fields are used by MXFP8/NVFP4 only and are
- *   written by moe_prepare_weights.
+ * Expert weights as the grouped GEMM consumes them, written by
+ * moe_prepare_weights (the caller allocates the buffers, sizes from
+ * moe_prepared_weights_size).
+ *   bf16, tile-major: a matrix of R rows and K columns (R % 128 == 0,
+ *   K % 64 == 0) is stored as 128 x 64 tiles of 16 KB, tile (r/128, k/64) at
+ *   index (r/128)*(K/64) + k/64, row-major inside the tile; element (r, k)
+ *   sits at bf16 offset ((r/128)*(K/64) + k/64)*8192 + (r%128)*64 + k%64.
+ *   w1, w3 hold [E*I rows, H columns] (expert e = rows e*I ..), w2 holds
+ *   [E*H rows, I columns]; ws1, ws3 [I_shared, H]; ws2 [H, I_shared].
+ *   The *_scales and *_global fields are reserved for MXFP8/NVFP4.
  * Shared-expert fields are ignored when I_shared == 0.
  */
 typedef struct moe_weights {
@@ -96,6 +101,31 @@ const char* moe_status_string(moe_status s);
  * rounded up to pad_multiple.  Either output pointer may be NULL.
  */
 moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes, int32_t* r_cap);
+
+/*
+ * Bytes of the prepared weight buffers: routed W1 (and W3) and W2, shared
+ * Ws1 (and Ws3) and Ws2.  Any output pointer may be NULL.
+ */
+moe_status moe_prepared_weights_size(const moe_config* cfg, size_t* w13_bytes,
+                                     size_t* w2_bytes, size_t* shared13_bytes,
+                                     size_t* shared2_bytes);
+
+/*
+ * Weight preparation (the static re-layout of expert weights for the grouped
+ * GEMM kernels; the pages' counterpart is the kernel-specific weight
+ * reordering and shuffling of sglang PR "Mistral Large 3 NVFP4 TRTLLM MoE
+ * support", Gemini summary, "Optimized Weight Handling").
+ *   which == 0: routed experts e_begin .. e_begin+e_count-1; w1, w3 point at
+ *               their row-major bf16 [e_count, I, H] and w2 at [e_count, H, I];
+ *               written into dst->w1/w3/w2 at those experts' place.
+ *   which == 1: the shared expert (e_begin 0, e_count 1); w1, w3 [I_shared, H],
+ *               w2 [H, I_shared] -> dst->ws1/ws3/ws2.
+ * Can be called per expert range so a large layer never needs all its source
+ * weights resident at once.  Source and destination must not overlap.
+ */
+moe_status moe_prepare_weights(const moe_config* cfg, int32_t which, int32_t e_begin,
+                               int32_t e_count, const void* w1, const void* w3, const void* w2,
+                               const moe_weights* dst, void* stream);
 
 /*
  * Router (DeepSeekV3MoE bullet: "fused sigmoid router with aux-loss-free bias

@@ -22,5 +22,8 @@ from .binding import (  # noqa: F401
     moe_combine,
     moe_forward,
     moe_get_device_status,
+    moe_prepared_weights_size,
+    moe_prepare_weights,
+    prepare_weights,
     MoELayer,
 )

@@ -87,6 +87,10 @@ def lib() -> ctypes.CDLL:
             "moe_forward": ([_CFG, ctypes.POINTER(MoEWeights), _VP, _VP, _VP, _VP,
                              ctypes.c_int32, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
             "moe_get_device_status": ([_VP, ctypes.POINTER(ctypes.c_int32), _VP], ctypes.c_int),
+            "moe_prepared_weights_size": ([_CFG] + [ctypes.POINTER(ctypes.c_size_t)] * 4,
+                                          ctypes.c_int),
+            "moe_prepare_weights": ([_CFG, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _VP,
+                                     _VP, _VP, ctypes.POINTER(MoEWeights), _VP], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -176,6 +180,42 @@ def weights_struct(w: dict) -> MoEWeights:
                          for k in _WEIGHT_FIELDS})
 
 
+def moe_prepared_weights_size(cfg: MoEConfig):
+    v = [ctypes.c_size_t() for _ in range(4)]
+    _check("moe_prepared_weights_size", lib().moe_prepared_weights_size(
+        ctypes.byref(cfg), *[ctypes.byref(x) for x in v]))
+    return tuple(x.value for x in v)
+
+
+def moe_prepare_weights(cfg, which, e_begin, e_count, w1, w3, w2, dst, stream=None):
+    """Re-lay bf16 row-major expert weights into the kernels' layout (dst)."""
+    ws = dst if isinstance(dst, MoEWeights) else weights_struct(dst)
+    bf = torch.bfloat16
+    _check("moe_prepare_weights", lib().moe_prepare_weights(
+        ctypes.byref(cfg), which, e_begin, e_count, _p(_cuda(w1, bf, "w1")),
+        _p(_cuda(w3, bf, "w3")), _p(_cuda(w2, bf, "w2")), ctypes.byref(ws), _stream(stream)))
+
+
+def prepare_weights(cfg, raw: dict, stream=None) -> dict:
+    """Allocate the prepared weight buffers (torch) and fill them from the
+    row-major bf16 tensors in ``raw`` (keys w1, w3, w2 and, with a shared
+    expert, ws1, ws3, ws2)."""
+    dev = raw["w1"].device
+    n13, n2, s13, s2 = moe_prepared_weights_size(cfg)
+    out = {"w1": torch.empty(n13 // 2, dtype=torch.bfloat16, device=dev),
+           "w3": torch.empty(n13 // 2, dtype=torch.bfloat16, device=dev),
+           "w2": torch.empty(n2 // 2, dtype=torch.bfloat16, device=dev)}
+    if cfg.I_shared > 0:
+        out["ws1"] = torch.empty(s13 // 2, dtype=torch.bfloat16, device=dev)
+        out["ws3"] = torch.empty(s13 // 2, dtype=torch.bfloat16, device=dev)
+        out["ws2"] = torch.empty(s2 // 2, dtype=torch.bfloat16, device=dev)
+    dst = weights_struct(out)
+    moe_prepare_weights(cfg, 0, 0, cfg.E, raw["w1"], raw["w3"], raw["w2"], dst, stream)
+    if cfg.I_shared > 0:
+        moe_prepare_weights(cfg, 1, 0, 1, raw["ws1"], raw["ws3"], raw["ws2"], dst, stream)
+    return out
+
+
 def moe_grouped_mlp(cfg, weights, rows, counts, offsets, out_rows, workspace, x=None,
                     shared_out=None, row_scales=None, x_scales=None, x_global=None,
                     stream=None):
@@ -218,12 +258,15 @@ class MoELayer:
     """A layer with its weights resident on the device.
 
     ``weights`` maps the moe_weights field names (w1, w3, w2, ws1, ...) to
-    device tensors; ``forward(x)`` runs the whole layer through moe_forward.
+    row-major bf16 device tensors, which are prepared once into the kernels'
+    layout (or to already prepared buffers with ``prepared=True``);
+    ``forward(x)`` runs the whole layer through moe_forward.
     """
 
-    def __init__(self, cfg: MoEConfig, weights: dict, w_router, bias, device="cuda"):
+    def __init__(self, cfg: MoEConfig, weights: dict, w_router, bias, device="cuda",
+                 prepared=False):
         self.cfg = cfg
-        self.weights = dict(weights)
+        self.weights = dict(weights) if prepared else prepare_weights(cfg, weights)
         self._ws_struct = weights_struct(self.weights)
         self.w_router = w_router
         self.bias = bias

@@ -5,11 +5,13 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include "common.cuh"
 #include "grouped_gemm.cuh"
+#include "prepare.cuh"
 #include "route_permute_combine.cuh"
 
 using namespace moe;
@@ -24,9 +26,23 @@ inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a
 // Workspace layout of the step calls.
 // ---------------------------------------------------------------------------
 struct StepLayout {
-  size_t status, hist, h, h_shared, total;
-  int32_t r_cap, ntiles;
+  size_t status, hist, h, h_shared, router_partials, total;
+  int32_t r_cap, ntiles, router_splits;
 };
+
+constexpr int kRouterTileN = 64;
+
+// K splits of the router GEMM: enough tiles for about two per SM, at least
+// four k-steps per split, at most 32 splits.
+int router_splits_of(const moe_config& c) {
+  const int chunks = (c.T + kRouterTileN - 1) / kRouterTileN;
+  const int slabs = (c.E + kBM - 1) / kBM;
+  const int k_tiles = c.H / kBK;
+  int s = (2 * 148 + chunks * slabs - 1) / (chunks * slabs);
+  s = s < k_tiles / 4 ? s : k_tiles / 4;
+  s = s < 32 ? s : 32;
+  return s < 1 ? 1 : s;
+}
 
 int32_t r_cap_of(const moe_config& c) {
   const int64_t P = c.pad_multiple;
@@ -43,6 +59,9 @@ StepLayout step_layout(const moe_config& c) {
   L.hist = o; o = align_up(o + static_cast<size_t>(L.ntiles) * c.E * 4);
   L.h = o; o = align_up(o + static_cast<size_t>(L.r_cap) * c.I * 2);
   L.h_shared = o; o = align_up(o + static_cast<size_t>(c.T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
+  L.router_splits = router_splits_of(c);
+  L.router_partials = o;
+  o = align_up(o + static_cast<size_t>(L.router_splits) * c.T * c.E * 4);
   L.total = o;
   return L;
 }
@@ -156,6 +175,25 @@ moe_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, in
   return MOE_OK;
 }
 
+// 3-D map over a tile-major matrix of `rows` x K bf16: box = one 128 x 64 tile.
+moe_status make_tiled_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MOE_ERR_CUDA;
+  if (reinterpret_cast<uintptr_t>(base) % 16) return MOE_ERR_INVALID_ARG;
+  cuuint64_t dims[3] = {64, 128, (rows / 128) * (K / 64)};
+  cuuint64_t strides[2] = {128, 128 * 128};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fprintf(stderr, "moe_b200: cuTensorMapEncodeTiled (3-D) failed (%d)\n", static_cast<int>(r));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -163,16 +201,28 @@ int sm_count() {
   return n;
 }
 
-template <int MODE>
+template <int MODE, int TILE_N>
 moe_status launch_gemm(const GemmParams& p, int max_units, cudaStream_t s) {
-  using C = GemmCfg<MODE>;
-  MOE_CUDA(cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+  using C = GemmCfg<MODE, TILE_N>;
+  MOE_CUDA(cudaFuncSetAttribute(grouped_gemm_kernel<MODE, TILE_N>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
   int grid = sm_count();
   if (max_units < grid) grid = max_units;
   if (grid < 1) return MOE_OK;
-  grouped_gemm_kernel<MODE><<<grid, kGemmThreads, C::SMEM_BYTES, s>>>(p);
+  grouped_gemm_kernel<MODE, TILE_N><<<grid, kGemmThreads, C::SMEM_BYTES, s>>>(p);
   return launch_check();
+}
+
+// Token chunk of the expert GEMMs: 256 (each weight slab streams once per
+// 256 tokens of its expert; one accumulator set) unless MOE_GEMM_TILE_N=128
+// asks for 128 (double-buffered accumulators, slabs re-streamed per 128).
+int expert_tile_n() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MOE_GEMM_TILE_N");
+    v = (e && atoi(e) == 128) ? 128 : 256;
+  }
+  return v;
 }
 
 int32_t* status_ptr(void* ws) { return static_cast<int32_t*>(ws); }
@@ -183,36 +233,41 @@ int32_t* status_ptr(void* ws) { return static_cast<int32_t*>(ws); }
 moe_status do_route(const moe_config& c, const void* x, const void* w_router, const float* bias,
                     const float* logits_in, float* logits_out, int32_t* topk_idx, float* topk_w,
                     void* ws, cudaStream_t s) {
-  const float* logits = logits_in;
+  SelArgs a;
+  memset(&a, 0, sizeof(a));
   if (!logits_in) {
+    const StepLayout L = step_layout(c);
+    float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.router_partials);
     GemmParams p;
     memset(&p, 0, sizeof(p));
     MOE_TRY(make_map(&p.a0[1], w_router, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.H, c.E,
                      static_cast<uint64_t>(c.H) * 2, kBM));
     MOE_TRY(make_map(&p.b[1], x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.H, c.T,
                      static_cast<uint64_t>(c.H) * 2, kBoxRows));
-    p.a0[0] = p.a0[1];
-    p.a1[0] = p.a1[1] = p.a0[1];
+    p.a0[0] = p.a1[0] = p.a1[1] = p.a0[1];
     p.b[0] = p.b[1];
-    p.g[1].a_rows_per_expert = 0;
-    p.g[1].a_valid_rows = c.E;
-    p.g[1].n_slabs = (c.E + kBM - 1) / kBM;
-    p.g[1].k_tiles = c.H / kBK;
-    p.g[1].out = logits_out;
-    p.g[1].out_ld = c.E;
-    p.g[0] = p.g[1];
-    p.counts = nullptr;
-    p.offsets = nullptr;
+    GemmGroup g;
+    g.a_rows_per_expert = 0;
+    g.a_valid_rows = c.E;
+    g.n_slabs = (c.E + kBM - 1) / kBM;
+    g.k_tiles = c.H / kBK;
+    g.k_splits = L.router_splits;
+    g.out = partials;
+    g.out_ld = c.E;
+    g.split_stride = static_cast<int64_t>(c.T) * c.E;
+    p.g[0] = p.g[1] = g;
     p.E = 0;
     p.dense_rows = c.T;
-    p.tile_n = 64;
     p.status = status_ptr(ws);
-    const int units = ((c.T + 63) / 64) * p.g[1].n_slabs;
-    MOE_TRY(launch_gemm<kRouter>(p, units, s));
-    logits = logits_out;
+    const int units = ((c.T + kRouterTileN - 1) / kRouterTileN) * g.n_slabs * g.k_splits;
+    MOE_TRY((launch_gemm<kRouter, kRouterTileN>(p, units, s)));
+    a.partials = partials;
+    a.n_splits = L.router_splits;
+    a.logits_out = logits_out;
+  } else {
+    a.logits = logits_in;
+    a.n_splits = 0;
   }
-  SelArgs a;
-  a.logits = logits;
   a.bias = bias;
   a.topk_idx = topk_idx;
   a.topk_w = topk_w;
@@ -270,9 +325,10 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
   return launch_check();
 }
 
-moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void* rows,
-                          const void* x, const int32_t* counts, const int32_t* offsets,
-                          void* out_rows, void* shared_out, void* ws, cudaStream_t s) {
+template <int TILE_N>
+moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const void* rows,
+                             const void* x, const int32_t* counts, const int32_t* offsets,
+                             void* out_rows, void* shared_out, void* ws, cudaStream_t s) {
   const StepLayout L = step_layout(c);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   void* h = wsb + L.h;
@@ -280,44 +336,42 @@ moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void*
   const bool sh = c.I_shared > 0;
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
-  const int tile_n = 256;
-  // fc1 + SwiGLU
+  const int max_chunks = c.E + (c.T * c.top_k) / TILE_N + 1;
+  const int dense_chunks = (c.T + TILE_N - 1) / TILE_N;
+  // fc1 + SwiGLU: one 128-feature slab of W1 and of W3 per tile
   {
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    MOE_TRY(make_map(&p.a0[0], w.w1, BF, 2, H, E * I, H * 2, kBM));
-    MOE_TRY(make_map(&p.a1[0], w.w3, BF, 2, H, E * I, H * 2, kBM));
+    MOE_TRY(make_tiled_map(&p.a0[0], w.w1, E * I, H));
+    MOE_TRY(make_tiled_map(&p.a1[0], w.w3, E * I, H));
     MOE_TRY(make_map(&p.b[0], rows, BF, 2, H, L.r_cap, H * 2, kBoxRows));
     if (sh) {
-      MOE_TRY(make_map(&p.a0[1], w.ws1, BF, 2, H, Is, H * 2, kBM));
-      MOE_TRY(make_map(&p.a1[1], w.ws3, BF, 2, H, Is, H * 2, kBM));
+      MOE_TRY(make_tiled_map(&p.a0[1], w.ws1, Is, H));
+      MOE_TRY(make_tiled_map(&p.a1[1], w.ws3, Is, H));
       MOE_TRY(make_map(&p.b[1], x, BF, 2, H, T, H * 2, kBoxRows));
     } else {
       p.a0[1] = p.a0[0];
       p.a1[1] = p.a1[0];
       p.b[1] = p.b[0];
     }
-    p.g[0] = GemmGroup{c.I, c.I, c.I / kBM, c.H / kBK, h, c.I};
-    p.g[1] = GemmGroup{0, c.I_shared, c.I_shared / kBM, c.H / kBK, hs, c.I_shared};
+    p.g[0] = GemmGroup{c.I, c.I, c.I / kBM, c.H / kBK, 1, h, c.I, 0};
+    p.g[1] = GemmGroup{0, c.I_shared, c.I_shared / kBM, c.H / kBK, 1, hs, c.I_shared, 0};
     p.counts = counts;
     p.offsets = offsets;
     p.E = c.E;
     p.dense_rows = sh ? c.T : 0;
-    p.tile_n = tile_n;
     p.status = status_ptr(ws);
-    const int max_chunks = c.E + (c.T * c.top_k) / tile_n + 1;
-    const int units = max_chunks * p.g[0].n_slabs +
-                      (sh ? ((c.T + tile_n - 1) / tile_n) * p.g[1].n_slabs : 0);
-    MOE_TRY(launch_gemm<kFc1>(p, units, s));
+    const int units = max_chunks * p.g[0].n_slabs + (sh ? dense_chunks * p.g[1].n_slabs : 0);
+    MOE_TRY((launch_gemm<kFc1, TILE_N>(p, units, s)));
   }
-  // fc2
+  // fc2: two adjacent 128-row slabs of W2 (256 output features) per tile
   {
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    MOE_TRY(make_map(&p.a0[0], w.w2, BF, 2, I, E * H, I * 2, kBM));
+    MOE_TRY(make_tiled_map(&p.a0[0], w.w2, E * H, I));
     MOE_TRY(make_map(&p.b[0], h, BF, 2, I, L.r_cap, I * 2, kBoxRows));
     if (sh) {
-      MOE_TRY(make_map(&p.a0[1], w.ws2, BF, 2, Is, H, Is * 2, kBM));
+      MOE_TRY(make_tiled_map(&p.a0[1], w.ws2, H, Is));
       MOE_TRY(make_map(&p.b[1], hs, BF, 2, Is, T, Is * 2, kBoxRows));
     } else {
       p.a0[1] = p.a0[0];
@@ -325,20 +379,26 @@ moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void*
     }
     p.a1[0] = p.a0[0];
     p.a1[1] = p.a0[1];
-    p.g[0] = GemmGroup{c.H, c.H, c.H / kBM, c.I / kBK, out_rows, c.H};
-    p.g[1] = GemmGroup{0, c.H, c.H / kBM, (sh ? c.I_shared : 64) / kBK, shared_out, c.H};
+    const int slabs = (c.H + 2 * kBM - 1) / (2 * kBM);
+    p.g[0] = GemmGroup{c.H, c.H, slabs, c.I / kBK, 1, out_rows, c.H, 0};
+    p.g[1] = GemmGroup{0, c.H, slabs, (sh ? c.I_shared : kBK) / kBK, 1, shared_out, c.H, 0};
     p.counts = counts;
     p.offsets = offsets;
     p.E = c.E;
     p.dense_rows = sh ? c.T : 0;
-    p.tile_n = tile_n;
     p.status = status_ptr(ws);
-    const int max_chunks = c.E + (c.T * c.top_k) / tile_n + 1;
-    const int units = max_chunks * p.g[0].n_slabs +
-                      (sh ? ((c.T + tile_n - 1) / tile_n) * p.g[1].n_slabs : 0);
-    MOE_TRY(launch_gemm<kFc2>(p, units, s));
+    const int units = max_chunks * slabs + (sh ? dense_chunks * slabs : 0);
+    MOE_TRY((launch_gemm<kFc2, TILE_N>(p, units, s)));
   }
   return MOE_OK;
+}
+
+moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void* rows,
+                          const void* x, const int32_t* counts, const int32_t* offsets,
+                          void* out_rows, void* shared_out, void* ws, cudaStream_t s) {
+  if (expert_tile_n() == 256)
+    return grouped_mlp_tiles<256>(c, w, rows, x, counts, offsets, out_rows, shared_out, ws, s);
+  return grouped_mlp_tiles<128>(c, w, rows, x, counts, offsets, out_rows, shared_out, ws, s);
 }
 
 moe_status do_combine(const moe_config& c, const void* out_rows, const int32_t* token_row,
@@ -352,7 +412,18 @@ moe_status do_combine(const moe_config& c, const void* out_rows, const int32_t* 
   a.T = c.T;
   a.H = c.H;
   a.k = c.top_k;
-  combine_kernel<<<(c.T + 7) / 8, 256, 0, s>>>(a);
+  const int threads = (c.H / 8) < 256 ? (c.H / 8) : 256;
+  switch (c.top_k) {
+    case 1: combine_kernel<1><<<c.T, threads, 0, s>>>(a); break;
+    case 2: combine_kernel<2><<<c.T, threads, 0, s>>>(a); break;
+    case 3: combine_kernel<3><<<c.T, threads, 0, s>>>(a); break;
+    case 4: combine_kernel<4><<<c.T, threads, 0, s>>>(a); break;
+    case 5: combine_kernel<5><<<c.T, threads, 0, s>>>(a); break;
+    case 6: combine_kernel<6><<<c.T, threads, 0, s>>>(a); break;
+    case 7: combine_kernel<7><<<c.T, threads, 0, s>>>(a); break;
+    case 8: combine_kernel<8><<<c.T, threads, 0, s>>>(a); break;
+    default: combine_kernel<0><<<c.T, threads, 0, s>>>(a); break;
+  }
   return launch_check();
 }
 
@@ -462,6 +533,67 @@ moe_status moe_combine(const moe_config* cfg, const void* out_rows, const int32_
     return MOE_ERR_INVALID_ARG;
   return do_combine(*cfg, out_rows, token_row, topk_w, shared_out, y,
                     static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_prepared_weights_size(const moe_config* cfg, size_t* w13_bytes,
+                                     size_t* w2_bytes, size_t* shared13_bytes,
+                                     size_t* shared2_bytes) {
+  MOE_TRY(check_config(cfg));
+  MOE_TRY(check_dtype(cfg));
+  const size_t H = cfg->H, I = cfg->I, E = cfg->E, Is = cfg->I_shared;
+  if (w13_bytes) *w13_bytes = E * I * H * 2;
+  if (w2_bytes) *w2_bytes = E * H * I * 2;
+  if (shared13_bytes) *shared13_bytes = Is * H * 2;
+  if (shared2_bytes) *shared2_bytes = H * Is * 2;
+  return MOE_OK;
+}
+
+moe_status moe_prepare_weights(const moe_config* cfg, int32_t which, int32_t e_begin,
+                               int32_t e_count, const void* w1, const void* w3, const void* w2,
+                               const moe_weights* dst, void* stream) {
+  MOE_TRY(check_config(cfg));
+  MOE_TRY(check_dtype(cfg));
+  if (!dst || !w1 || !w3 || !w2) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w1) || !aligned16(w3) || !aligned16(w2)) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = *cfg;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int64_t rows13, rows2, k13, k2;
+  void *d1, *d3, *d2;
+  if (which == 0) {
+    if (e_begin < 0 || e_count < 1 || e_begin + e_count > c.E) return MOE_ERR_INVALID_ARG;
+    if (!dst->w1 || !dst->w3 || !dst->w2) return MOE_ERR_INVALID_ARG;
+    rows13 = static_cast<int64_t>(e_count) * c.I;
+    rows2 = static_cast<int64_t>(e_count) * c.H;
+    k13 = c.H;
+    k2 = c.I;
+    // experts are contiguous in the tile-major layout: expert e starts at tile e*(I/128)*(H/64)
+    d1 = static_cast<uint8_t*>(dst->w1) + static_cast<size_t>(e_begin) * c.I * c.H * 2;
+    d3 = static_cast<uint8_t*>(dst->w3) + static_cast<size_t>(e_begin) * c.I * c.H * 2;
+    d2 = static_cast<uint8_t*>(dst->w2) + static_cast<size_t>(e_begin) * c.H * c.I * 2;
+  } else if (which == 1) {
+    if (c.I_shared <= 0 || e_begin != 0 || e_count != 1) return MOE_ERR_INVALID_ARG;
+    if (!dst->ws1 || !dst->ws3 || !dst->ws2) return MOE_ERR_INVALID_ARG;
+    rows13 = c.I_shared;
+    rows2 = c.H;
+    k13 = c.H;
+    k2 = c.I_shared;
+    d1 = dst->ws1;
+    d3 = dst->ws3;
+    d2 = dst->ws2;
+  } else {
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (!aligned16(d1) || !aligned16(d3) || !aligned16(d2)) return MOE_ERR_INVALID_ARG;
+  const int64_t t13 = (rows13 / 128) * (k13 / 64), t2 = (rows2 / 128) * (k2 / 64);
+  tile_rows_kernel<<<static_cast<unsigned>(t13), 256, 0, s>>>(
+      static_cast<const uint4*>(w1), static_cast<uint4*>(d1), rows13, static_cast<int>(k13));
+  MOE_TRY(launch_check());
+  tile_rows_kernel<<<static_cast<unsigned>(t13), 256, 0, s>>>(
+      static_cast<const uint4*>(w3), static_cast<uint4*>(d3), rows13, static_cast<int>(k13));
+  MOE_TRY(launch_check());
+  tile_rows_kernel<<<static_cast<unsigned>(t2), 256, 0, s>>>(
+      static_cast<const uint4*>(w2), static_cast<uint4*>(d2), rows2, static_cast<int>(k2));
+  return launch_check();
 }
 
 moe_status moe_forward_workspace_size(const moe_config* cfg, size_t* bytes) {

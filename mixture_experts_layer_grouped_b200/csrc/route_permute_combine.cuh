@@ -8,6 +8,7 @@
 namespace moe {
 
 constexpr int kPermTile = 256;  // (t, j) entries per histogram / rank tile
+constexpr int kMaxExpertsPerm = 1024;
 
 // ---------------------------------------------------------------------------
 // Selection: one warp per token.
@@ -21,8 +22,11 @@ constexpr int kSelMaxPerLane = 32;  // E <= 1024
 constexpr int kSelWarps = 4;
 
 struct SelArgs {
-  const float* logits;  // [T, E]
-  const float* bias;    // [E]
+  const float* logits;    // [T, E] (when n_splits == 0)
+  const float* partials;  // [n_splits, T, E] router GEMM partial sums (n_splits > 0)
+  float* logits_out;      // [T, E] sum of the partials, in split order (n_splits > 0)
+  int n_splits;
+  const float* bias;      // [E]
   int32_t* topk_idx;    // [T, k]
   float* topk_w;        // [T, k]
   int T, E, G, g, k;
@@ -46,14 +50,23 @@ __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(SelArgs a)
   const int t = blockIdx.x * kSelWarps + w;
   if (t >= a.T) return;
   const int gs = a.E / a.G;
-  const float* lg = a.logits + static_cast<int64_t>(t) * a.E;
+  const int64_t row = static_cast<int64_t>(t) * a.E;
+  const int64_t split_stride = static_cast<int64_t>(a.T) * a.E;
 
   float s[PER], b[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
     if (e < a.E) {
-      const float l = lg[e];
+      float l;
+      if (a.n_splits > 0) {
+        // fixed summation order over the K splits: deterministic logits
+        l = a.partials[row + e];
+        for (int sp = 1; sp < a.n_splits; ++sp) l += a.partials[sp * split_stride + row + e];
+        a.logits_out[row + e] = l;
+      } else {
+        l = a.logits[row + e];
+      }
       s[i] = 1.0f / (1.0f + expf(-l));
       b[i] = s[i] + a.bias[e];
       sb[w][e] = b[i];
@@ -155,23 +168,35 @@ __global__ void __launch_bounds__(256) permute_hist_kernel(PermArgs a) {
     a.hist[static_cast<int64_t>(blockIdx.x) * a.E + e] = h[e];
 }
 
-// One block of 1024 threads; thread e owns expert e.
+// One block of 1024 threads.  Phase 1: a warp per expert turns that expert's
+// column of tile counts into exclusive tile bases (lanes over tiles, shuffle
+// scan).  Phase 2: thread e pads counts[e] and a block scan gives offsets.
 __global__ void __launch_bounds__(1024) permute_scan_kernel(PermArgs a) {
   __shared__ int32_t warp_sums[32];
-  const int e = threadIdx.x;
-  int cnt = 0;
-  if (e < a.E) {
-    for (int b = 0; b < a.ntiles; ++b) {
+  __shared__ int32_t s_cnt[kMaxExpertsPerm];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int e = w; e < a.E; e += 32) {
+    int run = 0;
+    for (int b0 = 0; b0 < a.ntiles; b0 += 32) {
+      const int b = b0 + lane;
       int32_t* p = a.hist + static_cast<int64_t>(b) * a.E + e;
-      const int v = *p;
-      *p = cnt;  // becomes the tile's base rank for this expert
-      cnt += v;
+      const int v = (b < a.ntiles) ? *p : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (b < a.ntiles) *p = run + incl - v;  // the tile's base rank for this expert
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    a.counts[e] = cnt;
+    if (lane == 0) s_cnt[e] = run;
   }
+  __syncthreads();
+  const int e = tid;
+  const int cnt = (e < a.E) ? s_cnt[e] : 0;
+  if (e < a.E) a.counts[e] = cnt;
   const int padded = (e < a.E) ? (cnt + a.P - 1) / a.P * a.P : 0;
-  // block exclusive scan of padded
-  const int lane = e & 31, w = e >> 5;
   int incl = padded;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -181,7 +206,7 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(PermArgs a) {
   if (lane == 31) warp_sums[w] = incl;
   __syncthreads();
   if (w == 0) {
-    int ws = warp_sums[lane];
+    const int ws = warp_sums[lane];
     int wi = ws;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -196,31 +221,44 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(PermArgs a) {
     a.offsets[e] = off;
     for (int r = off + cnt; r < off + padded; ++r) a.row_token[r] = -1;
   }
-  if (e == a.E - 1) a.offsets[a.E] = off + padded;
+  __shared__ int32_t s_total;
+  if (e == a.E - 1) {
+    a.offsets[a.E] = off + padded;
+    s_total = off + padded;
+  }
   __syncthreads();
   // rows past the last segment
-  const int total = (a.E > 0) ? a.offsets[a.E] : 0;
-  for (int r = total + e; r < a.r_cap; r += blockDim.x) a.row_token[r] = -1;
+  for (int r = s_total + e; r < a.r_cap; r += blockDim.x) a.row_token[r] = -1;
 }
 
-// One warp per tile, walking its entries in order.
+// One warp per tile, walking its entries in order.  The tile's indices and
+// the per-expert bases (tile base + segment offset) are loaded up front, so
+// the ordered walk touches shared memory only.
 __global__ void __launch_bounds__(32) permute_rank_kernel(PermArgs a) {
-  extern __shared__ int32_t run[];
+  extern __shared__ int32_t run[];  // [E]: next free slot per expert
   const int lane = threadIdx.x;
-  for (int e = lane; e < a.E; e += 32) run[e] = a.hist[static_cast<int64_t>(blockIdx.x) * a.E + e];
-  __syncwarp();
+  for (int e = lane; e < a.E; e += 32)
+    run[e] = a.offsets[e] + a.hist[static_cast<int64_t>(blockIdx.x) * a.E + e];
   const int base = blockIdx.x * kPermTile;
-  for (int c = 0; c < kPermTile; c += 32) {
-    const int f = base + c + lane;
+  int ev[kPermTile / 32];
+#pragma unroll
+  for (int c = 0; c < kPermTile / 32; ++c) {
+    const int f = base + c * 32 + lane;
     int e = -1;
     if (f < a.n) {
       e = a.topk_idx[f];
       if (e < 0 || e >= a.E) e = -1;
     }
+    ev[c] = e;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < kPermTile / 32; ++c) {
+    const int f = base + c * 32 + lane;
+    const int e = ev[c];
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
     if (e >= 0) {
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int slot = a.offsets[e] + run[e] + rank;
+      const int slot = run[e] + __popc(peers & ((1u << lane) - 1u));
       a.token_row[f] = slot;
       a.row_token[slot] = f / a.k;
     } else if (f < a.n) {
@@ -270,41 +308,57 @@ struct CombineArgs {
   int T, H, k;
 };
 
-__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= a.T) return;
-  const int lane = threadIdx.x & 31;
-  const int vecs = a.H >> 3;
-  int rows[32];
-  float ws[32];
-  for (int j = 0; j < a.k; ++j) {
-    rows[j] = a.token_row[static_cast<int64_t>(t) * a.k + j];
-    ws[j] = a.topk_w[static_cast<int64_t>(t) * a.k + j];
+__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& raw, float w) {
+  const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = __bfloat1622float2(p2[q]);
+    acc[2 * q] = fmaf(w, f.x, acc[2 * q]);
+    acc[2 * q + 1] = fmaf(w, f.y, acc[2 * q + 1]);
   }
-  for (int v = lane; v < vecs; v += 32) {
+}
+
+// One block per token; each thread owns 8 bf16 columns at a time and issues
+// the loads of all K rows before accumulating them in j order.
+template <int K>
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  const int t = blockIdx.x;
+  const int kk = (K > 0) ? K : a.k;
+  int rows[K > 0 ? K : 32];
+  float ws[K > 0 ? K : 32];
+#pragma unroll
+  for (int j = 0; j < (K > 0 ? K : 32); ++j) {
+    if (j < kk) {
+      rows[j] = __ldg(a.token_row + static_cast<int64_t>(t) * kk + j);
+      ws[j] = __ldg(a.topk_w + static_cast<int64_t>(t) * kk + j);
+    }
+  }
+  const int vecs = a.H >> 3;
+  for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int j = 0; j < a.k; ++j) {
-      if (rows[j] < 0) continue;  // entry dropped by the permute (bad expert index)
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(a.out_rows + static_cast<int64_t>(rows[j]) * a.H) + v);
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    if (K > 0) {
+      uint4 raw[K > 0 ? K : 1];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(p2[q]);
-        acc[2 * q] = fmaf(ws[j], f.x, acc[2 * q]);
-        acc[2 * q + 1] = fmaf(ws[j], f.y, acc[2 * q + 1]);
+      for (int j = 0; j < K; ++j)
+        raw[j] = rows[j] >= 0 ? __ldg(reinterpret_cast<const uint4*>(
+                                          a.out_rows + static_cast<int64_t>(rows[j]) * a.H) + v)
+                              : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < K; ++j) acc_bf16x8(acc, raw[j], rows[j] >= 0 ? ws[j] : 0.f);
+    } else {
+      for (int j = 0; j < kk; ++j) {
+        if (rows[j] < 0) continue;  // entry dropped by the permute (bad expert index)
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+                                    a.out_rows + static_cast<int64_t>(rows[j]) * a.H) + v);
+        acc_bf16x8(acc, raw, ws[j]);
       }
     }
     if (a.shared) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(a.shared + static_cast<int64_t>(t) * a.H) + v);
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(p2[q]);
-        acc[2 * q] += f.x;
-        acc[2 * q + 1] += f.y;
-      }
+      const uint4 raw =
+          __ldg(reinterpret_cast<const uint4*>(a.shared + static_cast<int64_t>(t) * a.H) + v);
+      acc_bf16x8(acc, raw, 1.0f);
     }
     uint4 o;
     __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);

@@ -103,7 +103,8 @@ def run_steps(cfg, d, logits_in=None):
     out["out_rows"] = torch.zeros(r_cap, H, dtype=torch.bfloat16, device=dev)
     out["shared_out"] = (torch.empty(T, H, dtype=torch.bfloat16, device=dev)
                          if cfg.I_shared > 0 else None)
-    M.moe_grouped_mlp(c, weights_dict(d), out["rows"], out["counts"], out["offsets"],
+    prepared = M.prepare_weights(c, weights_dict(d))
+    M.moe_grouped_mlp(c, prepared, out["rows"], out["counts"], out["offsets"],
                       out["out_rows"], ws, x=d["x"], shared_out=out["shared_out"])
     out["y"] = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     M.moe_combine(c, out["out_rows"], out["token_row"], out["topk_w"], out["y"],

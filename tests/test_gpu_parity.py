@@ -172,8 +172,8 @@ def test_grouped_mlp(M, name):
     out_rows = torch.zeros(r_cap, cfg.H, dtype=torch.bfloat16, device="cuda")
     shared_out = (torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
                   if cfg.I_shared else None)
-    M.moe_grouped_mlp(c, weights_dict(d), rows, counts, offsets, out_rows, ws, x=d["x"],
-                      shared_out=shared_out)
+    M.moe_grouped_mlp(c, M.prepare_weights(c, weights_dict(d)), rows, counts, offsets, out_rows,
+                      ws, x=d["x"], shared_out=shared_out)
     torch.cuda.synchronize()
     assert M.moe_get_device_status(ws) == 0
     got = f64(out_rows)
@@ -265,3 +265,39 @@ def test_device_status_reports_bad_index(M):
     torch.cuda.synchronize()
     assert M.moe_get_device_status(ws) == 4
     assert M.moe_get_device_status(ws) == 0  # cleared by the read
+
+
+# ---------------------------------------------------------------- weight preparation
+def _tile_major(w, R, K):
+    """The documented tile-major layout of a row-major [R, K] matrix."""
+    return (w.reshape(R // 128, 128, K // 64, 64).permute(0, 2, 1, 3).reshape(-1))
+
+
+@pytest.mark.parametrize("name", ["tiny_bf16_T64", "one_token", "ragged_pad1"])
+def test_prepare_weights_layout(M, name):
+    cfg = _cfg(name)
+    c = M.config_from_shape(cfg)
+    d = gen_device_inputs(cfg)
+    if cfg.I_shared:
+        d.update(zip(("ws1", "ws3", "ws2"), synth.gen_shared_weights(cfg, "cuda")))
+    p = M.prepare_weights(c, weights_dict(d))
+    torch.cuda.synchronize()
+    E, H, I = cfg.E, cfg.H, cfg.I
+    assert torch.equal(p["w1"], _tile_major(d["w1"].reshape(E * I, H), E * I, H))
+    assert torch.equal(p["w3"], _tile_major(d["w3"].reshape(E * I, H), E * I, H))
+    assert torch.equal(p["w2"], _tile_major(d["w2"].reshape(E * H, I), E * H, I))
+    if cfg.I_shared:
+        Is = cfg.I_shared
+        assert torch.equal(p["ws1"], _tile_major(d["ws1"], Is, H))
+        assert torch.equal(p["ws2"], _tile_major(d["ws2"], H, Is))
+    # preparing one expert range at a time gives the same buffers
+    q = {k: torch.zeros_like(v) for k, v in p.items()}
+    dst = M.binding.weights_struct(q)
+    for e0 in range(0, E, 3):
+        n = min(3, E - e0)
+        M.moe_prepare_weights(c, 0, e0, n, d["w1"][e0:e0 + n].contiguous(),
+                              d["w3"][e0:e0 + n].contiguous(), d["w2"][e0:e0 + n].contiguous(),
+                              dst)
+    torch.cuda.synchronize()
+    for k in ("w1", "w3", "w2"):
+        assert torch.equal(q[k], p[k])
