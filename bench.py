@@ -191,10 +191,13 @@ def run_reference(args, cfg):
 # our arm
 # ---------------------------------------------------------------------------
 
+WEIGHT_BYTES = {"bf16": 2.0, "mxfp8": 1.0 + 1.0 / 32}  # per element, scales included
+
+
 def grouped_mlp_algorithmic(cfg, touched):
     """Bytes and FLOPs the grouped MLP call cannot avoid: every touched routed
     expert's and the shared expert's weights read once; 6*H*I per row."""
-    wbytes = 2 * 3 * cfg.H * (touched * cfg.I + cfg.I_shared)
+    wbytes = int(WEIGHT_BYTES[cfg.dtype] * 3 * cfg.H * (touched * cfg.I + cfg.I_shared))
     flops = 6 * cfg.H * (cfg.T * cfg.top_k * cfg.I + cfg.T * cfg.I_shared)
     return wbytes, flops
 
@@ -302,23 +305,34 @@ def run_ours(args, cfg):
     tw = torch.empty(cfg.T, cfg.top_k, dtype=torch.float32, device=dev)
     counts, offsets = torch.empty(cfg.E, **i32), torch.empty(cfg.E + 1, **i32)
     row_token, token_row = torch.empty(r_cap, **i32), torch.empty(cfg.T * cfg.top_k, **i32)
-    rows = torch.empty(r_cap, cfg.H, dtype=torch.bfloat16, device=dev)
+    mx = cfg.dtype == "mxfp8"
+    rows = torch.empty(r_cap, cfg.H, dtype=torch.uint8 if mx else torch.bfloat16, device=dev)
+    xc = xs = rows_sf = None
+    if mx:
+        xc = torch.empty(cfg.T, cfg.H, dtype=torch.uint8, device=dev)
+        xs = torch.zeros(M.scale_bytes(cfg.T, cfg.H), dtype=torch.uint8, device=dev)
+        rows_sf = torch.zeros(M.scale_bytes(r_cap, cfg.H), dtype=torch.uint8, device=dev)
     out_rows = torch.empty(r_cap, cfg.H, dtype=torch.bfloat16, device=dev)
     shared_out = (torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
                   if cfg.I_shared else None)
-    steps_ms = {"route": [], "permute": [], "grouped_mlp": [], "combine": []}
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    steps_ms = {"route": [], "quantize": [], "permute": [], "grouped_mlp": [], "combine": []}
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     for it in range(args.warmup + args.steps):
         evs[0].record(stream)
         M.moe_route(c, x, d["w_router"], d["bias"], idx, tw, wsp, logits_out=logits)
         evs[1].record(stream)
-        M.moe_permute(c, idx, x, counts, offsets, row_token, token_row, rows, wsp)
+        if mx:
+            M.moe_quantize("mxfp8", x, xc, xs)
         evs[2].record(stream)
-        M.moe_grouped_mlp(c, layer.weights, rows, counts, offsets, out_rows, wsp, x=x,
-                          shared_out=shared_out)
+        M.moe_permute(c, idx, xc if mx else x, counts, offsets, row_token, token_row, rows, wsp,
+                      src_scales=xs, dst_scales=rows_sf)
         evs[3].record(stream)
-        M.moe_combine(c, out_rows, token_row, tw, y, shared_out=shared_out)
+        M.moe_grouped_mlp(c, layer.weights, rows, counts, offsets, out_rows, wsp,
+                          x=xc if mx else x, shared_out=shared_out, row_scales=rows_sf,
+                          x_scales=xs)
         evs[4].record(stream)
+        M.moe_combine(c, out_rows, token_row, tw, y, shared_out=shared_out)
+        evs[5].record(stream)
         torch.cuda.synchronize()
         if it >= args.warmup:
             for i, k in enumerate(steps_ms):
@@ -327,9 +341,11 @@ def run_ours(args, cfg):
     mlp_ms = statistics.mean(steps_ms["grouped_mlp"])
     wbytes, flops = grouped_mlp_algorithmic(cfg, touched)
     hbm, tf_burst, tf_sus, peak_kind = _peaks()
+    # a contraction takes the peak of its own dtype: fp8 dense = 2 x bf16 (nominal ratio)
+    tf_dtype = tf_burst * (2.0 if mx else 1.0)
     achieved_gbs = wbytes / (mlp_ms * 1e-3) / 1e9
     lb, lf = layer_algorithmic(cfg, touched)
-    roof_ms = max(lb / (hbm * 1e9), lf / (tf_burst * 1e12)) * 1e3
+    roof_ms = max(lb / (hbm * 1e9), lf / (tf_dtype * 1e12)) * 1e3
 
     if dist is not None:
         dist.barrier()
@@ -348,25 +364,27 @@ def run_ours(args, cfg):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3+e8m0 (mxfp8), fp32 acc" if mx else "bf16",
         "data": "synthetic (seeded normal inputs and random-init weights of the workload)",
         "config": dict(_workload(cfg, "inputs larger than L2: %.0f MB of expert weights per step"
-                                 % (2 * 3 * cfg.H * cfg.I * cfg.E / 1e6)),
+                                 % (WEIGHT_BYTES[cfg.dtype] * 3 * cfg.H * cfg.I * cfg.E / 1e6)),
                        launch="CUDA graph of the one-call forward", parallelism=f"replicas{ws_n}"),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
                      "frac": achieved_gbs / hbm, "traffic": None,
                      "kernel": "moe_grouped_mlp (fc1+SwiGLU and fc2 tcgen05 kernels)",
                      "algorithmic_bytes_per_launch": wbytes, "ms_per_launch": mlp_ms,
                      "tensor_tflops": flops / (mlp_ms * 1e-3) / 1e12,
-                     "tensor_frac": flops / (mlp_ms * 1e-3) / 1e12 / tf_burst,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs / bf16_tflops)"},
+                     "tensor_frac": flops / (mlp_ms * 1e-3) / 1e12 / tf_dtype,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs; bf16_tflops"
+                                    + (" x 2 for fp8)" if mx else ")")},
         "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_max,
                            "bytes": lb, "flops": lf, "experts_touched": touched},
         "step_ms": {k: statistics.mean(v) for k, v in steps_ms.items()},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
-        "gpu_launches": 9 * args.steps,
+        "gpu_launches": (10 if mx else 9) * args.steps,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"], "samples": clocks["samples"]},
         "tile_n": int(os.environ.get("MOE_GEMM_TILE_N", "256")),

@@ -58,7 +58,8 @@ typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1, MOE_NVFP4 = 2 } moe_dtype;
  * Supported: 1 <= T; H, I, I_shared multiples of 128; 1 <= E <= 1024;
  * E % n_group == 0 with E/n_group >= 2 and n_group <= 32; 1 <= topk_group <=
  * n_group; 1 <= top_k <= min(32, topk_group*E/n_group); pad_multiple >= 1
- * (MXFP8/NVFP4: pad_multiple == 128).
+ * (MXFP8: pad_multiple == 128).  dtype MOE_NVFP4 is not built yet: the data
+ * calls return MOE_ERR_UNSUPPORTED for it (routing works for every dtype).
  */
 typedef struct moe_config {
   int32_t T, H, I, E;
@@ -79,7 +80,10 @@ typedef struct moe_config {
  *   sits at bf16 offset ((r/128)*(K/64) + k/64)*8192 + (r%128)*64 + k%64.
  *   w1, w3 hold [E*I rows, H columns] (expert e = rows e*I ..), w2 holds
  *   [E*H rows, I columns]; ws1, ws3 [I_shared, H]; ws2 [H, I_shared].
- *   The *_scales and *_global fields are reserved for MXFP8/NVFP4.
+ *   MXFP8: the same tile-major layout over bytes (128 rows x 128 e4m3 codes
+ *   per 16 KB tile), and *_scales hold the e8m0 scales per 32 K elements in
+ *   the MMA scale layout of moe_quantize over the same rows (w1_scales for
+ *   the E*I rows of w1, ...).  The *_global fields are reserved for NVFP4.
  * Shared-expert fields are ignored when I_shared == 0.
  */
 typedef struct moe_weights {
@@ -102,13 +106,31 @@ const char* moe_status_string(moe_status s);
  */
 moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes, int32_t* r_cap);
 
+/* Bytes of each prepared weight buffer (scale buffers are 0 for bf16). */
+typedef struct moe_weight_sizes {
+  size_t w13, w2, ws13, ws2;                       /* codes (w1 and w3 each w13) */
+  size_t w13_scales, w2_scales, ws13_scales, ws2_scales;
+} moe_weight_sizes;
+
+moe_status moe_prepared_weights_size(const moe_config* cfg, moe_weight_sizes* sizes);
+
 /*
- * Bytes of the prepared weight buffers: routed W1 (and W3) and W2, shared
- * Ws1 (and Ws3) and Ws2.  Any output pointer may be NULL.
+ * Block-scaled quantization of a row-major bf16 matrix in [rows, cols]
+ * (TransformerEngine PR "DeepSeekV3Layer", Performance, "MXFP8 quantization":
+ * group_quantize_mxfp8 / quantize_mxfp8_kernel_cast_only).
+ *   dtype MOE_MXFP8: codes [rows, cols] e4m3 (round to nearest even,
+ *   saturating at +-448), one e8m0 scale per 32 consecutive elements of a row:
+ *   2^(floor(log2 amax) - 8), biased exponent clamped to [0, 254], 127 for an
+ *   all-zero block.  cols % 128 == 0.
+ *   Scale layout ("MMA scale layout"): for a matrix with KB = cols/32 blocks
+ *   per row, the scale of (row r, block kb) is at byte
+ *     ((r/128)*(KB/4) + kb/4)*512 + (r%32)*16 + ((r%128)/32)*4 + kb%4,
+ *   so `scales` holds ceil(rows/128)*128*KB bytes.
+ *   dtype MOE_NVFP4: not built yet (MOE_ERR_UNSUPPORTED).  global_scale is
+ *   reserved for it.
  */
-moe_status moe_prepared_weights_size(const moe_config* cfg, size_t* w13_bytes,
-                                     size_t* w2_bytes, size_t* shared13_bytes,
-                                     size_t* shared2_bytes);
+moe_status moe_quantize(int32_t dtype, const void* in, int32_t rows, int32_t cols, void* codes,
+                        void* scales, float* global_scale, void* stream);
 
 /*
  * Weight preparation (the static re-layout of expert weights for the grouped
@@ -153,10 +175,11 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
  *   counts rounded up to pad_multiple.  row_token [r_cap] int32: token of each
  *   row, -1 for pad rows and rows past offsets[E].  token_row [T*top_k] int32:
  *   row of (t, j).  Within a segment tokens ascend.
- *   src_rows: bf16 x [T, H] (BF16), e4m3 codes [T, H] (MXFP8), packed e2m1
- *   codes [T, H/2] (NVFP4).  dst_rows [r_cap, same row bytes]; pad rows zero.
- *   src_scales / dst_scales: block scales (MXFP8/NVFP4) in the MMA scale
- *   layout of moe_quantize, for T and r_cap rows; NULL for BF16.
+ *   src_rows: bf16 x [T, H] (BF16) or e4m3 codes [T, H] (MXFP8, from
+ *   moe_quantize).  dst_rows [r_cap, same row bytes]; pad rows zero.
+ *   src_scales / dst_scales (MXFP8): block scales in the MMA scale layout of
+ *   moe_quantize, for T and r_cap rows; pad rows get zero scale bytes.  NULL
+ *   for BF16.
  */
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx,
                        const void* src_rows, const void* src_scales,
@@ -201,7 +224,9 @@ moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx,
  * and the same for the shared expert on all T tokens of x.
  *   rows [r_cap, H] (as moe_permute's dst_rows), counts/offsets from
  *   moe_permute; x [T, H] in token order (shared expert input; may be NULL
- *   when I_shared == 0).
+ *   when I_shared == 0).  MXFP8: rows and x are e4m3 codes, row_scales /
+ *   x_scales their scales (MMA scale layout), and h is rounded to bf16 and
+ *   quantized to MXFP8 before fc2.  x_global is reserved for NVFP4.
  *   out_rows [r_cap, H] bf16: fc2 output per row (rows of pads untouched).
  *   shared_out [T, H] bf16 or NULL when I_shared == 0.
  * Tensor-core kernels: tcgen05 MMA with TMEM accumulators fed by TMA.

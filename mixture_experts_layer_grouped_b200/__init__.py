@@ -24,6 +24,8 @@ from .binding import (  # noqa: F401
     moe_get_device_status,
     moe_prepared_weights_size,
     moe_prepare_weights,
+    moe_quantize,
+    scale_bytes,
     prepare_weights,
     MoELayer,
 )

@@ -48,6 +48,12 @@ class MoEWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in _WEIGHT_FIELDS]
 
 
+class MoEWeightSizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("w13", "w2", "ws13", "ws2", "w13_scales", "w2_scales", "ws13_scales",
+                 "ws2_scales")]
+
+
 def config_from_shape(s, T=None) -> MoEConfig:
     """MoEConfig from any object with the layer's shape attributes."""
     return MoEConfig(
@@ -87,8 +93,9 @@ def lib() -> ctypes.CDLL:
             "moe_forward": ([_CFG, ctypes.POINTER(MoEWeights), _VP, _VP, _VP, _VP,
                              ctypes.c_int32, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
             "moe_get_device_status": ([_VP, ctypes.POINTER(ctypes.c_int32), _VP], ctypes.c_int),
-            "moe_prepared_weights_size": ([_CFG] + [ctypes.POINTER(ctypes.c_size_t)] * 4,
-                                          ctypes.c_int),
+            "moe_prepared_weights_size": ([_CFG, ctypes.POINTER(MoEWeightSizes)], ctypes.c_int),
+            "moe_quantize": ([ctypes.c_int32, _VP, ctypes.c_int32, ctypes.c_int32, _VP, _VP, _VP,
+                              _VP], ctypes.c_int),
             "moe_prepare_weights": ([_CFG, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _VP,
                                      _VP, _VP, ctypes.POINTER(MoEWeights), _VP], ctypes.c_int),
         }
@@ -180,11 +187,24 @@ def weights_struct(w: dict) -> MoEWeights:
                          for k in _WEIGHT_FIELDS})
 
 
-def moe_prepared_weights_size(cfg: MoEConfig):
-    v = [ctypes.c_size_t() for _ in range(4)]
-    _check("moe_prepared_weights_size", lib().moe_prepared_weights_size(
-        ctypes.byref(cfg), *[ctypes.byref(x) for x in v]))
-    return tuple(x.value for x in v)
+def moe_prepared_weights_size(cfg: MoEConfig) -> dict:
+    v = MoEWeightSizes()
+    _check("moe_prepared_weights_size", lib().moe_prepared_weights_size(ctypes.byref(cfg),
+                                                                        ctypes.byref(v)))
+    return {n: getattr(v, n) for n, _ in MoEWeightSizes._fields_}
+
+
+def moe_quantize(dtype, x, codes, scales, global_scale=None, stream=None):
+    """Block-scaled quantization of a bf16 [rows, cols] tensor (MXFP8)."""
+    rows, cols = x.shape
+    _check("moe_quantize", lib().moe_quantize(
+        DTYPES[dtype] if isinstance(dtype, str) else dtype, _p(_cuda(x, torch.bfloat16, "x")),
+        rows, cols, _p(codes), _p(scales), _p(global_scale), _stream(stream)))
+
+
+def scale_bytes(rows, cols):
+    """Bytes of the MMA-layout scale buffer of a [rows, cols] MXFP8 matrix."""
+    return (rows + 127) // 128 * 128 * (cols // 32)
 
 
 def moe_prepare_weights(cfg, which, e_begin, e_count, w1, w3, w2, dst, stream=None):
@@ -201,14 +221,22 @@ def prepare_weights(cfg, raw: dict, stream=None) -> dict:
     row-major bf16 tensors in ``raw`` (keys w1, w3, w2 and, with a shared
     expert, ws1, ws3, ws2)."""
     dev = raw["w1"].device
-    n13, n2, s13, s2 = moe_prepared_weights_size(cfg)
-    out = {"w1": torch.empty(n13 // 2, dtype=torch.bfloat16, device=dev),
-           "w3": torch.empty(n13 // 2, dtype=torch.bfloat16, device=dev),
-           "w2": torch.empty(n2 // 2, dtype=torch.bfloat16, device=dev)}
+    sz = moe_prepared_weights_size(cfg)
+    u8 = dict(dtype=torch.uint8, device=dev)
+    out = {"w1": torch.empty(sz["w13"], **u8), "w3": torch.empty(sz["w13"], **u8),
+           "w2": torch.empty(sz["w2"], **u8)}
+    if sz["w13_scales"]:
+        out["w1_scales"] = torch.empty(sz["w13_scales"], **u8)
+        out["w3_scales"] = torch.empty(sz["w13_scales"], **u8)
+        out["w2_scales"] = torch.empty(sz["w2_scales"], **u8)
     if cfg.I_shared > 0:
-        out["ws1"] = torch.empty(s13 // 2, dtype=torch.bfloat16, device=dev)
-        out["ws3"] = torch.empty(s13 // 2, dtype=torch.bfloat16, device=dev)
-        out["ws2"] = torch.empty(s2 // 2, dtype=torch.bfloat16, device=dev)
+        out["ws1"] = torch.empty(sz["ws13"], **u8)
+        out["ws3"] = torch.empty(sz["ws13"], **u8)
+        out["ws2"] = torch.empty(sz["ws2"], **u8)
+        if sz["ws13_scales"]:
+            out["ws1_scales"] = torch.empty(sz["ws13_scales"], **u8)
+            out["ws3_scales"] = torch.empty(sz["ws13_scales"], **u8)
+            out["ws2_scales"] = torch.empty(sz["ws2_scales"], **u8)
     dst = weights_struct(out)
     moe_prepare_weights(cfg, 0, 0, cfg.E, raw["w1"], raw["w3"], raw["w2"], dst, stream)
     if cfg.I_shared > 0:

@@ -211,3 +211,93 @@ __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
 }  // namespace moe
+
+namespace moe {
+
+// 1-D bulk copy global -> shared, completing on an mbarrier (16-byte aligned,
+// size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// D[tmem] (+)= A * B^T with MXFP8 operands (e4m3) and e8m0 scales per 32 K
+// elements read from TMEM; sf ids select the byte of the scale word.
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+      "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy one 128 x 4 scale-factor chunk (512 bytes: 32 rows of 16 bytes in
+// shared memory) into TMEM lanes 0-127 (each 32-row group receives the same
+// 32 x 128-bit block), 4 columns.
+__device__ __forceinline__ void tmem_cp_sf_chunk(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Descriptor of a contiguous 512-byte scale chunk: no swizzle, 8-row core
+// matrices of 16-byte rows, 128 bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sf_chunk(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128 >> 4) << 16;  // leading byte offset
+  d |= static_cast<uint64_t>(128 >> 4) << 32;  // stride byte offset: next 8 rows
+  d |= static_cast<uint64_t>(1) << 46;         // descriptor version (sm_100)
+  return d;                                    // layout type 0: no swizzle
+}
+
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: e4m3 A/B, e8m0 scales,
+// both K-major, fp32 D; a_sf_id / b_sf_id pick the scale byte.
+__device__ __forceinline__ uint32_t idesc_mxf8(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4)                                // b_sf_id
+         | (0u << 7) | (0u << 10)                    // A, B: E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (1u << 23)                                // scale format E8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)     // M / 16
+         | (sf_id << 29);                            // a_sf_id
+}
+
+// Offset of block scale (row r, k-block kb) in the MMA scale layout of a
+// matrix with KB k-blocks per row (KB % 4 == 0): 128-row x 4-block chunks of
+// 512 bytes, chunk (r/128, kb/4) at index (r/128)*(KB/4) + kb/4, and inside a
+// chunk byte (r%32)*16 + ((r%128)/32)*4 + kb%4.
+__host__ __device__ __forceinline__ int64_t sf_offset(int64_t r, int kb, int KB) {
+  return ((r >> 7) * (KB >> 2) + (kb >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+}
+
+// MXFP8 scale code of a block from its amax (OCP MX rule: 2^(floor(log2 amax) - 8),
+// biased exponent clamped to [0, 254]; amax 0 -> 127).
+__device__ __forceinline__ uint32_t mx_scale_code(float amax) {
+  if (amax == 0.0f) return 127u;
+  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF);  // biased exponent
+  const int code = e - 8;  // floor(log2 amax) - 8 + 127 for normal amax
+  return static_cast<uint32_t>(code < 0 ? 0 : (code > 254 ? 254 : code));
+}
+
+// 2^(127 - code) as fp32 (code in [0, 253]), the exact reciprocal of the scale.
+__device__ __forceinline__ float mx_inv_scale(uint32_t code) {
+  return __uint_as_float((254u - code) << 23);
+}
+
+// fp32 -> e4m3 code, round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint8_t to_e4m3(float v) {
+  uint16_t r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tmov.b16 %0, t;\n\t}"
+      : "=h"(r)
+      : "f"(0.0f), "f"(v));
+  return static_cast<uint8_t>(r & 0xFF);
+}
+
+}  // namespace moe

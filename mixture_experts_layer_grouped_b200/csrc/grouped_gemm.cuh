@@ -39,6 +39,7 @@ constexpr int kMaxExperts = 1024;
 constexpr int kRingBytes = 192 * 1024;
 
 enum GemmMode { kRouter = 0, kFc1 = 1, kFc2 = 2 };
+enum GemmDtype { kBF16 = 0, kMXF8 = 1 };
 
 struct GemmGroup {
   int32_t a_rows_per_expert;  // rows of each expert's A (row-major or tile-major view)
@@ -56,6 +57,14 @@ struct GemmParams {
   CUtensorMap a1[2];  // [routed, dense]: W3 (fc1 only)
   CUtensorMap b[2];   // [routed, dense]: token rows
   GemmGroup g[2];
+  // block scales (MXFP8) in the 128x4-chunk MMA layout, per group
+  const uint8_t* sfa0[2];   // scales of a0's rows
+  const uint8_t* sfa1[2];   // scales of a1's rows
+  const uint8_t* sfb[2];    // scales of the token rows
+  int32_t kb4[2];           // chunk columns per row chunk (K / 128)
+  // fc1 with quantized output: h codes [rows, ld] and scales (MMA layout, KB = ld/32)
+  uint8_t* q_out[2];
+  uint8_t* q_sf[2];
   const int32_t* counts;   // [E]
   const int32_t* offsets;  // [E+1]
   int32_t E;               // routed experts (0: no routed group)
@@ -69,16 +78,24 @@ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-template <int MODE, int TILE_N>
+template <int MODE, int TILE_N, int DT = kBF16>
 struct GemmCfg {
   static constexpr int NA = (MODE == kRouter) ? 1 : 2;
   static constexpr int A_BYTES = kBM * 128;
   static constexpr int B_BYTES = TILE_N * 128;
-  static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
+  static constexpr int SF_CHUNK = 512;                          // one 128x4 scale chunk
+  // token row chunks of scales: a tile starts at a row that is a multiple of 32
+  // (segments are 128-aligned, tiles TILE_N apart), so it spans at most
+  // ceil((TILE_N + 96) / 128) chunks
+  static constexpr int SFB_CHUNKS = (TILE_N + 96 + 127) / 128;
+  static constexpr int SF_BYTES = (DT == kMXF8) ? (NA + SFB_CHUNKS) * SF_CHUNK : 0;
+  static constexpr int STAGE_BYTES = (NA * A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
   static constexpr int STAGES = (kRingBytes / STAGE_BYTES) > 8 ? 8 : (kRingBytes / STAGE_BYTES);
   static constexpr int ACC_COLS = NA * TILE_N;  // TMEM columns of one tile
-  static constexpr int ACC_BUFS = (2 * ACC_COLS <= 512) ? 2 : 1;
-  static constexpr uint32_t TMEM_COLS = pow2_at_least(ACC_BUFS * ACC_COLS);
+  static constexpr int SF_COLS = (DT == kMXF8) ? 4 * NA + 4 * SFB_CHUNKS : 0;
+  static constexpr int ACC_BUFS = (2 * ACC_COLS + SF_COLS <= 512) ? 2 : 1;
+  static constexpr int SF_TMEM = ACC_BUFS * ACC_COLS;  // first scale-factor column
+  static constexpr uint32_t TMEM_COLS = pow2_at_least(ACC_BUFS * ACC_COLS + SF_COLS);
   static constexpr int SLAB_ROWS = (MODE == kFc2) ? 2 * kBM : kBM;  // features per tile
   static constexpr int STG_BYTES = kEpiWarps * 32 * 32 * 2;  // per warp 32x32 bf16
   static constexpr int BAR_BYTES = 256;
@@ -86,6 +103,7 @@ struct GemmCfg {
       1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES + 4 * (kMaxExperts + 1);
   static_assert(TMEM_COLS <= 512, "TMEM overflow");
   static_assert(SMEM_BYTES <= 232448, "smem overflow");
+  static_assert(STAGE_BYTES % 1024 == 0 || DT != kBF16, "stage alignment");
 };
 
 struct Tile {
@@ -95,7 +113,7 @@ struct Tile {
 template <int MODE, int TILE_N>
 __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const int* prefix,
                                             int units_routed) {
-  using C = GemmCfg<MODE, TILE_N>;
+  using C = GemmCfg<MODE, TILE_N, kBF16>;
   Tile t;
   if (u < units_routed) {
     const int ns = p.g[0].n_slabs;
@@ -136,10 +154,10 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
 // silu(g) = g * sigmoid(g); fast exp and division (well inside bf16 rounding).
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-template <int MODE, int TILE_N>
+template <int MODE, int TILE_N, int DT>
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     const __grid_constant__ GemmParams p) {
-  using C = GemmCfg<MODE, TILE_N>;
+  using C = GemmCfg<MODE, TILE_N, DT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -227,7 +245,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const Tile t = decode_tile<MODE, TILE_N>(u, p, prefix, units_routed);
         const int nbox = (t.n_tok + kBoxRows - 1) / kBoxRows;
-        const uint32_t bytes = C::NA * C::A_BYTES + nbox * kBoxRows * 128;
+        const int nsfb = ((t.row0 & 127) + t.n_tok + 127) / 128;
+        const uint32_t bytes = C::NA * C::A_BYTES + nbox * kBoxRows * 128 +
+                               (DT == kMXF8 ? (C::NA + nsfb) * C::SF_CHUNK : 0);
         for (int kt = t.k_begin; kt < t.k_end; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           uint8_t* sa = ring + stage * C::STAGE_BYTES;
@@ -247,8 +267,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
           }
           uint8_t* sb = sa + C::NA * C::A_BYTES;
           for (int bx = 0; bx < nbox; ++bx)
-            tma_load_2d(sb + bx * kBoxRows * 128, &p.b[t.grp], &full[stage], kt * kBK,
-                        t.row0 + bx * kBoxRows, pol_x);
+            tma_load_2d(sb + bx * kBoxRows * 128, &p.b[t.grp], &full[stage],
+                        kt * (DT == kBF16 ? kBK : 128), t.row0 + bx * kBoxRows, pol_x);
+          if (DT == kMXF8) {
+            // scale chunks: A rows [a_row, +128) (and the second operand), token rows
+            uint8_t* ssf = sb + C::B_BYTES;
+            const int kb4 = p.kb4[t.grp];
+            const int64_t ca = (static_cast<int64_t>(t.a_row) / 128) * kb4 + kt;
+            bulk_load(ssf, p.sfa0[t.grp] + ca * C::SF_CHUNK, C::SF_CHUNK, &full[stage], pol_w);
+            if (MODE == kFc1)
+              bulk_load(ssf + C::SF_CHUNK, p.sfa1[t.grp] + ca * C::SF_CHUNK, C::SF_CHUNK,
+                        &full[stage], pol_w);
+            else if (MODE == kFc2)
+              bulk_load(ssf + C::SF_CHUNK, p.sfa0[t.grp] + (ca + kb4) * C::SF_CHUNK, C::SF_CHUNK,
+                        &full[stage], pol_w);
+            for (int cb = 0; cb < nsfb; ++cb) {
+              const int64_t cbi = (static_cast<int64_t>(t.row0) / 128 + cb) * kb4 + kt;
+              bulk_load(ssf + (C::NA + cb) * C::SF_CHUNK, p.sfb[t.grp] + cbi * C::SF_CHUNK,
+                        C::SF_CHUNK, &full[stage], pol_x);
+            }
+          }
           last_phase[stage] = phase;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
@@ -276,6 +314,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         const Tile t = decode_tile<MODE, TILE_N>(u, p, prefix, units_routed);
         const int n_mma = (t.n_tok + 15) & ~15;
         const uint32_t idesc = idesc_bf16(kBM, n_mma);
+        const int nsfb = ((t.row0 & 127) + t.n_tok + 127) / 128;
+        // token j's scale sits at chunk row (row0 % 128) + j: shift the TMEM base
+        const uint32_t sfb_shift = static_cast<uint32_t>((t.row0 & 127) >> 5);
         const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
@@ -287,12 +328,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
           const uint64_t da0 = sdesc_kmajor_sw128(sa);
           const uint64_t da1 = sdesc_kmajor_sw128(sa + C::A_BYTES);
           const uint64_t db = sdesc_kmajor_sw128(sb);
+          if (DT == kBF16) {
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint32_t accum = (kt > t.k_begin || kk) ? 1u : 0u;
-            // advance 16 bf16 = 32 bytes along K inside the swizzle atom
-            mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
-            if (C::NA == 2) mma_bf16(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t accum = (kt > t.k_begin || kk) ? 1u : 0u;
+              // advance 16 bf16 = 32 bytes along K inside the swizzle atom
+              mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
+              if (C::NA == 2) mma_bf16(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+            }
+          } else {
+            // scale factors of this stage: smem -> TMEM (in order with the MMAs below)
+            const uint32_t ssf = sb + C::B_BYTES;
+            const uint32_t sf_a0 = tmem_base + C::SF_TMEM;
+            const uint32_t sf_a1 = sf_a0 + 4;
+            const uint32_t sf_b = sf_a0 + 4 * C::NA;
+            tmem_cp_sf_chunk(sf_a0, sdesc_sf_chunk(ssf));
+            if (C::NA == 2) tmem_cp_sf_chunk(sf_a1, sdesc_sf_chunk(ssf + C::SF_CHUNK));
+            for (int cb = 0; cb < nsfb; ++cb)
+              tmem_cp_sf_chunk(sf_b + 4 * cb, sdesc_sf_chunk(ssf + (C::NA + cb) * C::SF_CHUNK));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t accum = (kt > t.k_begin || kk) ? 1u : 0u;
+              const uint32_t id = idesc_mxf8(kBM, n_mma, kk);
+              const uint32_t byte = static_cast<uint32_t>(kk) << 30;
+              // advance 32 e4m3 = 32 bytes along K; k-block kk of the scale words
+              const uint32_t sfb = (sf_b + sfb_shift) | byte;
+              mma_mxf8(d0, da0 + 2 * kk, db + 2 * kk, id, sf_a0 | byte, sfb, accum);
+              if (C::NA == 2)
+                mma_mxf8(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, id, sf_a1 | byte, sfb, accum);
+            }
           }
           mma_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -338,6 +402,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
               if (j < rows_here)
                 out[static_cast<int64_t>(t.row0 + c0 + j) * G.out_ld + e] = __uint_as_float(r0[j]);
           }
+          continue;
+        }
+        if (MODE == kFc1 && DT == kMXF8) {
+          // h = bf16(silu(gate) * up), then MXFP8: the 32 features of this warp are
+          // one scale block per token; codes staged [32 tokens][32 bytes].
+          uint8_t* s8 = my_stg;
+          uint8_t* qo = p.q_out[t.grp];
+          uint8_t* qs = p.q_sf[t.grp];
+          const int KBh = static_cast<int>(G.out_ld) / 32;
+          const int kb = f_base / 32;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float hv = __bfloat162float(__float2bfloat16_rn(
+                silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j])));
+            float amax = fabsf(hv);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const uint32_t code = mx_scale_code(amax);
+            s8[j * 32 + lane] = to_e4m3(hv * mx_inv_scale(code));
+            if (lane == 0 && j < rows_here && f_base < G.a_valid_rows)
+              qs[sf_offset(t.row0 + c0 + j, kb, KBh)] = static_cast<uint8_t>(code);
+          }
+          __syncwarp();
+          const uint4* s4q = reinterpret_cast<const uint4*>(my_stg);
+#pragma unroll
+          for (int it = 0; it < 2; ++it) {
+            const int c = it * 32 + lane;
+            const int j = c >> 1, part = c & 1;
+            if (j < rows_here && f_base < G.a_valid_rows)
+              *reinterpret_cast<uint4*>(qo + static_cast<int64_t>(t.row0 + c0 + j) * G.out_ld +
+                                        f_base + part * 16) = s4q[j * 2 + part];
+          }
+          __syncwarp();
           continue;
         }
         // bf16 outputs: stage [32 tokens][32 features] per warp, then 16-byte stores

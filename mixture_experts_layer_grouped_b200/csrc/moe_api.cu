@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "grouped_gemm.cuh"
 #include "prepare.cuh"
+#include "quantize.cuh"
 #include "route_permute_combine.cuh"
 
 using namespace moe;
@@ -21,12 +22,13 @@ namespace {
 constexpr size_t kAlign = 256;
 
 inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+inline int64_t pad128(int64_t v) { return (v + 127) / 128 * 128; }
 
 // ---------------------------------------------------------------------------
 // Workspace layout of the step calls.
 // ---------------------------------------------------------------------------
 struct StepLayout {
-  size_t status, hist, h, h_shared, router_partials, total;
+  size_t status, hist, h, h_sf, h_shared, h_shared_sf, router_partials, total;
   int32_t r_cap, ntiles, router_splits;
 };
 
@@ -57,8 +59,13 @@ StepLayout step_layout(const moe_config& c) {
   size_t o = 0;
   L.status = o; o = align_up(o + 4);
   L.hist = o; o = align_up(o + static_cast<size_t>(L.ntiles) * c.E * 4);
-  L.h = o; o = align_up(o + static_cast<size_t>(L.r_cap) * c.I * 2);
-  L.h_shared = o; o = align_up(o + static_cast<size_t>(c.T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
+  const size_t eb = (c.dtype == MOE_BF16) ? 2 : 1;  // bytes per h element
+  const size_t Is = c.I_shared > 0 ? c.I_shared : 0;
+  const size_t Tp = static_cast<size_t>(pad128(c.T));
+  L.h = o; o = align_up(o + static_cast<size_t>(L.r_cap) * c.I * eb);
+  L.h_sf = o; o = align_up(o + (eb == 1 ? static_cast<size_t>(pad128(L.r_cap)) * c.I / 32 : 0));
+  L.h_shared = o; o = align_up(o + Tp * Is * eb);
+  L.h_shared_sf = o; o = align_up(o + (eb == 1 ? Tp * Is / 32 : 0));
   L.router_splits = router_splits_of(c);
   L.router_partials = o;
   o = align_up(o + static_cast<size_t>(L.router_splits) * c.T * c.E * 4);
@@ -68,8 +75,8 @@ StepLayout step_layout(const moe_config& c) {
 
 struct FwdLayout {
   StepLayout step;
-  size_t logits, topk_idx, topk_w, counts, offsets, row_token, token_row, rows, out_rows,
-      shared_out, x, y, total;
+  size_t logits, topk_idx, topk_w, counts, offsets, row_token, token_row, rows, rows_sf,
+      out_rows, shared_out, x, x_q, x_sf, y, total;
 };
 
 FwdLayout fwd_layout(const moe_config& c) {
@@ -84,10 +91,15 @@ FwdLayout fwd_layout(const moe_config& c) {
   F.offsets = o; o = align_up(o + (E + 1) * 4);
   F.row_token = o; o = align_up(o + R * 4);
   F.token_row = o; o = align_up(o + T * k * 4);
-  F.rows = o; o = align_up(o + R * H * 2);
+  const bool mx = c.dtype == MOE_MXFP8;
+  const size_t Tp = static_cast<size_t>(pad128(c.T));
+  F.rows = o; o = align_up(o + R * H * (mx ? 1 : 2));
+  F.rows_sf = o; o = align_up(o + (mx ? static_cast<size_t>(pad128(R)) * H / 32 : 0));
   F.out_rows = o; o = align_up(o + R * H * 2);
   F.shared_out = o; o = align_up(o + (c.I_shared > 0 ? T * H * 2 : 0));
   F.x = o; o = align_up(o + T * H * 2);
+  F.x_q = o; o = align_up(o + (mx ? T * H : 0));
+  F.x_sf = o; o = align_up(o + (mx ? Tp * H / 32 : 0));
   F.y = o; o = align_up(o + T * H * 2);
   F.total = o;
   return F;
@@ -111,10 +123,15 @@ moe_status check_config(const moe_config* c) {
   return MOE_OK;
 }
 
-// Data paths built so far: bf16.
+// Data paths built so far: bf16 and MXFP8 (which keeps 128-row scale chunks
+// aligned with expert segments: pad_multiple must be 128).
 moe_status check_dtype(const moe_config* c) {
-  return c->dtype == MOE_BF16 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+  if (c->dtype == MOE_BF16) return MOE_OK;
+  if (c->dtype == MOE_MXFP8) return c->pad_multiple == 128 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+  return MOE_ERR_UNSUPPORTED;
 }
+
+inline bool is_mx(const moe_config& c) { return c.dtype == MOE_MXFP8; }
 
 inline moe_status cuda_check(cudaError_t e) {
   if (e == cudaSuccess) return MOE_OK;
@@ -175,16 +192,17 @@ moe_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, in
   return MOE_OK;
 }
 
-// 3-D map over a tile-major matrix of `rows` x K bf16: box = one 128 x 64 tile.
-moe_status make_tiled_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
+// 3-D map over a tile-major matrix of `rows` rows and `k_bytes` bytes per row:
+// tiles of 128 rows x 128 bytes, box = one tile.
+moe_status make_tiled_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t k_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return MOE_ERR_CUDA;
   if (reinterpret_cast<uintptr_t>(base) % 16) return MOE_ERR_INVALID_ARG;
-  cuuint64_t dims[3] = {64, 128, (rows / 128) * (K / 64)};
+  cuuint64_t dims[3] = {128, 128, (rows / 128) * (k_bytes / 128)};
   cuuint64_t strides[2] = {128, 128 * 128};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {128, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -201,15 +219,15 @@ int sm_count() {
   return n;
 }
 
-template <int MODE, int TILE_N>
+template <int MODE, int TILE_N, int DT>
 moe_status launch_gemm(const GemmParams& p, int max_units, cudaStream_t s) {
-  using C = GemmCfg<MODE, TILE_N>;
-  MOE_CUDA(cudaFuncSetAttribute(grouped_gemm_kernel<MODE, TILE_N>,
+  using C = GemmCfg<MODE, TILE_N, DT>;
+  MOE_CUDA(cudaFuncSetAttribute(grouped_gemm_kernel<MODE, TILE_N, DT>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
   int grid = sm_count();
   if (max_units < grid) grid = max_units;
   if (grid < 1) return MOE_OK;
-  grouped_gemm_kernel<MODE, TILE_N><<<grid, kGemmThreads, C::SMEM_BYTES, s>>>(p);
+  grouped_gemm_kernel<MODE, TILE_N, DT><<<grid, kGemmThreads, C::SMEM_BYTES, s>>>(p);
   return launch_check();
 }
 
@@ -260,7 +278,7 @@ moe_status do_route(const moe_config& c, const void* x, const void* w_router, co
     p.dense_rows = c.T;
     p.status = status_ptr(ws);
     const int units = ((c.T + kRouterTileN - 1) / kRouterTileN) * g.n_slabs * g.k_splits;
-    MOE_TRY((launch_gemm<kRouter, kRouterTileN>(p, units, s)));
+    MOE_TRY((launch_gemm<kRouter, kRouterTileN, kBF16>(p, units, s)));
     a.partials = partials;
     a.n_splits = L.router_splits;
     a.logits_out = logits_out;
@@ -290,8 +308,9 @@ moe_status do_route(const moe_config& c, const void* x, const void* w_router, co
 }
 
 moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* src_rows,
-                      int32_t* counts, int32_t* offsets, int32_t* row_token, int32_t* token_row,
-                      void* dst_rows, void* ws, cudaStream_t s) {
+                      const void* src_scales, int32_t* counts, int32_t* offsets,
+                      int32_t* row_token, int32_t* token_row, void* dst_rows, void* dst_scales,
+                      void* ws, cudaStream_t s) {
   const StepLayout L = step_layout(c);
   PermArgs a;
   a.topk_idx = topk_idx;
@@ -314,6 +333,19 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
   MOE_TRY(launch_check());
   permute_rank_kernel<<<L.ntiles, 32, hsm, s>>>(a);
   MOE_TRY(launch_check());
+  if (is_mx(c)) {
+    GatherMxArgs g;
+    g.src_codes = static_cast<const uint8_t*>(src_rows);
+    g.src_scales = static_cast<const uint8_t*>(src_scales);
+    g.dst_codes = static_cast<uint8_t*>(dst_rows);
+    g.dst_scales = static_cast<uint8_t*>(dst_scales);
+    g.row_token = row_token;
+    g.offsets = offsets;
+    g.E = c.E;
+    g.H = c.H;
+    permute_gather_mx_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
+    return launch_check();
+  }
   GatherArgs g;
   g.src = static_cast<const uint8_t*>(src_rows);
   g.dst = static_cast<uint8_t*>(dst_rows);
@@ -325,16 +357,27 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
   return launch_check();
 }
 
-template <int TILE_N>
+// Quantized inputs of the grouped MLP (MXFP8): row scales, token-order x codes
+// and scales for the shared expert.
+struct MlpQuant {
+  const void* row_scales;
+  const void* x_scales;
+};
+
+template <int TILE_N, int DT>
 moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const void* rows,
-                             const void* x, const int32_t* counts, const int32_t* offsets,
-                             void* out_rows, void* shared_out, void* ws, cudaStream_t s) {
+                             const void* x, const MlpQuant& q, const int32_t* counts,
+                             const int32_t* offsets, void* out_rows, void* shared_out, void* ws,
+                             cudaStream_t s) {
   const StepLayout L = step_layout(c);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   void* h = wsb + L.h;
   void* hs = wsb + L.h_shared;
   const bool sh = c.I_shared > 0;
-  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const bool mx = DT == kMXF8;
+  const auto tok_t = mx ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int eb = mx ? 1 : 2;                  // bytes per element of activations / weights
+  const int kstep = mx ? 128 : kBK;           // K elements per k-step
   const uint64_t H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
   const int max_chunks = c.E + (c.T * c.top_k) / TILE_N + 1;
   const int dense_chunks = (c.T + TILE_N - 1) / TILE_N;
@@ -342,37 +385,50 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
   {
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    MOE_TRY(make_tiled_map(&p.a0[0], w.w1, E * I, H));
-    MOE_TRY(make_tiled_map(&p.a1[0], w.w3, E * I, H));
-    MOE_TRY(make_map(&p.b[0], rows, BF, 2, H, L.r_cap, H * 2, kBoxRows));
+    MOE_TRY(make_tiled_map(&p.a0[0], w.w1, E * I, H * eb));
+    MOE_TRY(make_tiled_map(&p.a1[0], w.w3, E * I, H * eb));
+    MOE_TRY(make_map(&p.b[0], rows, tok_t, eb, H, L.r_cap, H * eb, kBoxRows));
     if (sh) {
-      MOE_TRY(make_tiled_map(&p.a0[1], w.ws1, Is, H));
-      MOE_TRY(make_tiled_map(&p.a1[1], w.ws3, Is, H));
-      MOE_TRY(make_map(&p.b[1], x, BF, 2, H, T, H * 2, kBoxRows));
+      MOE_TRY(make_tiled_map(&p.a0[1], w.ws1, Is, H * eb));
+      MOE_TRY(make_tiled_map(&p.a1[1], w.ws3, Is, H * eb));
+      MOE_TRY(make_map(&p.b[1], x, tok_t, eb, H, T, H * eb, kBoxRows));
     } else {
       p.a0[1] = p.a0[0];
       p.a1[1] = p.a1[0];
       p.b[1] = p.b[0];
     }
-    p.g[0] = GemmGroup{c.I, c.I, c.I / kBM, c.H / kBK, 1, h, c.I, 0};
-    p.g[1] = GemmGroup{0, c.I_shared, c.I_shared / kBM, c.H / kBK, 1, hs, c.I_shared, 0};
+    p.g[0] = GemmGroup{c.I, c.I, c.I / kBM, c.H / kstep, 1, h, c.I, 0};
+    p.g[1] = GemmGroup{0, c.I_shared, c.I_shared / kBM, c.H / kstep, 1, hs, c.I_shared, 0};
+    if (mx) {
+      p.sfa0[0] = static_cast<const uint8_t*>(w.w1_scales);
+      p.sfa1[0] = static_cast<const uint8_t*>(w.w3_scales);
+      p.sfb[0] = static_cast<const uint8_t*>(q.row_scales);
+      p.sfa0[1] = static_cast<const uint8_t*>(w.ws1_scales);
+      p.sfa1[1] = static_cast<const uint8_t*>(w.ws3_scales);
+      p.sfb[1] = static_cast<const uint8_t*>(q.x_scales);
+      p.kb4[0] = p.kb4[1] = c.H / 128;
+      p.q_out[0] = static_cast<uint8_t*>(h);
+      p.q_sf[0] = wsb + L.h_sf;
+      p.q_out[1] = static_cast<uint8_t*>(hs);
+      p.q_sf[1] = wsb + L.h_shared_sf;
+    }
     p.counts = counts;
     p.offsets = offsets;
     p.E = c.E;
     p.dense_rows = sh ? c.T : 0;
     p.status = status_ptr(ws);
     const int units = max_chunks * p.g[0].n_slabs + (sh ? dense_chunks * p.g[1].n_slabs : 0);
-    MOE_TRY((launch_gemm<kFc1, TILE_N>(p, units, s)));
+    MOE_TRY((launch_gemm<kFc1, TILE_N, DT>(p, units, s)));
   }
   // fc2: two adjacent 128-row slabs of W2 (256 output features) per tile
   {
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    MOE_TRY(make_tiled_map(&p.a0[0], w.w2, E * H, I));
-    MOE_TRY(make_map(&p.b[0], h, BF, 2, I, L.r_cap, I * 2, kBoxRows));
+    MOE_TRY(make_tiled_map(&p.a0[0], w.w2, E * H, I * eb));
+    MOE_TRY(make_map(&p.b[0], h, tok_t, eb, I, L.r_cap, I * eb, kBoxRows));
     if (sh) {
-      MOE_TRY(make_tiled_map(&p.a0[1], w.ws2, H, Is));
-      MOE_TRY(make_map(&p.b[1], hs, BF, 2, Is, T, Is * 2, kBoxRows));
+      MOE_TRY(make_tiled_map(&p.a0[1], w.ws2, H, Is * eb));
+      MOE_TRY(make_map(&p.b[1], hs, tok_t, eb, Is, T, Is * eb, kBoxRows));
     } else {
       p.a0[1] = p.a0[0];
       p.b[1] = p.b[0];
@@ -380,25 +436,39 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     p.a1[0] = p.a0[0];
     p.a1[1] = p.a0[1];
     const int slabs = (c.H + 2 * kBM - 1) / (2 * kBM);
-    p.g[0] = GemmGroup{c.H, c.H, slabs, c.I / kBK, 1, out_rows, c.H, 0};
-    p.g[1] = GemmGroup{0, c.H, slabs, (sh ? c.I_shared : kBK) / kBK, 1, shared_out, c.H, 0};
+    p.g[0] = GemmGroup{c.H, c.H, slabs, c.I / kstep, 1, out_rows, c.H, 0};
+    p.g[1] = GemmGroup{0, c.H, slabs, (sh ? c.I_shared : kstep) / kstep, 1, shared_out, c.H, 0};
+    if (mx) {
+      p.sfa0[0] = static_cast<const uint8_t*>(w.w2_scales);
+      p.sfb[0] = wsb + L.h_sf;
+      p.sfa0[1] = static_cast<const uint8_t*>(w.ws2_scales);
+      p.sfb[1] = wsb + L.h_shared_sf;
+      p.kb4[0] = c.I / 128;
+      p.kb4[1] = sh ? c.I_shared / 128 : 1;
+    }
     p.counts = counts;
     p.offsets = offsets;
     p.E = c.E;
     p.dense_rows = sh ? c.T : 0;
     p.status = status_ptr(ws);
     const int units = max_chunks * slabs + (sh ? dense_chunks * slabs : 0);
-    MOE_TRY((launch_gemm<kFc2, TILE_N>(p, units, s)));
+    MOE_TRY((launch_gemm<kFc2, TILE_N, DT>(p, units, s)));
   }
   return MOE_OK;
 }
 
 moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void* rows,
-                          const void* x, const int32_t* counts, const int32_t* offsets,
-                          void* out_rows, void* shared_out, void* ws, cudaStream_t s) {
-  if (expert_tile_n() == 256)
-    return grouped_mlp_tiles<256>(c, w, rows, x, counts, offsets, out_rows, shared_out, ws, s);
-  return grouped_mlp_tiles<128>(c, w, rows, x, counts, offsets, out_rows, shared_out, ws, s);
+                          const void* x, const MlpQuant& q, const int32_t* counts,
+                          const int32_t* offsets, void* out_rows, void* shared_out, void* ws,
+                          cudaStream_t s) {
+  if (is_mx(c))
+    return grouped_mlp_tiles<192, kMXF8>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
+                                         ws, s);
+  if (expert_tile_n() == 128)
+    return grouped_mlp_tiles<128, kBF16>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
+                                         ws, s);
+  return grouped_mlp_tiles<256, kBF16>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
+                                       ws, s);
 }
 
 moe_status do_combine(const moe_config& c, const void* out_rows, const int32_t* token_row,
@@ -493,16 +563,17 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
                        const void* src_scales, int32_t* counts, int32_t* offsets,
                        int32_t* row_token, int32_t* token_row, void* dst_rows, void* dst_scales,
                        void* workspace, size_t workspace_bytes, void* stream) {
-  (void)src_scales;
-  (void)dst_scales;
   MOE_TRY(check_config(cfg));
   MOE_TRY(check_dtype(cfg));
   MOE_TRY(check_ws(*cfg, workspace, workspace_bytes));
   if (!topk_idx || !src_rows || !counts || !offsets || !row_token || !token_row || !dst_rows)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(src_rows) || !aligned16(dst_rows)) return MOE_ERR_INVALID_ARG;
-  return do_permute(*cfg, topk_idx, src_rows, counts, offsets, row_token, token_row, dst_rows,
-                    workspace, static_cast<cudaStream_t>(stream));
+  if (is_mx(*cfg) && (!src_scales || !dst_scales || !aligned16(src_scales) ||
+                      !aligned16(dst_scales)))
+    return MOE_ERR_INVALID_ARG;
+  return do_permute(*cfg, topk_idx, src_rows, src_scales, counts, offsets, row_token, token_row,
+                    dst_rows, dst_scales, workspace, static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w, const void* rows,
@@ -510,8 +581,6 @@ moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w, const vo
                            const float* x_global, const int32_t* counts, const int32_t* offsets,
                            void* out_rows, void* shared_out, void* workspace,
                            size_t workspace_bytes, void* stream) {
-  (void)row_scales;
-  (void)x_scales;
   (void)x_global;
   MOE_TRY(check_config(cfg));
   MOE_TRY(check_dtype(cfg));
@@ -521,7 +590,15 @@ moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w, const vo
   if (!aligned16(rows) || !aligned16(out_rows)) return MOE_ERR_INVALID_ARG;
   if (cfg->I_shared > 0 && (!x || !shared_out || !aligned16(x) || !aligned16(shared_out)))
     return MOE_ERR_INVALID_ARG;
-  return do_grouped_mlp(*cfg, *w, rows, x, counts, offsets, out_rows, shared_out, workspace,
+  if (is_mx(*cfg)) {
+    if (!row_scales || !aligned16(row_scales)) return MOE_ERR_INVALID_ARG;
+    if (cfg->I_shared > 0 && (!x_scales || !aligned16(x_scales))) return MOE_ERR_INVALID_ARG;
+    if (!w->w1_scales || !w->w3_scales || !w->w2_scales) return MOE_ERR_INVALID_ARG;
+    if (cfg->I_shared > 0 && (!w->ws1_scales || !w->ws3_scales || !w->ws2_scales))
+      return MOE_ERR_INVALID_ARG;
+  }
+  MlpQuant q{row_scales, x_scales};
+  return do_grouped_mlp(*cfg, *w, rows, x, q, counts, offsets, out_rows, shared_out, workspace,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -535,16 +612,21 @@ moe_status moe_combine(const moe_config* cfg, const void* out_rows, const int32_
                     static_cast<cudaStream_t>(stream));
 }
 
-moe_status moe_prepared_weights_size(const moe_config* cfg, size_t* w13_bytes,
-                                     size_t* w2_bytes, size_t* shared13_bytes,
-                                     size_t* shared2_bytes) {
+moe_status moe_prepared_weights_size(const moe_config* cfg, moe_weight_sizes* sizes) {
   MOE_TRY(check_config(cfg));
   MOE_TRY(check_dtype(cfg));
+  if (!sizes) return MOE_ERR_INVALID_ARG;
   const size_t H = cfg->H, I = cfg->I, E = cfg->E, Is = cfg->I_shared;
-  if (w13_bytes) *w13_bytes = E * I * H * 2;
-  if (w2_bytes) *w2_bytes = E * H * I * 2;
-  if (shared13_bytes) *shared13_bytes = Is * H * 2;
-  if (shared2_bytes) *shared2_bytes = H * Is * 2;
+  const size_t eb = is_mx(*cfg) ? 1 : 2;
+  sizes->w13 = E * I * H * eb;
+  sizes->w2 = E * H * I * eb;
+  sizes->ws13 = Is * H * eb;
+  sizes->ws2 = H * Is * eb;
+  const bool mx = is_mx(*cfg);
+  sizes->w13_scales = mx ? E * I * H / 32 : 0;
+  sizes->w2_scales = mx ? E * H * I / 32 : 0;
+  sizes->ws13_scales = mx ? Is * H / 32 : 0;
+  sizes->ws2_scales = mx ? H * Is / 32 : 0;
   return MOE_OK;
 }
 
@@ -584,6 +666,28 @@ moe_status moe_prepare_weights(const moe_config* cfg, int32_t which, int32_t e_b
     return MOE_ERR_INVALID_ARG;
   }
   if (!aligned16(d1) || !aligned16(d3) || !aligned16(d2)) return MOE_ERR_INVALID_ARG;
+  if (is_mx(c)) {
+    // codes tile-major, scales in the MMA layout; byte offsets of the expert range
+    const size_t off13 = which == 0 ? static_cast<size_t>(e_begin) * c.I * c.H : 0;
+    const size_t off2 = which == 0 ? static_cast<size_t>(e_begin) * c.H * c.I : 0;
+    uint8_t* s1 = static_cast<uint8_t*>(which == 0 ? dst->w1_scales : dst->ws1_scales);
+    uint8_t* s3 = static_cast<uint8_t*>(which == 0 ? dst->w3_scales : dst->ws3_scales);
+    uint8_t* s2 = static_cast<uint8_t*>(which == 0 ? dst->w2_scales : dst->ws2_scales);
+    if (!s1 || !s3 || !s2) return MOE_ERR_INVALID_ARG;
+    uint8_t* c1 = static_cast<uint8_t*>(which == 0 ? dst->w1 : dst->ws1) + off13;
+    uint8_t* c3 = static_cast<uint8_t*>(which == 0 ? dst->w3 : dst->ws3) + off13;
+    uint8_t* c2 = static_cast<uint8_t*>(which == 0 ? dst->w2 : dst->ws2) + off2;
+    const int64_t b13 = rows13 * (k13 / 32), b2 = rows2 * (k2 / 32);
+    quantize_mxfp8_tiles_kernel<<<static_cast<unsigned>((b13 + 255) / 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(w1), c1, s1 + off13 / 32, rows13, static_cast<int>(k13));
+    MOE_TRY(launch_check());
+    quantize_mxfp8_tiles_kernel<<<static_cast<unsigned>((b13 + 255) / 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(w3), c3, s3 + off13 / 32, rows13, static_cast<int>(k13));
+    MOE_TRY(launch_check());
+    quantize_mxfp8_tiles_kernel<<<static_cast<unsigned>((b2 + 255) / 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(w2), c2, s2 + off2 / 32, rows2, static_cast<int>(k2));
+    return launch_check();
+  }
   const int64_t t13 = (rows13 / 128) * (k13 / 64), t2 = (rows2 / 128) * (k2 / 64);
   tile_rows_kernel<<<static_cast<unsigned>(t13), 256, 0, s>>>(
       static_cast<const uint4*>(w1), static_cast<uint4*>(d1), rows13, static_cast<int>(k13));
@@ -593,6 +697,21 @@ moe_status moe_prepare_weights(const moe_config* cfg, int32_t which, int32_t e_b
   MOE_TRY(launch_check());
   tile_rows_kernel<<<static_cast<unsigned>(t2), 256, 0, s>>>(
       static_cast<const uint4*>(w2), static_cast<uint4*>(d2), rows2, static_cast<int>(k2));
+  return launch_check();
+}
+
+moe_status moe_quantize(int32_t dtype, const void* in, int32_t rows, int32_t cols, void* codes,
+                        void* scales, float* global_scale, void* stream) {
+  (void)global_scale;
+  if (dtype != MOE_MXFP8) return dtype == MOE_NVFP4 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (!in || !codes || !scales || rows < 1 || cols < 1) return MOE_ERR_INVALID_ARG;
+  if (cols % 128) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(in) || !aligned16(codes)) return MOE_ERR_INVALID_ARG;
+  const int64_t blocks = static_cast<int64_t>(rows) * (cols / 32);
+  quantize_mxfp8_rows_kernel<<<static_cast<unsigned>((blocks + 255) / 256), 256, 0,
+                               static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(in), static_cast<uint8_t*>(codes),
+      static_cast<uint8_t*>(scales), rows, cols);
   return launch_check();
 }
 
@@ -637,8 +756,17 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   void* out_rows = b + F.out_rows;
   void* shared_out = c.I_shared > 0 ? b + F.shared_out : nullptr;
   MOE_TRY(do_route(c, xd, w_router, bias, nullptr, logits, topk_idx, topk_w, workspace, s));
-  MOE_TRY(do_permute(c, topk_idx, xd, counts, offsets, row_token, token_row, rows, workspace, s));
-  MOE_TRY(do_grouped_mlp(c, *w, rows, xd, counts, offsets, out_rows, shared_out, workspace, s));
+  const void* xq = xd;
+  MlpQuant q{nullptr, nullptr};
+  if (is_mx(c)) {
+    MOE_TRY(moe_quantize(MOE_MXFP8, xd, c.T, c.H, b + F.x_q, b + F.x_sf, nullptr, s));
+    xq = b + F.x_q;
+    q = MlpQuant{b + F.rows_sf, b + F.x_sf};
+  }
+  MOE_TRY(do_permute(c, topk_idx, xq, q.x_scales, counts, offsets, row_token, token_row, rows,
+                     b + F.rows_sf, workspace, s));
+  MOE_TRY(do_grouped_mlp(c, *w, rows, xq, q, counts, offsets, out_rows, shared_out, workspace,
+                         s));
   MOE_TRY(do_combine(c, out_rows, token_row, topk_w, shared_out, yd, s));
   if (xy_on_host) MOE_CUDA(cudaMemcpyAsync(y, yd, xbytes, cudaMemcpyDeviceToHost, s));
   return MOE_OK;
@@ -706,7 +834,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   (void)src_scales;
   (void)dst_scales;
   MOE_TRY(check_config(cfg));
-  MOE_TRY(check_dtype(cfg));
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;  // gathers bf16 rows only
   if (!topk_idx || !src_rows || !counts || !offsets || !row_token || !token_row || !dst_rows)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(src_rows) || !aligned16(dst_rows)) return MOE_ERR_INVALID_ARG;

@@ -283,13 +283,14 @@ def test_prepare_weights_layout(M, name):
     p = M.prepare_weights(c, weights_dict(d))
     torch.cuda.synchronize()
     E, H, I = cfg.E, cfg.H, cfg.I
-    assert torch.equal(p["w1"], _tile_major(d["w1"].reshape(E * I, H), E * I, H))
-    assert torch.equal(p["w3"], _tile_major(d["w3"].reshape(E * I, H), E * I, H))
-    assert torch.equal(p["w2"], _tile_major(d["w2"].reshape(E * H, I), E * H, I))
+    bf = lambda t: t.view(torch.bfloat16)  # prepared buffers are raw bytes
+    assert torch.equal(bf(p["w1"]), _tile_major(d["w1"].reshape(E * I, H), E * I, H))
+    assert torch.equal(bf(p["w3"]), _tile_major(d["w3"].reshape(E * I, H), E * I, H))
+    assert torch.equal(bf(p["w2"]), _tile_major(d["w2"].reshape(E * H, I), E * H, I))
     if cfg.I_shared:
         Is = cfg.I_shared
-        assert torch.equal(p["ws1"], _tile_major(d["ws1"], Is, H))
-        assert torch.equal(p["ws2"], _tile_major(d["ws2"], H, Is))
+        assert torch.equal(bf(p["ws1"]), _tile_major(d["ws1"], Is, H))
+        assert torch.equal(bf(p["ws2"]), _tile_major(d["ws2"], H, Is))
     # preparing one expert range at a time gives the same buffers
     q = {k: torch.zeros_like(v) for k, v in p.items()}
     dst = M.binding.weights_struct(q)
