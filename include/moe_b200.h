@@ -110,6 +110,7 @@ moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes, int32_t* r_c
 typedef struct moe_weight_sizes {
   size_t w13, w2, ws13, ws2;                       /* codes (w1 and w3 each w13) */
   size_t w13_scales, w2_scales, ws13_scales, ws2_scales;
+  size_t w_globals, ws_globals;   /* NVFP4: w13_global and w2_global each; shared */
 } moe_weight_sizes;
 
 moe_status moe_prepared_weights_size(const moe_config* cfg, moe_weight_sizes* sizes);

@@ -51,7 +51,7 @@ class MoEWeights(ctypes.Structure):
 class MoEWeightSizes(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("w13", "w2", "ws13", "ws2", "w13_scales", "w2_scales", "ws13_scales",
-                 "ws2_scales")]
+                 "ws2_scales", "w_globals", "ws_globals")]
 
 
 def config_from_shape(s, T=None) -> MoEConfig:
@@ -202,9 +202,9 @@ def moe_quantize(dtype, x, codes, scales, global_scale=None, stream=None):
         rows, cols, _p(codes), _p(scales), _p(global_scale), _stream(stream)))
 
 
-def scale_bytes(rows, cols):
-    """Bytes of the MMA-layout scale buffer of a [rows, cols] MXFP8 matrix."""
-    return (rows + 127) // 128 * 128 * (cols // 32)
+def scale_bytes(rows, cols, dtype="mxfp8"):
+    """Bytes of the MMA-layout scale buffer of a [rows, cols] block-scaled matrix."""
+    return (rows + 127) // 128 * 128 * (cols // (32 if dtype == "mxfp8" else 16))
 
 
 def moe_prepare_weights(cfg, which, e_begin, e_count, w1, w3, w2, dst, stream=None):
@@ -237,6 +237,12 @@ def prepare_weights(cfg, raw: dict, stream=None) -> dict:
             out["ws1_scales"] = torch.empty(sz["ws13_scales"], **u8)
             out["ws3_scales"] = torch.empty(sz["ws13_scales"], **u8)
             out["ws2_scales"] = torch.empty(sz["ws2_scales"], **u8)
+        if sz["ws_globals"]:
+            out["ws13_global"] = torch.empty(1, dtype=torch.float32, device=dev)
+            out["ws2_global"] = torch.empty(1, dtype=torch.float32, device=dev)
+    if sz["w_globals"]:
+        out["w13_global"] = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+        out["w2_global"] = torch.empty(cfg.E, dtype=torch.float32, device=dev)
     dst = weights_struct(out)
     moe_prepare_weights(cfg, 0, 0, cfg.E, raw["w1"], raw["w3"], raw["w2"], dst, stream)
     if cfg.I_shared > 0:

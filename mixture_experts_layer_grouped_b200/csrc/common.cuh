@@ -301,3 +301,87 @@ __device__ __forceinline__ uint8_t to_e4m3(float v) {
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// D[tmem] (+)= A * B^T with NVFP4 operands (packed e2m1) and ue4m3 scales per
+// 16 K elements read from TMEM (one 32-bit scale word per row per MMA).
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor, kind::mxf4nvf4 block-scaled: e2m1 A/B, ue4m3 scales,
+// K = 64 per MMA, both K-major, fp32 D.
+__device__ __forceinline__ uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10)                      // A, B: E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (0u << 23)                                // scale format UE4M3
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Value of an e4m3 code (bias 7, 3 mantissa bits, subnormals at exponent 0);
+// the codes used here are finite and non-negative.
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  if (e == 0) return static_cast<float>(m) * 0.001953125f;  // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));    // (1 + m/8) * 2^(e-7)
+}
+
+// Two fp32 -> one byte of two e2m1 codes (round to nearest even, saturating
+// at +-6); element `lo` in the low nibble, `hi` in the high nibble.
+__device__ __forceinline__ uint32_t to_e2m1x2(float lo, float hi) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  return static_cast<uint32_t>(r) & 0xFFu;
+}
+
+// NVFP4 global encode scale 2688 / amax (448 * 6), 1 when amax is 0.
+__device__ __forceinline__ float nv_global_scale(float amax) {
+  return amax > 0.0f ? __fdiv_rn(2688.0f, amax) : 1.0f;
+}
+
+// Quantize 16 values of one NVFP4 block with global scale g.  Writes 8 bytes
+// of packed codes and returns the ue4m3 block scale code.  Every step is one
+// IEEE fp32 operation: t = (amax / 6) * g; sb = e4m3(t); r = g / value(sb);
+// q = e2m1(v * r); a zero scale gives an all-zero block.
+__device__ __forceinline__ uint32_t nv_quantize_block16(const float (&v)[16], float g,
+                                                        uint32_t (&packed)[2]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), g);
+  const uint32_t sb = to_e4m3(t) & 0x7Fu;
+  if (sb == 0) {
+    packed[0] = packed[1] = 0u;
+    return 0u;
+  }
+  const float r = __fdiv_rn(g, e4m3_value(sb));
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int i = w * 8 + 2 * b;
+      acc |= to_e2m1x2(__fmul_rn(v[i], r), __fmul_rn(v[i + 1], r)) << (8 * b);
+    }
+    packed[w] = acc;
+  }
+  return sb;
+}
+
+// atomic max of a non-negative float stored as bits
+__device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
+  atomicMax(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));
+}
+
+}  // namespace moe

@@ -39,7 +39,7 @@ constexpr int kMaxExperts = 1024;
 constexpr int kRingBytes = 192 * 1024;
 
 enum GemmMode { kRouter = 0, kFc1 = 1, kFc2 = 2 };
-enum GemmDtype { kBF16 = 0, kMXF8 = 1 };
+enum GemmDtype { kBF16 = 0, kMXF8 = 1, kNVF4 = 2 };
 
 struct GemmGroup {
   int32_t a_rows_per_expert;  // rows of each expert's A (row-major or tile-major view)
@@ -57,11 +57,18 @@ struct GemmParams {
   CUtensorMap a1[2];  // [routed, dense]: W3 (fc1 only)
   CUtensorMap b[2];   // [routed, dense]: token rows
   GemmGroup g[2];
-  // block scales (MXFP8) in the 128x4-chunk MMA layout, per group
+  // block scales (MXFP8 / NVFP4) in the 128x4-chunk MMA layout, per group
   const uint8_t* sfa0[2];   // scales of a0's rows
   const uint8_t* sfa1[2];   // scales of a1's rows
   const uint8_t* sfb[2];    // scales of the token rows
-  int32_t kb4[2];           // chunk columns per row chunk (K / 128)
+  int32_t kb4[2];           // chunk columns per row chunk (K/128 MXFP8, K/64 NVFP4)
+  // NVFP4 global scales: acc * 1 / (ga[e * ga_stride] * gw[e * gw_stride])
+  const float* ga[2];
+  int32_t ga_stride[2];
+  const float* gw[2];
+  int32_t gw_stride[2];
+  float* amax_out[2];       // fc1 NVFP4: per-expert amax of h (atomic max)
+  int32_t amax_stride[2];
   // fc1 with quantized output: h codes [rows, ld] and scales (MMA layout, KB = ld/32)
   uint8_t* q_out[2];
   uint8_t* q_sf[2];
@@ -84,15 +91,16 @@ struct GemmCfg {
   static constexpr int A_BYTES = kBM * 128;
   static constexpr int B_BYTES = TILE_N * 128;
   static constexpr int SF_CHUNK = 512;                          // one 128x4 scale chunk
+  static constexpr int SF_KCH = (DT == kNVF4) ? 4 : 1;          // scale chunks per k-step
   // token row chunks of scales: a tile starts at a row that is a multiple of 32
   // (segments are 128-aligned, tiles TILE_N apart), so it spans at most
   // ceil((TILE_N + 96) / 128) chunks
   static constexpr int SFB_CHUNKS = (TILE_N + 96 + 127) / 128;
-  static constexpr int SF_BYTES = (DT == kMXF8) ? (NA + SFB_CHUNKS) * SF_CHUNK : 0;
+  static constexpr int SF_BYTES = (DT != kBF16) ? (NA + SFB_CHUNKS) * SF_KCH * SF_CHUNK : 0;
   static constexpr int STAGE_BYTES = (NA * A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
   static constexpr int STAGES = (kRingBytes / STAGE_BYTES) > 8 ? 8 : (kRingBytes / STAGE_BYTES);
   static constexpr int ACC_COLS = NA * TILE_N;  // TMEM columns of one tile
-  static constexpr int SF_COLS = (DT == kMXF8) ? 4 * NA + 4 * SFB_CHUNKS : 0;
+  static constexpr int SF_COLS = (DT != kBF16) ? 4 * SF_KCH * (NA + SFB_CHUNKS) : 0;
   static constexpr int ACC_BUFS = (2 * ACC_COLS + SF_COLS <= 512) ? 2 : 1;
   static constexpr int SF_TMEM = ACC_BUFS * ACC_COLS;  // first scale-factor column
   static constexpr uint32_t TMEM_COLS = pow2_at_least(ACC_BUFS * ACC_COLS + SF_COLS);
@@ -107,7 +115,7 @@ struct GemmCfg {
 };
 
 struct Tile {
-  int grp, slab, row0, n_tok, k_begin, k_end, a_row, split;
+  int grp, e, slab, row0, n_tok, k_begin, k_end, a_row, split;
 };
 
 template <int MODE, int TILE_N>
@@ -126,6 +134,7 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
     }
     const int chunk = q - prefix[lo];
     t.grp = 0;
+    t.e = lo;
     t.row0 = __ldg(p.offsets + lo) + chunk * TILE_N;
     t.n_tok = min(TILE_N, __ldg(p.counts + lo) - chunk * TILE_N);
     t.a_row = lo * p.g[0].a_rows_per_expert + t.slab * C::SLAB_ROWS;
@@ -141,6 +150,7 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
     const int chunk = v / ns;
     t.slab = v - chunk * ns;
     t.grp = 1;
+    t.e = 0;
     t.row0 = chunk * TILE_N;
     t.n_tok = min(TILE_N, p.dense_rows - t.row0);
     t.a_row = t.slab * C::SLAB_ROWS;
@@ -247,7 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         const int nbox = (t.n_tok + kBoxRows - 1) / kBoxRows;
         const int nsfb = ((t.row0 & 127) + t.n_tok + 127) / 128;
         const uint32_t bytes = C::NA * C::A_BYTES + nbox * kBoxRows * 128 +
-                               (DT == kMXF8 ? (C::NA + nsfb) * C::SF_CHUNK : 0);
+                               (DT != kBF16 ? (C::NA + nsfb) * C::SF_KCH * C::SF_CHUNK : 0);
         for (int kt = t.k_begin; kt < t.k_end; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           uint8_t* sa = ring + stage * C::STAGE_BYTES;
@@ -269,22 +279,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
           for (int bx = 0; bx < nbox; ++bx)
             tma_load_2d(sb + bx * kBoxRows * 128, &p.b[t.grp], &full[stage],
                         kt * (DT == kBF16 ? kBK : 128), t.row0 + bx * kBoxRows, pol_x);
-          if (DT == kMXF8) {
-            // scale chunks: A rows [a_row, +128) (and the second operand), token rows
+          if (DT != kBF16) {
+            // scale chunks of this k-step (SF_KCH consecutive chunks per 128-row chunk):
+            // A rows [a_row, +128) (and the second operand), then the token row chunks
+            constexpr uint32_t cb_bytes = C::SF_KCH * C::SF_CHUNK;
             uint8_t* ssf = sb + C::B_BYTES;
             const int kb4 = p.kb4[t.grp];
-            const int64_t ca = (static_cast<int64_t>(t.a_row) / 128) * kb4 + kt;
-            bulk_load(ssf, p.sfa0[t.grp] + ca * C::SF_CHUNK, C::SF_CHUNK, &full[stage], pol_w);
+            const int64_t ca = (static_cast<int64_t>(t.a_row) / 128) * kb4 + kt * C::SF_KCH;
+            bulk_load(ssf, p.sfa0[t.grp] + ca * C::SF_CHUNK, cb_bytes, &full[stage], pol_w);
             if (MODE == kFc1)
-              bulk_load(ssf + C::SF_CHUNK, p.sfa1[t.grp] + ca * C::SF_CHUNK, C::SF_CHUNK,
-                        &full[stage], pol_w);
+              bulk_load(ssf + cb_bytes, p.sfa1[t.grp] + ca * C::SF_CHUNK, cb_bytes, &full[stage],
+                        pol_w);
             else if (MODE == kFc2)
-              bulk_load(ssf + C::SF_CHUNK, p.sfa0[t.grp] + (ca + kb4) * C::SF_CHUNK, C::SF_CHUNK,
+              bulk_load(ssf + cb_bytes, p.sfa0[t.grp] + (ca + kb4) * C::SF_CHUNK, cb_bytes,
                         &full[stage], pol_w);
             for (int cb = 0; cb < nsfb; ++cb) {
-              const int64_t cbi = (static_cast<int64_t>(t.row0) / 128 + cb) * kb4 + kt;
-              bulk_load(ssf + (C::NA + cb) * C::SF_CHUNK, p.sfb[t.grp] + cbi * C::SF_CHUNK,
-                        C::SF_CHUNK, &full[stage], pol_x);
+              const int64_t cbi = (static_cast<int64_t>(t.row0) / 128 + cb) * kb4 + kt * C::SF_KCH;
+              bulk_load(ssf + (C::NA + cb) * cb_bytes, p.sfb[t.grp] + cbi * C::SF_CHUNK, cb_bytes,
+                        &full[stage], pol_x);
             }
           }
           last_phase[stage] = phase;
@@ -336,6 +348,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
               mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
               if (C::NA == 2) mma_bf16(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, idesc, accum);
             }
+          } else if (DT == kNVF4) {
+            // scale factors: chunk kk of each operand feeds MMA kk (one 32-bit word
+            // of four 16-element block scales per row); token row chunk cb of MMA kk
+            // sits at sf_b + 4 * (kk * SFB_CHUNKS + cb)
+            constexpr uint32_t cb_bytes = C::SF_KCH * C::SF_CHUNK;
+            const uint32_t ssf = sb + C::B_BYTES;
+            const uint32_t sf_a0 = tmem_base + C::SF_TMEM;
+            const uint32_t sf_a1 = sf_a0 + 4 * C::SF_KCH;
+            const uint32_t sf_b = sf_a0 + 4 * C::SF_KCH * C::NA;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              tmem_cp_sf_chunk(sf_a0 + 4 * kk, sdesc_sf_chunk(ssf + kk * C::SF_CHUNK));
+              if (C::NA == 2)
+                tmem_cp_sf_chunk(sf_a1 + 4 * kk, sdesc_sf_chunk(ssf + cb_bytes + kk * C::SF_CHUNK));
+              for (int cb = 0; cb < nsfb; ++cb)
+                tmem_cp_sf_chunk(sf_b + 4 * (kk * C::SFB_CHUNKS + cb),
+                                 sdesc_sf_chunk(ssf + (C::NA + cb) * cb_bytes + kk * C::SF_CHUNK));
+            }
+            const uint32_t id = idesc_nvf4(kBM, n_mma);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t accum = (kt > t.k_begin || kk) ? 1u : 0u;
+              const uint32_t sfb = sf_b + 4 * kk * C::SFB_CHUNKS + sfb_shift;
+              // advance 64 e2m1 = 32 bytes along K
+              mma_nvf4(d0, da0 + 2 * kk, db + 2 * kk, id, sf_a0 + 4 * kk, sfb, accum);
+              if (C::NA == 2)
+                mma_nvf4(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, id, sf_a1 + 4 * kk, sfb, accum);
+            }
           } else {
             // scale factors of this stage: smem -> TMEM (in order with the MMAs below)
             const uint32_t ssf = sb + C::B_BYTES;
@@ -386,6 +426,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       const uint32_t lane_addr =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::ACC_COLS;
       const int f_base = t.slab * C::SLAB_ROWS + quarter * 32;
+      // NVFP4: undo the global encode scales of both operands
+      float alpha = 1.0f;
+      if (DT == kNVF4)
+        alpha = 1.0f / (__ldg(p.ga[t.grp] + t.e * p.ga_stride[t.grp]) *
+                        __ldg(p.gw[t.grp] + t.e * p.gw_stride[t.grp]));
+      float hmax = 0.f;  // fc1 NVFP4: amax of this warp's bf16 h values
       for (int c0 = member * 32; c0 < t.n_tok; c0 += 64) {
         const int rows_here = min(32, t.n_tok - c0);
         uint32_t r0[32], r1[32];
@@ -447,13 +493,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
           const int f0 = f_base + half * kBM;
           if (MODE == kFc1) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              s[j * 32 + lane] =
-                  __float2bfloat16_rn(silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j]));
+            for (int j = 0; j < 32; ++j) {
+              const __nv_bfloat16 hb = __float2bfloat16_rn(
+                  silu_f(__uint_as_float(r0[j]) * alpha) * (__uint_as_float(r1[j]) * alpha));
+              s[j * 32 + lane] = hb;
+              if (DT == kNVF4 && j < rows_here) hmax = fmaxf(hmax, fabsf(__bfloat162float(hb)));
+            }
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              s[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(half ? r1[j] : r0[j]));
+              s[j * 32 + lane] =
+                  __float2bfloat16_rn(__uint_as_float(half ? r1[j] : r0[j]) * alpha);
           }
           __syncwarp();
 #pragma unroll
@@ -472,6 +522,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (MODE == kFc1 && DT == kNVF4) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+        if (lane == 0 && hmax > 0.f && f_base < G.a_valid_rows)
+          atomic_max_nonneg(p.amax_out[t.grp] + t.e * p.amax_stride[t.grp], hmax);
+      }
       if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
     }
   }

@@ -28,7 +28,9 @@ inline int64_t pad128(int64_t v) { return (v + 127) / 128 * 128; }
 // Workspace layout of the step calls.
 // ---------------------------------------------------------------------------
 struct StepLayout {
-  size_t status, hist, h, h_sf, h_shared, h_shared_sf, router_partials, total;
+  // h: fc1 output (bf16; MXFP8: e4m3 codes); h_q: NVFP4 codes of h; h_sf: scales
+  size_t status, hist, h, h_q, h_sf, h_shared, h_shared_q, h_shared_sf, g_h, router_partials,
+      total;
   int32_t r_cap, ntiles, router_splits;
 };
 
@@ -59,13 +61,19 @@ StepLayout step_layout(const moe_config& c) {
   size_t o = 0;
   L.status = o; o = align_up(o + 4);
   L.hist = o; o = align_up(o + static_cast<size_t>(L.ntiles) * c.E * 4);
-  const size_t eb = (c.dtype == MOE_BF16) ? 2 : 1;  // bytes per h element
+  const bool mx = c.dtype == MOE_MXFP8, nv = c.dtype == MOE_NVFP4;
+  const size_t eb = mx ? 1 : 2;  // bytes per element of h as fc1 writes it
   const size_t Is = c.I_shared > 0 ? c.I_shared : 0;
   const size_t Tp = static_cast<size_t>(pad128(c.T));
+  const size_t Rp = static_cast<size_t>(pad128(L.r_cap));
+  const size_t blk = mx ? 32 : 16;  // elements per scale
   L.h = o; o = align_up(o + static_cast<size_t>(L.r_cap) * c.I * eb);
-  L.h_sf = o; o = align_up(o + (eb == 1 ? static_cast<size_t>(pad128(L.r_cap)) * c.I / 32 : 0));
+  L.h_q = o; o = align_up(o + (nv ? static_cast<size_t>(L.r_cap) * c.I / 2 : 0));
+  L.h_sf = o; o = align_up(o + ((mx || nv) ? Rp * c.I / blk : 0));
   L.h_shared = o; o = align_up(o + Tp * Is * eb);
-  L.h_shared_sf = o; o = align_up(o + (eb == 1 ? Tp * Is / 32 : 0));
+  L.h_shared_q = o; o = align_up(o + (nv ? Tp * Is / 2 : 0));
+  L.h_shared_sf = o; o = align_up(o + ((mx || nv) ? Tp * Is / blk : 0));
+  L.g_h = o; o = align_up(o + (nv ? (static_cast<size_t>(c.E) + 1) * 4 : 0));
   L.router_splits = router_splits_of(c);
   L.router_partials = o;
   o = align_up(o + static_cast<size_t>(L.router_splits) * c.T * c.E * 4);
@@ -76,7 +84,7 @@ StepLayout step_layout(const moe_config& c) {
 struct FwdLayout {
   StepLayout step;
   size_t logits, topk_idx, topk_w, counts, offsets, row_token, token_row, rows, rows_sf,
-      out_rows, shared_out, x, x_q, x_sf, y, total;
+      out_rows, shared_out, x, x_q, x_sf, x_g, y, total;
 };
 
 FwdLayout fwd_layout(const moe_config& c) {
@@ -91,15 +99,18 @@ FwdLayout fwd_layout(const moe_config& c) {
   F.offsets = o; o = align_up(o + (E + 1) * 4);
   F.row_token = o; o = align_up(o + R * 4);
   F.token_row = o; o = align_up(o + T * k * 4);
-  const bool mx = c.dtype == MOE_MXFP8;
+  const bool mx = c.dtype == MOE_MXFP8, nv = c.dtype == MOE_NVFP4, q = mx || nv;
   const size_t Tp = static_cast<size_t>(pad128(c.T));
-  F.rows = o; o = align_up(o + R * H * (mx ? 1 : 2));
-  F.rows_sf = o; o = align_up(o + (mx ? static_cast<size_t>(pad128(R)) * H / 32 : 0));
+  const size_t row_b = mx ? H : (nv ? H / 2 : 2 * H);  // bytes per permuted row
+  const size_t sf_b = mx ? H / 32 : H / 16;            // scale bytes per row
+  F.rows = o; o = align_up(o + R * row_b);
+  F.rows_sf = o; o = align_up(o + (q ? static_cast<size_t>(pad128(R)) * sf_b : 0));
   F.out_rows = o; o = align_up(o + R * H * 2);
   F.shared_out = o; o = align_up(o + (c.I_shared > 0 ? T * H * 2 : 0));
   F.x = o; o = align_up(o + T * H * 2);
-  F.x_q = o; o = align_up(o + (mx ? T * H : 0));
-  F.x_sf = o; o = align_up(o + (mx ? Tp * H / 32 : 0));
+  F.x_q = o; o = align_up(o + (q ? T * row_b : 0));
+  F.x_sf = o; o = align_up(o + (q ? Tp * sf_b : 0));
+  F.x_g = o; o = align_up(o + (nv ? 4 : 0));
   F.y = o; o = align_up(o + T * H * 2);
   F.total = o;
   return F;
@@ -123,15 +134,19 @@ moe_status check_config(const moe_config* c) {
   return MOE_OK;
 }
 
-// Data paths built so far: bf16 and MXFP8 (which keeps 128-row scale chunks
-// aligned with expert segments: pad_multiple must be 128).
+// Block-scaled paths keep 128-row scale chunks aligned with expert segments
+// (pad_multiple must be 128); NVFP4 k-steps are 256 elements wide.
 moe_status check_dtype(const moe_config* c) {
   if (c->dtype == MOE_BF16) return MOE_OK;
-  if (c->dtype == MOE_MXFP8) return c->pad_multiple == 128 ? MOE_OK : MOE_ERR_UNSUPPORTED;
-  return MOE_ERR_UNSUPPORTED;
+  if (c->pad_multiple != 128) return MOE_ERR_UNSUPPORTED;
+  if (c->dtype == MOE_NVFP4 && (c->H % 256 || c->I % 256 || c->I_shared % 256))
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
 }
 
 inline bool is_mx(const moe_config& c) { return c.dtype == MOE_MXFP8; }
+inline bool is_nv(const moe_config& c) { return c.dtype == MOE_NVFP4; }
+inline bool is_bf16(const moe_config& c) { return c.dtype == MOE_BF16; }
 
 inline moe_status cuda_check(cudaError_t e) {
   if (e == cudaSuccess) return MOE_OK;
@@ -333,7 +348,7 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
   MOE_TRY(launch_check());
   permute_rank_kernel<<<L.ntiles, 32, hsm, s>>>(a);
   MOE_TRY(launch_check());
-  if (is_mx(c)) {
+  if (is_mx(c) || is_nv(c)) {
     GatherMxArgs g;
     g.src_codes = static_cast<const uint8_t*>(src_rows);
     g.src_scales = static_cast<const uint8_t*>(src_scales);
@@ -343,7 +358,8 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
     g.offsets = offsets;
     g.E = c.E;
     g.H = c.H;
-    permute_gather_mx_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
+    if (is_nv(c)) permute_gather_nv_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
+    else permute_gather_mx_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
     return launch_check();
   }
   GatherArgs g;
@@ -362,6 +378,7 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
 struct MlpQuant {
   const void* row_scales;
   const void* x_scales;
+  const float* x_global;  // NVFP4 global encode scale of x
 };
 
 template <int TILE_N, int DT>
@@ -374,10 +391,15 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
   void* h = wsb + L.h;
   void* hs = wsb + L.h_shared;
   const bool sh = c.I_shared > 0;
-  const bool mx = DT == kMXF8;
-  const auto tok_t = mx ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const int eb = mx ? 1 : 2;                  // bytes per element of activations / weights
-  const int kstep = mx ? 128 : kBK;           // K elements per k-step
+  const bool mx = DT == kMXF8, nv = DT == kNVF4, qz = mx || nv;
+  const auto tok_t = qz ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // operand bytes per K element (NVFP4 packs two per byte), map element bytes
+  auto kbytes = [&](uint64_t k) -> uint64_t { return nv ? k / 2 : (mx ? k : 2 * k); };
+  const int me = qz ? 1 : 2;                  // tensor-map element bytes
+  const int kstep = nv ? 256 : (mx ? 128 : kBK);  // K elements per k-step
+  const int kb4_div = nv ? 64 : 128;          // K elements per scale chunk column
+  float* g_h = reinterpret_cast<float*>(wsb + L.g_h);
+  if (nv) MOE_CUDA(cudaMemsetAsync(g_h, 0, (static_cast<size_t>(c.E) + 1) * 4, s));
   const uint64_t H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
   const int max_chunks = c.E + (c.T * c.top_k) / TILE_N + 1;
   const int dense_chunks = (c.T + TILE_N - 1) / TILE_N;
@@ -385,13 +407,13 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
   {
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    MOE_TRY(make_tiled_map(&p.a0[0], w.w1, E * I, H * eb));
-    MOE_TRY(make_tiled_map(&p.a1[0], w.w3, E * I, H * eb));
-    MOE_TRY(make_map(&p.b[0], rows, tok_t, eb, H, L.r_cap, H * eb, kBoxRows));
+    MOE_TRY(make_tiled_map(&p.a0[0], w.w1, E * I, kbytes(H)));
+    MOE_TRY(make_tiled_map(&p.a1[0], w.w3, E * I, kbytes(H)));
+    MOE_TRY(make_map(&p.b[0], rows, tok_t, me, kbytes(H) / me, L.r_cap, kbytes(H), kBoxRows));
     if (sh) {
-      MOE_TRY(make_tiled_map(&p.a0[1], w.ws1, Is, H * eb));
-      MOE_TRY(make_tiled_map(&p.a1[1], w.ws3, Is, H * eb));
-      MOE_TRY(make_map(&p.b[1], x, tok_t, eb, H, T, H * eb, kBoxRows));
+      MOE_TRY(make_tiled_map(&p.a0[1], w.ws1, Is, kbytes(H)));
+      MOE_TRY(make_tiled_map(&p.a1[1], w.ws3, Is, kbytes(H)));
+      MOE_TRY(make_map(&p.b[1], x, tok_t, me, kbytes(H) / me, T, kbytes(H), kBoxRows));
     } else {
       p.a0[1] = p.a0[0];
       p.a1[1] = p.a1[0];
@@ -399,18 +421,32 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     }
     p.g[0] = GemmGroup{c.I, c.I, c.I / kBM, c.H / kstep, 1, h, c.I, 0};
     p.g[1] = GemmGroup{0, c.I_shared, c.I_shared / kBM, c.H / kstep, 1, hs, c.I_shared, 0};
-    if (mx) {
+    if (qz) {
       p.sfa0[0] = static_cast<const uint8_t*>(w.w1_scales);
       p.sfa1[0] = static_cast<const uint8_t*>(w.w3_scales);
       p.sfb[0] = static_cast<const uint8_t*>(q.row_scales);
       p.sfa0[1] = static_cast<const uint8_t*>(w.ws1_scales);
       p.sfa1[1] = static_cast<const uint8_t*>(w.ws3_scales);
       p.sfb[1] = static_cast<const uint8_t*>(q.x_scales);
-      p.kb4[0] = p.kb4[1] = c.H / 128;
+      p.kb4[0] = p.kb4[1] = c.H / kb4_div;
+    }
+    if (mx) {
       p.q_out[0] = static_cast<uint8_t*>(h);
       p.q_sf[0] = wsb + L.h_sf;
       p.q_out[1] = static_cast<uint8_t*>(hs);
       p.q_sf[1] = wsb + L.h_shared_sf;
+    }
+    if (nv) {
+      p.ga[0] = p.ga[1] = q.x_global;
+      p.ga_stride[0] = p.ga_stride[1] = 0;
+      p.gw[0] = w.w13_global;
+      p.gw_stride[0] = 1;
+      p.gw[1] = sh ? w.ws13_global : w.w13_global;
+      p.gw_stride[1] = 0;
+      p.amax_out[0] = g_h;
+      p.amax_stride[0] = 1;
+      p.amax_out[1] = g_h + c.E;
+      p.amax_stride[1] = 0;
     }
     p.counts = counts;
     p.offsets = offsets;
@@ -420,15 +456,34 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     const int units = max_chunks * p.g[0].n_slabs + (sh ? dense_chunks * p.g[1].n_slabs : 0);
     MOE_TRY((launch_gemm<kFc1, TILE_N, DT>(p, units, s)));
   }
+  // NVFP4: h's per-expert global scales from the amax fc1 gathered, then h codes
+  void* h_in = h;
+  void* hs_in = hs;
+  if (nv) {
+    amax_to_global_kernel<<<(c.E + 1 + 255) / 256, 256, 0, s>>>(g_h, c.E + 1);
+    MOE_TRY(launch_check());
+    quantize_h_nvfp4_kernel<<<sm_count() * 4, 256, (c.E + 1) * 4, s>>>(
+        static_cast<const __nv_bfloat16*>(h), wsb + L.h_q, wsb + L.h_sf, c.I, offsets, counts,
+        c.E, g_h, 0);
+    MOE_TRY(launch_check());
+    if (sh) {
+      quantize_h_nvfp4_kernel<<<sm_count() * 2, 256, (c.E + 1) * 4, s>>>(
+          static_cast<const __nv_bfloat16*>(hs), wsb + L.h_shared_q, wsb + L.h_shared_sf,
+          c.I_shared, offsets, counts, c.E, g_h + c.E, c.T);
+      MOE_TRY(launch_check());
+    }
+    h_in = wsb + L.h_q;
+    hs_in = wsb + L.h_shared_q;
+  }
   // fc2: two adjacent 128-row slabs of W2 (256 output features) per tile
   {
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    MOE_TRY(make_tiled_map(&p.a0[0], w.w2, E * H, I * eb));
-    MOE_TRY(make_map(&p.b[0], h, tok_t, eb, I, L.r_cap, I * eb, kBoxRows));
+    MOE_TRY(make_tiled_map(&p.a0[0], w.w2, E * H, kbytes(I)));
+    MOE_TRY(make_map(&p.b[0], h_in, tok_t, me, kbytes(I) / me, L.r_cap, kbytes(I), kBoxRows));
     if (sh) {
-      MOE_TRY(make_tiled_map(&p.a0[1], w.ws2, H, Is * eb));
-      MOE_TRY(make_map(&p.b[1], hs, tok_t, eb, Is, T, Is * eb, kBoxRows));
+      MOE_TRY(make_tiled_map(&p.a0[1], w.ws2, H, kbytes(Is)));
+      MOE_TRY(make_map(&p.b[1], hs_in, tok_t, me, kbytes(Is) / me, T, kbytes(Is), kBoxRows));
     } else {
       p.a0[1] = p.a0[0];
       p.b[1] = p.b[0];
@@ -438,13 +493,23 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     const int slabs = (c.H + 2 * kBM - 1) / (2 * kBM);
     p.g[0] = GemmGroup{c.H, c.H, slabs, c.I / kstep, 1, out_rows, c.H, 0};
     p.g[1] = GemmGroup{0, c.H, slabs, (sh ? c.I_shared : kstep) / kstep, 1, shared_out, c.H, 0};
-    if (mx) {
+    if (qz) {
       p.sfa0[0] = static_cast<const uint8_t*>(w.w2_scales);
       p.sfb[0] = wsb + L.h_sf;
       p.sfa0[1] = static_cast<const uint8_t*>(w.ws2_scales);
       p.sfb[1] = wsb + L.h_shared_sf;
-      p.kb4[0] = c.I / 128;
-      p.kb4[1] = sh ? c.I_shared / 128 : 1;
+      p.kb4[0] = c.I / kb4_div;
+      p.kb4[1] = sh ? c.I_shared / kb4_div : 1;
+    }
+    if (nv) {
+      p.ga[0] = g_h;
+      p.ga_stride[0] = 1;
+      p.ga[1] = g_h + c.E;
+      p.ga_stride[1] = 0;
+      p.gw[0] = w.w2_global;
+      p.gw_stride[0] = 1;
+      p.gw[1] = sh ? w.ws2_global : w.w2_global;
+      p.gw_stride[1] = 0;
     }
     p.counts = counts;
     p.offsets = offsets;
@@ -463,6 +528,9 @@ moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void*
                           cudaStream_t s) {
   if (is_mx(c))
     return grouped_mlp_tiles<192, kMXF8>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
+                                         ws, s);
+  if (is_nv(c))
+    return grouped_mlp_tiles<128, kNVF4>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
                                          ws, s);
   if (expert_tile_n() == 128)
     return grouped_mlp_tiles<128, kBF16>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
@@ -569,8 +637,8 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
   if (!topk_idx || !src_rows || !counts || !offsets || !row_token || !token_row || !dst_rows)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(src_rows) || !aligned16(dst_rows)) return MOE_ERR_INVALID_ARG;
-  if (is_mx(*cfg) && (!src_scales || !dst_scales || !aligned16(src_scales) ||
-                      !aligned16(dst_scales)))
+  if (!is_bf16(*cfg) && (!src_scales || !dst_scales || !aligned16(src_scales) ||
+                         !aligned16(dst_scales)))
     return MOE_ERR_INVALID_ARG;
   return do_permute(*cfg, topk_idx, src_rows, src_scales, counts, offsets, row_token, token_row,
                     dst_rows, dst_scales, workspace, static_cast<cudaStream_t>(stream));
@@ -581,7 +649,6 @@ moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w, const vo
                            const float* x_global, const int32_t* counts, const int32_t* offsets,
                            void* out_rows, void* shared_out, void* workspace,
                            size_t workspace_bytes, void* stream) {
-  (void)x_global;
   MOE_TRY(check_config(cfg));
   MOE_TRY(check_dtype(cfg));
   MOE_TRY(check_ws(*cfg, workspace, workspace_bytes));
@@ -590,14 +657,18 @@ moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w, const vo
   if (!aligned16(rows) || !aligned16(out_rows)) return MOE_ERR_INVALID_ARG;
   if (cfg->I_shared > 0 && (!x || !shared_out || !aligned16(x) || !aligned16(shared_out)))
     return MOE_ERR_INVALID_ARG;
-  if (is_mx(*cfg)) {
+  if (!is_bf16(*cfg)) {
     if (!row_scales || !aligned16(row_scales)) return MOE_ERR_INVALID_ARG;
     if (cfg->I_shared > 0 && (!x_scales || !aligned16(x_scales))) return MOE_ERR_INVALID_ARG;
     if (!w->w1_scales || !w->w3_scales || !w->w2_scales) return MOE_ERR_INVALID_ARG;
     if (cfg->I_shared > 0 && (!w->ws1_scales || !w->ws3_scales || !w->ws2_scales))
       return MOE_ERR_INVALID_ARG;
   }
-  MlpQuant q{row_scales, x_scales};
+  if (is_nv(*cfg)) {
+    if (!x_global || !w->w13_global || !w->w2_global) return MOE_ERR_INVALID_ARG;
+    if (cfg->I_shared > 0 && (!w->ws13_global || !w->ws2_global)) return MOE_ERR_INVALID_ARG;
+  }
+  MlpQuant q{row_scales, x_scales, x_global};
   return do_grouped_mlp(*cfg, *w, rows, x, q, counts, offsets, out_rows, shared_out, workspace,
                         static_cast<cudaStream_t>(stream));
 }
@@ -617,16 +688,19 @@ moe_status moe_prepared_weights_size(const moe_config* cfg, moe_weight_sizes* si
   MOE_TRY(check_dtype(cfg));
   if (!sizes) return MOE_ERR_INVALID_ARG;
   const size_t H = cfg->H, I = cfg->I, E = cfg->E, Is = cfg->I_shared;
-  const size_t eb = is_mx(*cfg) ? 1 : 2;
-  sizes->w13 = E * I * H * eb;
-  sizes->w2 = E * H * I * eb;
-  sizes->ws13 = Is * H * eb;
-  sizes->ws2 = H * Is * eb;
-  const bool mx = is_mx(*cfg);
-  sizes->w13_scales = mx ? E * I * H / 32 : 0;
-  sizes->w2_scales = mx ? E * H * I / 32 : 0;
-  sizes->ws13_scales = mx ? Is * H / 32 : 0;
-  sizes->ws2_scales = mx ? H * Is / 32 : 0;
+  // bytes per weight element x2 (NVFP4 packs two per byte), elements per scale
+  const size_t e2 = is_mx(*cfg) ? 2 : (is_nv(*cfg) ? 1 : 4);
+  const size_t blk = is_mx(*cfg) ? 32 : (is_nv(*cfg) ? 16 : 0);
+  sizes->w13 = E * I * H * e2 / 2;
+  sizes->w2 = E * H * I * e2 / 2;
+  sizes->ws13 = Is * H * e2 / 2;
+  sizes->ws2 = H * Is * e2 / 2;
+  sizes->w13_scales = blk ? E * I * H / blk : 0;
+  sizes->w2_scales = blk ? E * H * I / blk : 0;
+  sizes->ws13_scales = blk ? Is * H / blk : 0;
+  sizes->ws2_scales = blk ? H * Is / blk : 0;
+  sizes->w_globals = is_nv(*cfg) ? E * 4 : 0;
+  sizes->ws_globals = is_nv(*cfg) && Is ? 4 : 0;
   return MOE_OK;
 }
 
@@ -666,6 +740,53 @@ moe_status moe_prepare_weights(const moe_config* cfg, int32_t which, int32_t e_b
     return MOE_ERR_INVALID_ARG;
   }
   if (!aligned16(d1) || !aligned16(d3) || !aligned16(d2)) return MOE_ERR_INVALID_ARG;
+  if (is_nv(c)) {
+    // per-expert global scales from the amax of W1 and W3 together, and of W2;
+    // codes tile-major (128 rows x 256 elements), scales in the MMA layout
+    const size_t off13 = which == 0 ? static_cast<size_t>(e_begin) * c.I * c.H : 0;
+    const size_t off2 = which == 0 ? static_cast<size_t>(e_begin) * c.H * c.I : 0;
+    float* g13 = which == 0 ? dst->w13_global + e_begin : dst->ws13_global;
+    float* g2 = which == 0 ? dst->w2_global + e_begin : dst->ws2_global;
+    uint8_t* s1 = static_cast<uint8_t*>(which == 0 ? dst->w1_scales : dst->ws1_scales);
+    uint8_t* s3 = static_cast<uint8_t*>(which == 0 ? dst->w3_scales : dst->ws3_scales);
+    uint8_t* s2 = static_cast<uint8_t*>(which == 0 ? dst->w2_scales : dst->ws2_scales);
+    if (!s1 || !s3 || !s2 || !g13 || !g2) return MOE_ERR_INVALID_ARG;
+    uint8_t* c1 = static_cast<uint8_t*>(which == 0 ? dst->w1 : dst->ws1) + off13 / 2;
+    uint8_t* c3 = static_cast<uint8_t*>(which == 0 ? dst->w3 : dst->ws3) + off13 / 2;
+    uint8_t* c2 = static_cast<uint8_t*>(which == 0 ? dst->w2 : dst->ws2) + off2 / 2;
+    const int ng = which == 0 ? e_count : 1;
+    MOE_CUDA(cudaMemsetAsync(g13, 0, ng * 4, s));
+    MOE_CUDA(cudaMemsetAsync(g2, 0, ng * 4, s));
+    const int64_t per13 = rows13 / ng * k13, per2 = rows2 / ng * k2;  // elements per expert
+    const dim3 ga(static_cast<unsigned>((per13 / 8 + 255) / 256 < 64 ? (per13 / 8 + 255) / 256 : 64),
+                  ng);
+    const dim3 gb(static_cast<unsigned>((per2 / 8 + 255) / 256 < 64 ? (per2 / 8 + 255) / 256 : 64),
+                  ng);
+    amax_groups_kernel<<<ga, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w1), per13, g13);
+    MOE_TRY(launch_check());
+    amax_groups_kernel<<<ga, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w3), per13, g13);
+    MOE_TRY(launch_check());
+    amax_groups_kernel<<<gb, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w2), per2, g2);
+    MOE_TRY(launch_check());
+    amax_to_global_kernel<<<(ng + 255) / 256, 256, 0, s>>>(g13, ng);
+    MOE_TRY(launch_check());
+    amax_to_global_kernel<<<(ng + 255) / 256, 256, 0, s>>>(g2, ng);
+    MOE_TRY(launch_check());
+    const int64_t b13 = rows13 * (k13 / 16), b2 = rows2 * (k2 / 16);
+    const int64_t rpg13 = rows13 / ng, rpg2 = rows2 / ng;
+    quantize_nvfp4_kernel<<<static_cast<unsigned>((b13 + 255) / 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(w1), c1, s1 + off13 / 16, rows13,
+        static_cast<int>(k13), g13, rpg13, 1);
+    MOE_TRY(launch_check());
+    quantize_nvfp4_kernel<<<static_cast<unsigned>((b13 + 255) / 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(w3), c3, s3 + off13 / 16, rows13,
+        static_cast<int>(k13), g13, rpg13, 1);
+    MOE_TRY(launch_check());
+    quantize_nvfp4_kernel<<<static_cast<unsigned>((b2 + 255) / 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(w2), c2, s2 + off2 / 16, rows2, static_cast<int>(k2),
+        g2, rpg2, 1);
+    return launch_check();
+  }
   if (is_mx(c)) {
     // codes tile-major, scales in the MMA layout; byte offsets of the expert range
     const size_t off13 = which == 0 ? static_cast<size_t>(e_begin) * c.I * c.H : 0;
@@ -702,11 +823,27 @@ moe_status moe_prepare_weights(const moe_config* cfg, int32_t which, int32_t e_b
 
 moe_status moe_quantize(int32_t dtype, const void* in, int32_t rows, int32_t cols, void* codes,
                         void* scales, float* global_scale, void* stream) {
-  (void)global_scale;
-  if (dtype != MOE_MXFP8) return dtype == MOE_NVFP4 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_MXFP8 && dtype != MOE_NVFP4) return MOE_ERR_INVALID_ARG;
   if (!in || !codes || !scales || rows < 1 || cols < 1) return MOE_ERR_INVALID_ARG;
-  if (cols % 128) return MOE_ERR_UNSUPPORTED;
+  if (cols % (dtype == MOE_NVFP4 ? 256 : 128)) return MOE_ERR_UNSUPPORTED;
   if (!aligned16(in) || !aligned16(codes)) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_NVFP4) {
+    if (!global_scale) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n = static_cast<int64_t>(rows) * cols;
+    MOE_CUDA(cudaMemsetAsync(global_scale, 0, 4, st));
+    const unsigned nb = static_cast<unsigned>((n / 8 + 255) / 256 < 2048 ? (n / 8 + 255) / 256 : 2048);
+    amax_groups_kernel<<<dim3(nb, 1), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), n,
+                                                    global_scale);
+    MOE_TRY(launch_check());
+    amax_to_global_kernel<<<1, 32, 0, st>>>(global_scale, 1);
+    MOE_TRY(launch_check());
+    const int64_t blocks = static_cast<int64_t>(rows) * (cols / 16);
+    quantize_nvfp4_kernel<<<static_cast<unsigned>((blocks + 255) / 256), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(in), static_cast<uint8_t*>(codes),
+        static_cast<uint8_t*>(scales), rows, cols, global_scale, 0, 0);
+    return launch_check();
+  }
   const int64_t blocks = static_cast<int64_t>(rows) * (cols / 32);
   quantize_mxfp8_rows_kernel<<<static_cast<unsigned>((blocks + 255) / 256), 256, 0,
                                static_cast<cudaStream_t>(stream)>>>(
@@ -757,11 +894,12 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   void* shared_out = c.I_shared > 0 ? b + F.shared_out : nullptr;
   MOE_TRY(do_route(c, xd, w_router, bias, nullptr, logits, topk_idx, topk_w, workspace, s));
   const void* xq = xd;
-  MlpQuant q{nullptr, nullptr};
-  if (is_mx(c)) {
-    MOE_TRY(moe_quantize(MOE_MXFP8, xd, c.T, c.H, b + F.x_q, b + F.x_sf, nullptr, s));
+  MlpQuant q{nullptr, nullptr, nullptr};
+  if (!is_bf16(c)) {
+    float* xg = reinterpret_cast<float*>(b + F.x_g);
+    MOE_TRY(moe_quantize(c.dtype, xd, c.T, c.H, b + F.x_q, b + F.x_sf, xg, s));
     xq = b + F.x_q;
-    q = MlpQuant{b + F.rows_sf, b + F.x_sf};
+    q = MlpQuant{b + F.rows_sf, b + F.x_sf, xg};
   }
   MOE_TRY(do_permute(c, topk_idx, xq, q.x_scales, counts, offsets, row_token, token_row, rows,
                      b + F.rows_sf, workspace, s));

@@ -134,3 +134,162 @@ __global__ void __launch_bounds__(256) permute_gather_mx_kernel(GatherMxArgs a) 
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// NVFP4 (sglang PR "Mistral Large 3 NVFP4 TRTLLM MoE support", Modifications:
+// W4A4 NVFP4): e2m1 elements, a ue4m3 scale per 16 K elements and an fp32
+// global encode scale g = 2688 / amax of the tensor.  Codes are packed two per
+// byte (element 2i in the low nibble); scales use the MMA scale layout with
+// KB = cols / 16 blocks per row.
+// ---------------------------------------------------------------------------
+
+// amax per group: out[blockIdx.y] = max |in[blockIdx.y * group_elems + i]|
+// over a group of group_elems bf16 values (group_elems % 8 == 0; out must start
+// at zero).  Each block reduces a strided slice and issues one atomic.
+__global__ void __launch_bounds__(256) amax_groups_kernel(const __nv_bfloat16* __restrict__ in,
+                                                          int64_t group_elems, float* out) {
+  __shared__ float red[8];
+  const int64_t vecs = group_elems / 8;
+  const uint4* base = reinterpret_cast<const uint4*>(in + blockIdx.y * group_elems);
+  float m = 0.f;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < vecs;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 raw = base[v];
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(p2[i]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    if (m > 0.f) atomic_max_nonneg(out + blockIdx.y, m);
+  }
+}
+
+// In place: amax -> global encode scale.
+__global__ void amax_to_global_kernel(float* v, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) v[i] = nv_global_scale(v[i]);
+}
+
+__device__ __forceinline__ void load_bf16x16(const __nv_bfloat16* src, float (&v)[16]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint4 raw = s[q];
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(p2[i]);
+      v[q * 8 + 2 * i] = f.x;
+      v[q * 8 + 2 * i + 1] = f.y;
+    }
+  }
+}
+
+// One thread per 16-element block of a row-major bf16 [rows, cols] matrix,
+// global scale g[r / rows_per_group] (rows_per_group 0: g[0]).  tiled != 0
+// writes codes tile-major (128 rows x 128 bytes = 256 elements per tile).
+__global__ void __launch_bounds__(256) quantize_nvfp4_kernel(
+    const __nv_bfloat16* __restrict__ in, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, int64_t rows, int cols, const float* __restrict__ g,
+    int64_t rows_per_group, int tiled) {
+  const int KB = cols / 16;
+  const int64_t blk = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (blk >= rows * KB) return;
+  const int64_t r = blk / KB;
+  const int kb = static_cast<int>(blk - r * KB);
+  float v[16];
+  load_bf16x16(in + r * cols + kb * 16, v);
+  const float gs = g[rows_per_group > 0 ? r / rows_per_group : 0];
+  uint32_t packed[2];
+  const uint32_t sb = nv_quantize_block16(v, gs, packed);
+  uint8_t* dst;
+  if (tiled) {
+    const int64_t tile = (r >> 7) * (cols >> 8) + (kb >> 4);
+    dst = codes + tile * 16384 + (r & 127) * 128 + (kb & 15) * 8;
+  } else {
+    dst = codes + r * (cols / 2) + kb * 8;
+  }
+  *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+  scales[sf_offset(r, kb, KB)] = static_cast<uint8_t>(sb);
+}
+
+// NVFP4 quantization of the fc2 input h (bf16, expert-major rows): the row's
+// expert e comes from the segment offsets; global scale g_h[e]; pad rows
+// (past counts[e] in their segment) get zero codes and scales.  `dense` > 0
+// quantizes `dense` token-order rows with g_h[0] instead (shared expert).
+__global__ void __launch_bounds__(256) quantize_h_nvfp4_kernel(
+    const __nv_bfloat16* __restrict__ h, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, int cols, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ counts, int E, const float* __restrict__ g_h, int dense) {
+  extern __shared__ int32_t s_off[];  // [E + 1]
+  if (!dense)
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
+  __syncthreads();
+  const int KB = cols / 16;
+  const int64_t rows = dense ? dense : s_off[E];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t blk = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; blk < rows * KB;
+       blk += stride) {
+    const int64_t r = blk / KB;
+    const int kb = static_cast<int>(blk - r * KB);
+    int e = 0;
+    bool pad = false;
+    if (!dense) {
+      int lo = 0, hi = E;  // s_off[lo] <= r < s_off[lo+1]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_off[mid] <= r) lo = mid; else hi = mid;
+      }
+      e = lo;
+      pad = (r - s_off[e]) >= counts[e];
+    }
+    uint32_t packed[2] = {0u, 0u};
+    uint32_t sb = 0u;
+    if (!pad) {
+      float v[16];
+      load_bf16x16(h + r * cols + kb * 16, v);
+      sb = nv_quantize_block16(v, g_h[e], packed);
+    }
+    *reinterpret_cast<uint2*>(codes + r * (cols / 2) + kb * 8) = make_uint2(packed[0], packed[1]);
+    scales[sf_offset(r, kb, KB)] = static_cast<uint8_t>(sb);
+  }
+}
+
+// Expert-major gather of NVFP4 rows (packed codes, H/2 bytes per row) and
+// their scale words (4 blocks of 16 per 32-bit word).
+__global__ void __launch_bounds__(256) permute_gather_nv_kernel(GatherMxArgs a) {
+  const int rows = a.offsets[a.E];
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int row_bytes = a.H / 2;
+  const int vecs = row_bytes >> 4;
+  const int KB = a.H / 16, W = KB / 4;
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int t = a.row_token[r];
+    uint4* d = reinterpret_cast<uint4*>(a.dst_codes + static_cast<int64_t>(r) * row_bytes);
+    if (t >= 0) {
+      const uint4* s =
+          reinterpret_cast<const uint4*>(a.src_codes + static_cast<int64_t>(t) * row_bytes);
+      for (int v = lane; v < vecs; v += 32) d[v] = __ldg(s + v);
+      for (int w = lane; w < W; w += 32)
+        *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) =
+            *reinterpret_cast<const uint32_t*>(a.src_scales + sf_offset(t, 4 * w, KB));
+    } else {
+      for (int v = lane; v < vecs; v += 32) d[v] = make_uint4(0, 0, 0, 0);
+      for (int w = lane; w < W; w += 32)
+        *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) = 0u;
+    }
+  }
+}
+
+}  // namespace moe
