@@ -191,7 +191,8 @@ def run_reference(args, cfg):
 # our arm
 # ---------------------------------------------------------------------------
 
-WEIGHT_BYTES = {"bf16": 2.0, "mxfp8": 1.0 + 1.0 / 32}  # per element, scales included
+WEIGHT_BYTES = {"bf16": 2.0, "mxfp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}  # per element
+TENSOR_RATIO = {"bf16": 1.0, "mxfp8": 2.0, "nvfp4": 4.0}  # nominal dense peak vs bf16
 
 
 def grouped_mlp_algorithmic(cfg, touched):
@@ -211,6 +212,38 @@ def layer_algorithmic(cfg, touched):
     return b, f
 
 
+def prepare_streaming(M, cfg, c, dev):
+    """Prepared weights, drawn and converted one expert at a time."""
+    sz = M.moe_prepared_weights_size(c)
+    u8 = dict(dtype=torch.uint8, device=dev)
+    p = {"w1": torch.empty(sz["w13"], **u8), "w3": torch.empty(sz["w13"], **u8),
+         "w2": torch.empty(sz["w2"], **u8)}
+    if sz["w13_scales"]:
+        for k, n in (("w1_scales", "w13_scales"), ("w3_scales", "w13_scales"),
+                     ("w2_scales", "w2_scales")):
+            p[k] = torch.empty(sz[n], **u8)
+    if sz["w_globals"]:
+        p["w13_global"] = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+        p["w2_global"] = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+    if cfg.I_shared:
+        p["ws1"], p["ws3"] = torch.empty(sz["ws13"], **u8), torch.empty(sz["ws13"], **u8)
+        p["ws2"] = torch.empty(sz["ws2"], **u8)
+        if sz["ws13_scales"]:
+            for k, n in (("ws1_scales", "ws13_scales"), ("ws3_scales", "ws13_scales"),
+                         ("ws2_scales", "ws2_scales")):
+                p[k] = torch.empty(sz[n], **u8)
+        if sz["ws_globals"]:
+            p["ws13_global"] = torch.empty(1, dtype=torch.float32, device=dev)
+            p["ws2_global"] = torch.empty(1, dtype=torch.float32, device=dev)
+    dst = M.binding.weights_struct(p)
+    for e in range(cfg.E):
+        M.moe_prepare_weights(c, 0, e, 1, *synth.gen_expert_weights(cfg, e, dev), dst)
+    if cfg.I_shared:
+        M.moe_prepare_weights(c, 1, 0, 1, *synth.gen_shared_weights(cfg, dev), dst)
+    torch.cuda.synchronize()
+    return p
+
+
 def run_ours(args, cfg):
     import mixture_experts_layer_grouped_b200 as M
     ws_n, rank, local = _dist()
@@ -223,12 +256,10 @@ def run_ours(args, cfg):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     c = M.config_from_shape(cfg)
-    d = synth.gen_all(cfg, dev)
-    # each rank its own batch of tokens
-    if rank:
-        d["x"] = synth.gen_x(cfg.scaled(seed=rank), dev)
-    w = {k: d[k] for k in ("w1", "w3", "w2", "ws1", "ws3", "ws2") if k in d}
-    layer = M.MoELayer(c, w, d["w_router"], d["bias"])
+    d = {"x": synth.gen_x(cfg.scaled(seed=rank) if rank else cfg, dev)}  # each rank its batch
+    d["w_router"], d["bias"] = synth.gen_router(cfg, dev)
+    layer = M.MoELayer(c, prepare_streaming(M, cfg, c, dev), d["w_router"], d["bias"],
+                       prepared=True)
     x, y = d["x"], torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -305,13 +336,16 @@ def run_ours(args, cfg):
     tw = torch.empty(cfg.T, cfg.top_k, dtype=torch.float32, device=dev)
     counts, offsets = torch.empty(cfg.E, **i32), torch.empty(cfg.E + 1, **i32)
     row_token, token_row = torch.empty(r_cap, **i32), torch.empty(cfg.T * cfg.top_k, **i32)
-    mx = cfg.dtype == "mxfp8"
-    rows = torch.empty(r_cap, cfg.H, dtype=torch.uint8 if mx else torch.bfloat16, device=dev)
-    xc = xs = rows_sf = None
+    mx = cfg.dtype != "bf16"  # block-scaled: quantize x, permute codes and scales
+    rb = {"bf16": 2 * cfg.H, "mxfp8": cfg.H, "nvfp4": cfg.H // 2}[cfg.dtype]
+    rows = torch.empty(r_cap, rb, dtype=torch.uint8, device=dev)
+    xc = xs = rows_sf = xg = None
     if mx:
-        xc = torch.empty(cfg.T, cfg.H, dtype=torch.uint8, device=dev)
-        xs = torch.zeros(M.scale_bytes(cfg.T, cfg.H), dtype=torch.uint8, device=dev)
-        rows_sf = torch.zeros(M.scale_bytes(r_cap, cfg.H), dtype=torch.uint8, device=dev)
+        xc = torch.empty(cfg.T, rb, dtype=torch.uint8, device=dev)
+        xs = torch.zeros(M.scale_bytes(cfg.T, cfg.H, cfg.dtype), dtype=torch.uint8, device=dev)
+        rows_sf = torch.zeros(M.scale_bytes(r_cap, cfg.H, cfg.dtype), dtype=torch.uint8,
+                              device=dev)
+        xg = torch.empty(1, dtype=torch.float32, device=dev)
     out_rows = torch.empty(r_cap, cfg.H, dtype=torch.bfloat16, device=dev)
     shared_out = (torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
                   if cfg.I_shared else None)
@@ -322,14 +356,14 @@ def run_ours(args, cfg):
         M.moe_route(c, x, d["w_router"], d["bias"], idx, tw, wsp, logits_out=logits)
         evs[1].record(stream)
         if mx:
-            M.moe_quantize("mxfp8", x, xc, xs)
+            M.moe_quantize(cfg.dtype, x, xc, xs, global_scale=xg)
         evs[2].record(stream)
         M.moe_permute(c, idx, xc if mx else x, counts, offsets, row_token, token_row, rows, wsp,
                       src_scales=xs, dst_scales=rows_sf)
         evs[3].record(stream)
         M.moe_grouped_mlp(c, layer.weights, rows, counts, offsets, out_rows, wsp,
                           x=xc if mx else x, shared_out=shared_out, row_scales=rows_sf,
-                          x_scales=xs)
+                          x_scales=xs, x_global=xg)
         evs[4].record(stream)
         M.moe_combine(c, out_rows, token_row, tw, y, shared_out=shared_out)
         evs[5].record(stream)
@@ -341,8 +375,8 @@ def run_ours(args, cfg):
     mlp_ms = statistics.mean(steps_ms["grouped_mlp"])
     wbytes, flops = grouped_mlp_algorithmic(cfg, touched)
     hbm, tf_burst, tf_sus, peak_kind = _peaks()
-    # a contraction takes the peak of its own dtype: fp8 dense = 2 x bf16 (nominal ratio)
-    tf_dtype = tf_burst * (2.0 if mx else 1.0)
+    # a contraction takes the peak of its own dtype: bf16 peak x the nominal ratio
+    tf_dtype = tf_burst * TENSOR_RATIO[cfg.dtype]
     achieved_gbs = wbytes / (mlp_ms * 1e-3) / 1e9
     lb, lf = layer_algorithmic(cfg, touched)
     roof_ms = max(lb / (hbm * 1e9), lf / (tf_dtype * 1e12)) * 1e3
@@ -365,7 +399,8 @@ def run_ours(args, cfg):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3+e8m0 (mxfp8), fp32 acc" if mx else "bf16",
+        "dtype": {"bf16": "bf16", "mxfp8": "e4m3+e8m0 (mxfp8), fp32 acc",
+                  "nvfp4": "e2m1+ue4m3+fp32 global (nvfp4), fp32 acc"}[cfg.dtype],
         "data": "synthetic (seeded normal inputs and random-init weights of the workload)",
         "config": dict(_workload(cfg, "inputs larger than L2: %.0f MB of expert weights per step"
                                  % (WEIGHT_BYTES[cfg.dtype] * 3 * cfg.H * cfg.I * cfg.E / 1e6)),
@@ -376,15 +411,15 @@ def run_ours(args, cfg):
                      "algorithmic_bytes_per_launch": wbytes, "ms_per_launch": mlp_ms,
                      "tensor_tflops": flops / (mlp_ms * 1e-3) / 1e12,
                      "tensor_frac": flops / (mlp_ms * 1e-3) / 1e12 / tf_dtype,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs; bf16_tflops"
-                                    + (" x 2 for fp8)" if mx else ")")},
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs; bf16_tflops x "
+                                    f"{TENSOR_RATIO[cfg.dtype]:g} for {cfg.dtype})"},
         "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_max,
                            "bytes": lb, "flops": lf, "experts_touched": touched},
         "step_ms": {k: statistics.mean(v) for k, v in steps_ms.items()},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
                 "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
-        "gpu_launches": (10 if mx else 9) * args.steps,
+        "gpu_launches": ({"bf16": 9, "mxfp8": 10, "nvfp4": 14}[cfg.dtype] + (1 if cfg.dtype == "nvfp4" and cfg.I_shared else 0)) * args.steps,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"], "samples": clocks["samples"]},
         "tile_n": int(os.environ.get("MOE_GEMM_TILE_N", "256")),
