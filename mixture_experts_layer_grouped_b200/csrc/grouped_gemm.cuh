@@ -256,8 +256,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         const Tile t = decode_tile<MODE, TILE_N>(u, p, prefix, units_routed);
         const int nbox = (t.n_tok + kBoxRows - 1) / kBoxRows;
         const int nsfb = ((t.row0 & 127) + t.n_tok + 127) / 128;
+        // fc2's second 128-row slab may lie past the expert's last row (odd number of
+        // slabs): its outputs are masked, and its scale chunk (no bounds check on a bulk
+        // copy) is not loaded
+        const bool slab1 = (MODE != kFc2) ||
+                           (t.slab * C::SLAB_ROWS + kBM < p.g[t.grp].a_valid_rows);
+        const int n_sfa = (MODE == kRouter) ? 1 : (slab1 ? 2 : 1);
         const uint32_t bytes = C::NA * C::A_BYTES + nbox * kBoxRows * 128 +
-                               (DT != kBF16 ? (C::NA + nsfb) * C::SF_KCH * C::SF_CHUNK : 0);
+                               (DT != kBF16 ? (n_sfa + nsfb) * C::SF_KCH * C::SF_CHUNK : 0);
         for (int kt = t.k_begin; kt < t.k_end; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           uint8_t* sa = ring + stage * C::STAGE_BYTES;
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             if (MODE == kFc1)
               bulk_load(ssf + cb_bytes, p.sfa1[t.grp] + ca * C::SF_CHUNK, cb_bytes, &full[stage],
                         pol_w);
-            else if (MODE == kFc2)
+            else if (MODE == kFc2 && slab1)
               bulk_load(ssf + cb_bytes, p.sfa0[t.grp] + (ca + kb4) * C::SF_CHUNK, cb_bytes,
                         &full[stage], pol_w);
             for (int cb = 0; cb < nsfb; ++cb) {
