@@ -98,14 +98,16 @@ struct GemmCfg {
   static constexpr int SFB_CHUNKS = (TILE_N + 96 + 127) / 128;
   static constexpr int SF_BYTES = (DT != kBF16) ? (NA + SFB_CHUNKS) * SF_KCH * SF_CHUNK : 0;
   static constexpr int STAGE_BYTES = (NA * A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
-  static constexpr int STAGES = (kRingBytes / STAGE_BYTES) > 8 ? 8 : (kRingBytes / STAGE_BYTES);
+  static constexpr int RING = (DT == kNVF4) ? 198 * 1024 : kRingBytes;
+  static constexpr int STAGES = (RING / STAGE_BYTES) > 8 ? 8 : (RING / STAGE_BYTES);
   static constexpr int ACC_COLS = NA * TILE_N;  // TMEM columns of one tile
   static constexpr int SF_COLS = (DT != kBF16) ? 4 * SF_KCH * (NA + SFB_CHUNKS) : 0;
   static constexpr int ACC_BUFS = (2 * ACC_COLS + SF_COLS <= 512) ? 2 : 1;
   static constexpr int SF_TMEM = ACC_BUFS * ACC_COLS;  // first scale-factor column
   static constexpr uint32_t TMEM_COLS = pow2_at_least(ACC_BUFS * ACC_COLS + SF_COLS);
   static constexpr int SLAB_ROWS = (MODE == kFc2) ? 2 * kBM : kBM;  // features per tile
-  static constexpr int STG_BYTES = kEpiWarps * 32 * 32 * 2;  // per warp 32x32 bf16
+  static constexpr int STG_WARP = 32 * 34 * 2;                 // per warp 32 x 34 bf16
+  static constexpr int STG_BYTES = kEpiWarps * STG_WARP;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES + 4 * (kMaxExperts + 1);
@@ -421,7 +423,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     // ---------------- epilogue (warps 2..9) ----------------
     const int quarter = warp & 3;          // TMEM lane quarter this warp may access
     const int member = (warp - 2) >> 2;    // which of the quarter's two warps
-    uint8_t* my_stg = stg + (warp - 2) * (32 * 32 * 2);
+    uint8_t* my_stg = stg + (warp - 2) * C::STG_WARP;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
@@ -457,34 +459,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
           continue;
         }
         if (MODE == kFc1 && DT == kMXF8) {
-          // h = bf16(silu(gate) * up), then MXFP8: the 32 features of this warp are
-          // one scale block per token; codes staged [32 tokens][32 bytes].
-          uint8_t* s8 = my_stg;
-          uint8_t* qo = p.q_out[t.grp];
-          uint8_t* qs = p.q_sf[t.grp];
-          const int KBh = static_cast<int>(G.out_ld) / 32;
-          const int kb = f_base / 32;
+          // h = bf16(silu(gate) * up) staged as [32 tokens][32 features] (row stride 34
+          // bf16 to spread banks); then lane j takes token j: the warp's 32 features
+          // are one MXFP8 block, quantized from registers without cross-lane work.
+          constexpr int RS = 34;
+          __nv_bfloat16* hs_ = reinterpret_cast<__nv_bfloat16*>(my_stg);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float hv = __bfloat162float(__float2bfloat16_rn(
-                silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j])));
-            float amax = fabsf(hv);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            const uint32_t code = mx_scale_code(amax);
-            s8[j * 32 + lane] = to_e4m3(hv * mx_inv_scale(code));
-            if (lane == 0 && j < rows_here && f_base < G.a_valid_rows)
-              qs[sf_offset(t.row0 + c0 + j, kb, KBh)] = static_cast<uint8_t>(code);
-          }
+          for (int j = 0; j < 32; ++j)
+            hs_[j * RS + lane] = __float2bfloat16_rn(silu_f(__uint_as_float(r0[j])) *
+                                                     __uint_as_float(r1[j]));
           __syncwarp();
-          const uint4* s4q = reinterpret_cast<const uint4*>(my_stg);
+          if (lane < rows_here && f_base < G.a_valid_rows) {
+            float v[32];
+            float amax = 0.f;
+            const __nv_bfloat162* row = reinterpret_cast<const __nv_bfloat162*>(hs_ + lane * RS);
 #pragma unroll
-          for (int it = 0; it < 2; ++it) {
-            const int c = it * 32 + lane;
-            const int j = c >> 1, part = c & 1;
-            if (j < rows_here && f_base < G.a_valid_rows)
-              *reinterpret_cast<uint4*>(qo + static_cast<int64_t>(t.row0 + c0 + j) * G.out_ld +
-                                        f_base + part * 16) = s4q[j * 2 + part];
+            for (int i = 0; i < 16; ++i) {
+              const float2 f = __bfloat1622float2(row[i]);
+              v[2 * i] = f.x;
+              v[2 * i + 1] = f.y;
+              amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+            const uint32_t code = mx_scale_code(amax);
+            const float inv = mx_inv_scale(code);
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              w[i] = static_cast<uint32_t>(to_e4m3(v[4 * i] * inv)) |
+                     (static_cast<uint32_t>(to_e4m3(v[4 * i + 1] * inv)) << 8) |
+                     (static_cast<uint32_t>(to_e4m3(v[4 * i + 2] * inv)) << 16) |
+                     (static_cast<uint32_t>(to_e4m3(v[4 * i + 3] * inv)) << 24);
+            const int64_t r = t.row0 + c0 + lane;
+            uint4* dst = reinterpret_cast<uint4*>(p.q_out[t.grp] + r * G.out_ld + f_base);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            p.q_sf[t.grp][sf_offset(r, f_base / 32, static_cast<int>(G.out_ld) / 32)] =
+                static_cast<uint8_t>(code);
           }
           __syncwarp();
           continue;

@@ -530,7 +530,7 @@ moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void*
     return grouped_mlp_tiles<192, kMXF8>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
                                          ws, s);
   if (is_nv(c))
-    return grouped_mlp_tiles<128, kNVF4>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
+    return grouped_mlp_tiles<192, kNVF4>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
                                          ws, s);
   if (expert_tile_n() == 128)
     return grouped_mlp_tiles<128, kBF16>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
