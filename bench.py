@@ -352,6 +352,7 @@ def run_ours(args, cfg):
     steps_ms = {"route": [], "quantize": [], "permute": [], "grouped_mlp": [], "combine": []}
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     for it in range(args.warmup + args.steps):
+        torch.cuda.nvtx.range_push("moe_step")
         evs[0].record(stream)
         M.moe_route(c, x, d["w_router"], d["bias"], idx, tw, wsp, logits_out=logits)
         evs[1].record(stream)
@@ -367,6 +368,7 @@ def run_ours(args, cfg):
         evs[4].record(stream)
         M.moe_combine(c, out_rows, token_row, tw, y, shared_out=shared_out)
         evs[5].record(stream)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         if it >= args.warmup:
             for i, k in enumerate(steps_ms):
@@ -436,10 +438,16 @@ def main():
     ap.add_argument("--config", default=BENCH_CONFIG, choices=sorted(synth.CONFIGS))
     ap.add_argument("--ref-tokens", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling only: scale the workload to this many experts, keeping "
+                         "the rows per expert (T scales with E)")
     ap.add_argument("--soak-s", type=float, default=1.5,
                     help="untimed graph replays before the timed region (clock sampling)")
     args = ap.parse_args()
     cfg = synth.get_config(args.config)
+    if args.experts:
+        t = max(1, round(cfg.T * args.experts / cfg.E))
+        cfg = cfg.scaled(E=args.experts, T=t, name=f"{cfg.name}_E{args.experts}_T{t}")
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

@@ -58,8 +58,8 @@ typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1, MOE_NVFP4 = 2 } moe_dtype;
  * Supported: 1 <= T; H, I, I_shared multiples of 128; 1 <= E <= 1024;
  * E % n_group == 0 with E/n_group >= 2 and n_group <= 32; 1 <= topk_group <=
  * n_group; 1 <= top_k <= min(32, topk_group*E/n_group); pad_multiple >= 1
- * (MXFP8: pad_multiple == 128).  dtype MOE_NVFP4 is not built yet: the data
- * calls return MOE_ERR_UNSUPPORTED for it (routing works for every dtype).
+ * (MXFP8, NVFP4: pad_multiple % 64 == 0; NVFP4 also needs H, I, I_shared
+ * multiples of 256).
  */
 typedef struct moe_config {
   int32_t T, H, I, E;
@@ -83,7 +83,12 @@ typedef struct moe_config {
  *   MXFP8: the same tile-major layout over bytes (128 rows x 128 e4m3 codes
  *   per 16 KB tile), and *_scales hold the e8m0 scales per 32 K elements in
  *   the MMA scale layout of moe_quantize over the same rows (w1_scales for
- *   the E*I rows of w1, ...).  The *_global fields are reserved for NVFP4.
+ *   the E*I rows of w1, ...).
+ *   NVFP4: the same tile-major byte layout over packed e2m1 codes (a 16 KB
+ *   tile holds 128 rows x 256 elements), *_scales the e4m3 scales per 16 K
+ *   elements in the MMA scale layout, and the fp32 global encode scales:
+ *   w13_global [E] (W1_e and W3_e share one, as one stacked fc1 tensor),
+ *   w2_global [E], ws13_global [1], ws2_global [1].  Unused otherwise.
  * Shared-expert fields are ignored when I_shared == 0.
  */
 typedef struct moe_weights {
@@ -126,9 +131,15 @@ moe_status moe_prepared_weights_size(const moe_config* cfg, moe_weight_sizes* si
  *   Scale layout ("MMA scale layout"): for a matrix with KB = cols/32 blocks
  *   per row, the scale of (row r, block kb) is at byte
  *     ((r/128)*(KB/4) + kb/4)*512 + (r%32)*16 + ((r%128)/32)*4 + kb%4,
- *   so `scales` holds ceil(rows/128)*128*KB bytes.
- *   dtype MOE_NVFP4: not built yet (MOE_ERR_UNSUPPORTED).  global_scale is
- *   reserved for it.
+ *   so `scales` holds ceil(rows/128)*128*KB bytes.  global_scale unused.
+ *   dtype MOE_NVFP4 (sglang PR "Mistral Large 3 NVFP4 TRTLLM MoE support",
+ *   Modifications: W4A4 NVFP4): *global_scale (device fp32, written) =
+ *   2688 / amax over the whole matrix (1 when amax == 0); per 16 consecutive
+ *   elements of a row, the e4m3 block scale sb = e4m3((amax16 / 6) * g) and
+ *   codes e2m1(v * (g / sb)) (each step one fp32 operation, nearest-even,
+ *   saturating; a zero sb gives zero codes).  codes [rows, cols/2] bytes, two
+ *   e2m1 codes per byte, element 2i in the low nibble; scales in the MMA scale
+ *   layout with KB = cols/16.  cols % 256 == 0.
  */
 moe_status moe_quantize(int32_t dtype, const void* in, int32_t rows, int32_t cols, void* codes,
                         void* scales, float* global_scale, void* stream);
@@ -176,11 +187,13 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_router,
  *   counts rounded up to pad_multiple.  row_token [r_cap] int32: token of each
  *   row, -1 for pad rows and rows past offsets[E].  token_row [T*top_k] int32:
  *   row of (t, j).  Within a segment tokens ascend.
- *   src_rows: bf16 x [T, H] (BF16) or e4m3 codes [T, H] (MXFP8, from
- *   moe_quantize).  dst_rows [r_cap, same row bytes]; pad rows zero.
- *   src_scales / dst_scales (MXFP8): block scales in the MMA scale layout of
- *   moe_quantize, for T and r_cap rows; pad rows get zero scale bytes.  NULL
- *   for BF16.
+ *   src_rows: bf16 x [T, H] (BF16) or codes from moe_quantize (MXFP8 e4m3
+ *   [T, H], NVFP4 packed e2m1 [T, H/2]).  dst_rows [r_cap, same row bytes];
+ *   pad rows zero.  dst_rows may be NULL: no row is copied (moe_grouped_mlp
+ *   can gather the rows itself) and src_rows is then not read.
+ *   src_scales / dst_scales (MXFP8, NVFP4): block scales in the MMA scale
+ *   layout of moe_quantize, for T and r_cap rows; pad rows get zero scale
+ *   bytes.  NULL for BF16.
  */
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx,
                        const void* src_rows, const void* src_scales,
@@ -224,10 +237,19 @@ moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx,
  *   h = bf16(silu(X_e W1_e^T) * (X_e W3_e^T));  out = bf16(h W2_e^T),
  * and the same for the shared expert on all T tokens of x.
  *   rows [r_cap, H] (as moe_permute's dst_rows), counts/offsets from
- *   moe_permute; x [T, H] in token order (shared expert input; may be NULL
- *   when I_shared == 0).  MXFP8: rows and x are e4m3 codes, row_scales /
- *   x_scales their scales (MMA scale layout), and h is rounded to bf16 and
- *   quantized to MXFP8 before fc2.  x_global is reserved for NVFP4.
+ *   moe_permute; x [T, H] in token order (shared expert input).
+ *   rows may be NULL: fc1 then reads each expert's rows straight from x,
+ *   picking them by row_token [r_cap] (moe_permute's map) with 4-row TMA
+ *   gathers, so no expert-major copy of x is needed (saves r_cap * H * 2
+ *   bytes and the copy; on B200 the gathers stream rows more slowly than
+ *   32-row boxes, so at large batch this mode is the slower one).  row_token
+ *   is ignored when rows is given, and x may then be NULL if I_shared == 0.
+ *   MXFP8 / NVFP4: rows and x are codes from moe_quantize, row_scales /
+ *   x_scales their scales (MMA scale layout; row_scales as moe_permute's
+ *   dst_scales), and h is rounded to bf16 and quantized to the same format
+ *   before fc2.  NVFP4: x_global is x's global encode scale from
+ *   moe_quantize; h gets one global scale per expert (and one for the shared
+ *   expert) from the amax of that expert's h rows, computed on the device.
  *   out_rows [r_cap, H] bf16: fc2 output per row (rows of pads untouched).
  *   shared_out [T, H] bf16 or NULL when I_shared == 0.
  * Tensor-core kernels: tcgen05 MMA with TMEM accumulators fed by TMA.
@@ -236,7 +258,7 @@ moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w,
                            const void* rows, const void* row_scales,
                            const void* x, const void* x_scales, const float* x_global,
                            const int32_t* counts, const int32_t* offsets,
-                           void* out_rows, void* shared_out,
+                           const int32_t* row_token, void* out_rows, void* shared_out,
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*

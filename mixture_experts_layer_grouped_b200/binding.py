@@ -88,7 +88,8 @@ def lib() -> ctypes.CDLL:
             "moe_permute_noalloc": ([_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
                                     ctypes.c_int),
             "moe_grouped_mlp": ([_CFG, ctypes.POINTER(MoEWeights), _VP, _VP, _VP, _VP, _VP,
-                                 _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
+                                 _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP],
+                                ctypes.c_int),
             "moe_combine": ([_CFG, _VP, _VP, _VP, _VP, _VP, _VP], ctypes.c_int),
             "moe_forward": ([_CFG, ctypes.POINTER(MoEWeights), _VP, _VP, _VP, _VP,
                              ctypes.c_int32, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
@@ -252,13 +253,15 @@ def prepare_weights(cfg, raw: dict, stream=None) -> dict:
 
 def moe_grouped_mlp(cfg, weights, rows, counts, offsets, out_rows, workspace, x=None,
                     shared_out=None, row_scales=None, x_scales=None, x_global=None,
-                    stream=None):
+                    row_token=None, stream=None):
+    """rows=None: fc1 gathers each expert's rows from x through row_token."""
     ws = weights if isinstance(weights, MoEWeights) else weights_struct(weights)
     i32 = torch.int32
     _check("moe_grouped_mlp", lib().moe_grouped_mlp(
         ctypes.byref(cfg), ctypes.byref(ws), _p(rows), _p(row_scales), _p(x), _p(x_scales),
         _p(x_global), _p(_cuda(counts, i32, "counts")), _p(_cuda(offsets, i32, "offsets")),
-        _p(out_rows), _p(shared_out), _p(workspace), workspace.numel(), _stream(stream)))
+        _p(_cuda(row_token, i32, "row_token")), _p(out_rows), _p(shared_out), _p(workspace),
+        workspace.numel(), _stream(stream)))
 
 
 def moe_combine(cfg, out_rows, token_row, topk_w, y, shared_out=None, stream=None):

@@ -385,3 +385,60 @@ __device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// Exclusive scan of ceil(counts[e] / P) * P over e < E into s_out[0..E]
+// (E <= 1024), by a block of exactly 256 threads.
+__device__ __forceinline__ void block_scan_padded(const int32_t* counts, int E, int P,
+                                                  int32_t* s_out) {
+  __shared__ int32_t warp_tot[8];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  constexpr int PER = 4;
+  int v[PER];
+  int local = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = tid * PER + i;
+    const int c = e < E ? counts[e] : 0;
+    v[i] = (c + P - 1) / P * P;
+    local += v[i];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  int run = incl - local;
+  for (int i = 0; i < w; ++i) run += warp_tot[i];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = tid * PER + i;
+    if (e <= E) s_out[e] = run;
+    run += v[i];
+  }
+  if (tid == 255 && E == 4 * 256) s_out[E] = run;
+  __syncthreads();
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// Four rows of a 2-D tensor (row indices r0..r3, one 128-byte box row each)
+// into consecutive shared-memory rows; out-of-range rows read as zeros.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t r0, int32_t r1, int32_t r2,
+                                            int32_t r3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3), "l"(policy)
+      : "memory");
+}
+
+}  // namespace moe

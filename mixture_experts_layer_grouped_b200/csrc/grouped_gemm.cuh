@@ -69,6 +69,9 @@ struct GemmParams {
   int32_t gw_stride[2];
   float* amax_out[2];       // fc1 NVFP4: per-expert amax of h (atomic max)
   int32_t amax_stride[2];
+  // routed token rows gathered straight from token-order x: b[0] is then a map
+  // over x with one-row boxes, and tile row j is x[row_token[row0 + j]]
+  const int32_t* row_token;
   // fc1 with quantized output: h codes [rows, ld] and scales (MMA layout, KB = ld/32)
   uint8_t* q_out[2];
   uint8_t* q_sf[2];
@@ -92,10 +95,12 @@ struct GemmCfg {
   static constexpr int B_BYTES = TILE_N * 128;
   static constexpr int SF_CHUNK = 512;                          // one 128x4 scale chunk
   static constexpr int SF_KCH = (DT == kNVF4) ? 4 : 1;          // scale chunks per k-step
-  // token row chunks of scales: a tile starts at a row that is a multiple of 32
-  // (segments are 128-aligned, tiles TILE_N apart), so it spans at most
-  // ceil((TILE_N + 96) / 128) chunks
-  static constexpr int SFB_CHUNKS = (TILE_N + 96 + 127) / 128;
+  // token row chunks of scales: a tile starts at a row that is a multiple of 64
+  // (segments are 64-aligned, tiles TILE_N apart, TILE_N % 64 == 0), so it spans
+  // at most ceil((TILE_N + 64) / 128) chunks.  (The MMA's scale address must sit
+  // on an even TMEM column: the base shifts by (row0 % 128) / 32, i.e. 0 or 2.)
+  static_assert(DT == kBF16 || TILE_N % 64 == 0, "block-scaled tiles are 64-row multiples");
+  static constexpr int SFB_CHUNKS = (TILE_N + 64 + 127) / 128;
   static constexpr int SF_BYTES = (DT != kBF16) ? (NA + SFB_CHUNKS) * SF_KCH * SF_CHUNK : 0;
   static constexpr int STAGE_BYTES = (NA * A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
   static constexpr int RING = (DT == kNVF4) ? 198 * 1024 : kRingBytes;
@@ -104,7 +109,10 @@ struct GemmCfg {
   static constexpr int SF_COLS = (DT != kBF16) ? 4 * SF_KCH * (NA + SFB_CHUNKS) : 0;
   static constexpr int ACC_BUFS = (2 * ACC_COLS + SF_COLS <= 512) ? 2 : 1;
   static constexpr int SF_TMEM = ACC_BUFS * ACC_COLS;  // first scale-factor column
-  static constexpr uint32_t TMEM_COLS = pow2_at_least(ACC_BUFS * ACC_COLS + SF_COLS);
+  // scale factors alternate between two TMEM regions by stage when they fit, so
+  // the copies of stage s+1 do not overwrite columns stage s's MMAs still read
+  static constexpr int SF_BUFS = (SF_COLS > 0 && ACC_BUFS * ACC_COLS + 2 * SF_COLS <= 512) ? 2 : 1;
+  static constexpr uint32_t TMEM_COLS = pow2_at_least(ACC_BUFS * ACC_COLS + SF_BUFS * SF_COLS);
   static constexpr int SLAB_ROWS = (MODE == kFc2) ? 2 * kBM : kBM;  // features per tile
   static constexpr int STG_WARP = 32 * 34 * 2;                 // per warp 32 x 34 bf16
   static constexpr int STG_BYTES = kEpiWarps * STG_WARP;
@@ -243,9 +251,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
                               : 0;
   const int units = units_routed + units_dense;
 
+  // gathered token rows: the whole producer warp issues the row gathers
+  const bool warp_loads = (MODE == kFc1) && p.row_token != nullptr;
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
+    // ---------------- TMA producer (lane 0, or the whole warp when gathering) ----
+    if (lane == 0 || warp_loads) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
       int stage = 0;
@@ -256,6 +266,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const Tile t = decode_tile<MODE, TILE_N>(u, p, prefix, units_routed);
+        const bool gather = (MODE == kFc1) && t.grp == 0 && p.row_token != nullptr;
+        // gathered rows: lane l owns tile rows [8l, 8l + 8); rows past the MMA's N
+        // are not loaded, and rows between the tile's tokens and N repeat its first
+        // token (those accumulator columns are never stored)
+        const int n_load = (t.n_tok + 15) & ~15;
+        int ids[8];
+        if (gather) {
+          const int first = __ldg(p.row_token + t.row0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int j = lane * 8 + i;
+            ids[i] = j < t.n_tok ? __ldg(p.row_token + t.row0 + j) : first;
+          }
+        }
         const int nbox = (t.n_tok + kBoxRows - 1) / kBoxRows;
         const int nsfb = ((t.row0 & 127) + t.n_tok + 127) / 128;
         // fc2's second 128-row slab may lie past the expert's last row (odd number of
@@ -264,12 +288,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         const bool slab1 = (MODE != kFc2) ||
                            (t.slab * C::SLAB_ROWS + kBM < p.g[t.grp].a_valid_rows);
         const int n_sfa = (MODE == kRouter) ? 1 : (slab1 ? 2 : 1);
-        const uint32_t bytes = C::NA * C::A_BYTES + nbox * kBoxRows * 128 +
+        const uint32_t bytes = C::NA * C::A_BYTES + (gather ? n_load : nbox * kBoxRows) * 128 +
                                (DT != kBF16 ? (n_sfa + nsfb) * C::SF_KCH * C::SF_CHUNK : 0);
         for (int kt = t.k_begin; kt < t.k_end; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          // lane 0 waits and sets the expected bytes; the decision is shared so the
+          // warp stays converged
+          int okw = 1;
+          if (lane == 0) {
+            okw = mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status) ? 1 : 0;
+            if (okw) mbar_arrive_expect_tx(&full[stage], bytes);
+          }
+          if (warp_loads) okw = __shfl_sync(0xffffffffu, okw, 0);
+          if (!okw) { ok = false; break; }
           uint8_t* sa = ring + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], bytes);
+          if (gather) {
+            uint8_t* sbg = sa + C::NA * C::A_BYTES;
+            const int col = kt * (DT == kBF16 ? kBK : 128);
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              const int j = lane * 8 + g * 4;
+              if (j < n_load)
+                tma_gather4(sbg + j * 128, &p.b[0], &full[stage], col, ids[4 * g],
+                            ids[4 * g + 1], ids[4 * g + 2], ids[4 * g + 3], pol_x);
+            }
+          }
+          if (lane != 0) {
+            if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+            continue;
+          }
           if (MODE == kRouter) {
             tma_load_2d(sa, &p.a0[t.grp], &full[stage], kt * kBK, t.a_row, pol_w);
           } else {
@@ -284,9 +330,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
                           pol_w);
           }
           uint8_t* sb = sa + C::NA * C::A_BYTES;
-          for (int bx = 0; bx < nbox; ++bx)
-            tma_load_2d(sb + bx * kBoxRows * 128, &p.b[t.grp], &full[stage],
-                        kt * (DT == kBF16 ? kBK : 128), t.row0 + bx * kBoxRows, pol_x);
+          if (!gather)
+            for (int bx = 0; bx < nbox; ++bx)
+              tma_load_2d(sb + bx * kBoxRows * 128, &p.b[t.grp], &full[stage],
+                          kt * (DT == kBF16 ? kBK : 128), t.row0 + bx * kBoxRows, pol_x);
           if (DT != kBF16) {
             // scale chunks of this k-step (SF_KCH consecutive chunks per 128-row chunk):
             // A rows [a_row, +128) (and the second operand), then the token row chunks
@@ -362,7 +409,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             // sits at sf_b + 4 * (kk * SFB_CHUNKS + cb)
             constexpr uint32_t cb_bytes = C::SF_KCH * C::SF_CHUNK;
             const uint32_t ssf = sb + C::B_BYTES;
-            const uint32_t sf_a0 = tmem_base + C::SF_TMEM;
+            const uint32_t sf_a0 = tmem_base + C::SF_TMEM + (C::SF_BUFS == 2 ? (kt & 1) : 0) * C::SF_COLS;
             const uint32_t sf_a1 = sf_a0 + 4 * C::SF_KCH;
             const uint32_t sf_b = sf_a0 + 4 * C::SF_KCH * C::NA;
 #pragma unroll
@@ -387,7 +434,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
           } else {
             // scale factors of this stage: smem -> TMEM (in order with the MMAs below)
             const uint32_t ssf = sb + C::B_BYTES;
-            const uint32_t sf_a0 = tmem_base + C::SF_TMEM;
+            const uint32_t sf_a0 = tmem_base + C::SF_TMEM + (C::SF_BUFS == 2 ? (kt & 1) : 0) * C::SF_COLS;
             const uint32_t sf_a1 = sf_a0 + 4;
             const uint32_t sf_b = sf_a0 + 4 * C::NA;
             tmem_cp_sf_chunk(sf_a0, sdesc_sf_chunk(ssf));

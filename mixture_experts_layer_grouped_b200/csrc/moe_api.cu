@@ -34,17 +34,18 @@ struct StepLayout {
   int32_t r_cap, ntiles, router_splits;
 };
 
-constexpr int kRouterTileN = 64;
+// Router GEMM tiling: 256-token tiles for long batches (W_r re-read per tile
+// is then negligible), 64 otherwise; K split into at most kMaxSplits parts so
+// that about one wave of tiles covers the SMs.
+int router_tile_of(const moe_config& c) { return c.T >= 4096 ? 256 : 64; }
 
-// K splits of the router GEMM: enough tiles for about two per SM, at least
-// four k-steps per split, at most 32 splits.
 int router_splits_of(const moe_config& c) {
-  const int chunks = (c.T + kRouterTileN - 1) / kRouterTileN;
-  const int slabs = (c.E + kBM - 1) / kBM;
+  const int tn = router_tile_of(c);
+  const int units = ((c.T + tn - 1) / tn) * ((c.E + kBM - 1) / kBM);
   const int k_tiles = c.H / kBK;
-  int s = (2 * 148 + chunks * slabs - 1) / (chunks * slabs);
+  int s = (148 + units - 1) / units;
+  s = s < kMaxSplits ? s : kMaxSplits;
   s = s < k_tiles / 4 ? s : k_tiles / 4;
-  s = s < 32 ? s : 32;
   return s < 1 ? 1 : s;
 }
 
@@ -134,11 +135,12 @@ moe_status check_config(const moe_config* c) {
   return MOE_OK;
 }
 
-// Block-scaled paths keep 128-row scale chunks aligned with expert segments
-// (pad_multiple must be 128); NVFP4 k-steps are 256 elements wide.
+// Block-scaled paths need expert segments to start on 64-row boundaries: the
+// GEMM shifts its TMEM scale base by (row % 128) / 32 columns, and that address
+// must be even.  So pad_multiple % 64 == 0.  NVFP4 k-steps are 256 wide.
 moe_status check_dtype(const moe_config* c) {
   if (c->dtype == MOE_BF16) return MOE_OK;
-  if (c->pad_multiple != 128) return MOE_ERR_UNSUPPORTED;
+  if (c->pad_multiple % 64) return MOE_ERR_UNSUPPORTED;
   if (c->dtype == MOE_NVFP4 && (c->H % 256 || c->I % 256 || c->I_shared % 256))
     return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
@@ -292,8 +294,10 @@ moe_status do_route(const moe_config& c, const void* x, const void* w_router, co
     p.E = 0;
     p.dense_rows = c.T;
     p.status = status_ptr(ws);
-    const int units = ((c.T + kRouterTileN - 1) / kRouterTileN) * g.n_slabs * g.k_splits;
-    MOE_TRY((launch_gemm<kRouter, kRouterTileN, kBF16>(p, units, s)));
+    const int tn = router_tile_of(c);
+    const int units = ((c.T + tn - 1) / tn) * g.n_slabs * g.k_splits;
+    if (tn == 256) MOE_TRY((launch_gemm<kRouter, 256, kBF16>(p, units, s)));
+    else MOE_TRY((launch_gemm<kRouter, 64, kBF16>(p, units, s)));
     a.partials = partials;
     a.n_splits = L.router_splits;
     a.logits_out = logits_out;
@@ -344,9 +348,9 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
   const size_t hsm = static_cast<size_t>(c.E) * 4;
   permute_hist_kernel<<<L.ntiles, 256, hsm, s>>>(a);
   MOE_TRY(launch_check());
-  permute_scan_kernel<<<1, 1024, 0, s>>>(a);
+  permute_scan_kernel<<<(c.E + 7) / 8, 256, 0, s>>>(a);
   MOE_TRY(launch_check());
-  permute_rank_kernel<<<L.ntiles, 32, hsm, s>>>(a);
+  permute_rank_kernel<<<L.ntiles, 256, 0, s>>>(a);
   MOE_TRY(launch_check());
   if (is_mx(c) || is_nv(c)) {
     GatherMxArgs g;
@@ -362,6 +366,7 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
     else permute_gather_mx_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
     return launch_check();
   }
+  if (!dst_rows) return MOE_OK;  // rows are gathered later by the grouped GEMM
   GatherArgs g;
   g.src = static_cast<const uint8_t*>(src_rows);
   g.dst = static_cast<uint8_t*>(dst_rows);
@@ -378,7 +383,8 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
 struct MlpQuant {
   const void* row_scales;
   const void* x_scales;
-  const float* x_global;  // NVFP4 global encode scale of x
+  const float* x_global;     // NVFP4 global encode scale of x
+  const int32_t* row_token;  // with rows == nullptr: fc1 gathers token rows from x
 };
 
 template <int TILE_N, int DT>
@@ -409,7 +415,13 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     memset(&p, 0, sizeof(p));
     MOE_TRY(make_tiled_map(&p.a0[0], w.w1, E * I, kbytes(H)));
     MOE_TRY(make_tiled_map(&p.a1[0], w.w3, E * I, kbytes(H)));
-    MOE_TRY(make_map(&p.b[0], rows, tok_t, me, kbytes(H) / me, L.r_cap, kbytes(H), kBoxRows));
+    if (rows) {
+      MOE_TRY(make_map(&p.b[0], rows, tok_t, me, kbytes(H) / me, L.r_cap, kbytes(H), kBoxRows));
+    } else {
+      // gathered: one-row boxes over token-order x, rows picked by row_token
+      MOE_TRY(make_map(&p.b[0], x, tok_t, me, kbytes(H) / me, c.T, kbytes(H), 1));
+      p.row_token = q.row_token;
+    }
     if (sh) {
       MOE_TRY(make_tiled_map(&p.a0[1], w.ws1, Is, kbytes(H)));
       MOE_TRY(make_tiled_map(&p.a1[1], w.ws3, Is, kbytes(H)));
@@ -462,12 +474,12 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
   if (nv) {
     amax_to_global_kernel<<<(c.E + 1 + 255) / 256, 256, 0, s>>>(g_h, c.E + 1);
     MOE_TRY(launch_check());
-    quantize_h_nvfp4_kernel<<<sm_count() * 4, 256, (c.E + 1) * 4, s>>>(
+    quantize_h_nvfp4_kernel<<<sm_count() * 4, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(h), wsb + L.h_q, wsb + L.h_sf, c.I, offsets, counts,
         c.E, g_h, 0);
     MOE_TRY(launch_check());
     if (sh) {
-      quantize_h_nvfp4_kernel<<<sm_count() * 2, 256, (c.E + 1) * 4, s>>>(
+      quantize_h_nvfp4_kernel<<<sm_count() * 2, 256, 0, s>>>(
           static_cast<const __nv_bfloat16*>(hs), wsb + L.h_shared_q, wsb + L.h_shared_sf,
           c.I_shared, offsets, counts, c.E, g_h + c.E, c.T);
       MOE_TRY(launch_check());
@@ -634,9 +646,9 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
   MOE_TRY(check_config(cfg));
   MOE_TRY(check_dtype(cfg));
   MOE_TRY(check_ws(*cfg, workspace, workspace_bytes));
-  if (!topk_idx || !src_rows || !counts || !offsets || !row_token || !token_row || !dst_rows)
+  if (!topk_idx || !counts || !offsets || !row_token || !token_row) return MOE_ERR_INVALID_ARG;
+  if (dst_rows && (!src_rows || !aligned16(src_rows) || !aligned16(dst_rows)))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned16(src_rows) || !aligned16(dst_rows)) return MOE_ERR_INVALID_ARG;
   if (!is_bf16(*cfg) && (!src_scales || !dst_scales || !aligned16(src_scales) ||
                          !aligned16(dst_scales)))
     return MOE_ERR_INVALID_ARG;
@@ -647,14 +659,14 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
 moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w, const void* rows,
                            const void* row_scales, const void* x, const void* x_scales,
                            const float* x_global, const int32_t* counts, const int32_t* offsets,
-                           void* out_rows, void* shared_out, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+                           const int32_t* row_token, void* out_rows, void* shared_out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
   MOE_TRY(check_config(cfg));
   MOE_TRY(check_dtype(cfg));
   MOE_TRY(check_ws(*cfg, workspace, workspace_bytes));
   MOE_TRY(check_weights(*cfg, w));
-  if (!rows || !counts || !offsets || !out_rows) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(rows) || !aligned16(out_rows)) return MOE_ERR_INVALID_ARG;
+  if (!counts || !offsets || !out_rows || !aligned16(out_rows)) return MOE_ERR_INVALID_ARG;
+  if (rows ? !aligned16(rows) : (!row_token || !x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
   if (cfg->I_shared > 0 && (!x || !shared_out || !aligned16(x) || !aligned16(shared_out)))
     return MOE_ERR_INVALID_ARG;
   if (!is_bf16(*cfg)) {
@@ -668,7 +680,7 @@ moe_status moe_grouped_mlp(const moe_config* cfg, const moe_weights* w, const vo
     if (!x_global || !w->w13_global || !w->w2_global) return MOE_ERR_INVALID_ARG;
     if (cfg->I_shared > 0 && (!w->ws13_global || !w->ws2_global)) return MOE_ERR_INVALID_ARG;
   }
-  MlpQuant q{row_scales, x_scales, x_global};
+  MlpQuant q{row_scales, x_scales, x_global, rows ? nullptr : row_token};
   return do_grouped_mlp(*cfg, *w, rows, x, q, counts, offsets, out_rows, shared_out, workspace,
                         static_cast<cudaStream_t>(stream));
 }
@@ -889,18 +901,20 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   int32_t* offsets = reinterpret_cast<int32_t*>(b + F.offsets);
   int32_t* row_token = reinterpret_cast<int32_t*>(b + F.row_token);
   int32_t* token_row = reinterpret_cast<int32_t*>(b + F.token_row);
-  void* rows = b + F.rows;
   void* out_rows = b + F.out_rows;
   void* shared_out = c.I_shared > 0 ? b + F.shared_out : nullptr;
   MOE_TRY(do_route(c, xd, w_router, bias, nullptr, logits, topk_idx, topk_w, workspace, s));
   const void* xq = xd;
-  MlpQuant q{nullptr, nullptr, nullptr};
+  MlpQuant q{nullptr, nullptr, nullptr, nullptr};
   if (!is_bf16(c)) {
     float* xg = reinterpret_cast<float*>(b + F.x_g);
     MOE_TRY(moe_quantize(c.dtype, xd, c.T, c.H, b + F.x_q, b + F.x_sf, xg, s));
     xq = b + F.x_q;
-    q = MlpQuant{b + F.rows_sf, b + F.x_sf, xg};
+    q = MlpQuant{b + F.rows_sf, b + F.x_sf, xg, nullptr};
   }
+  // an expert-major copy of the rows: fc1 reads it with 32-row TMA boxes, which
+  // streams faster than per-row gathers from x (moe_grouped_mlp with rows == NULL)
+  void* rows = b + F.rows;
   MOE_TRY(do_permute(c, topk_idx, xq, q.x_scales, counts, offsets, row_token, token_row, rows,
                      b + F.rows_sf, workspace, s));
   MOE_TRY(do_grouped_mlp(c, *w, rows, xq, q, counts, offsets, out_rows, shared_out, workspace,
@@ -1006,9 +1020,9 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   const size_t hsm = static_cast<size_t>(c.E) * 4;
   permute_hist_kernel<<<L.ntiles, 256, hsm, s>>>(a);
   MOE_TRY(launch_check());
-  permute_scan_kernel<<<1, 1024, 0, s>>>(a);
+  permute_scan_kernel<<<(c.E + 7) / 8, 256, 0, s>>>(a);
   MOE_TRY(launch_check());
-  permute_rank_kernel<<<L.ntiles, 32, hsm, s>>>(a);
+  permute_rank_kernel<<<L.ntiles, 256, 0, s>>>(a);
   MOE_TRY(launch_check());
   GatherArgs g;
   g.src = static_cast<const uint8_t*>(src_rows);

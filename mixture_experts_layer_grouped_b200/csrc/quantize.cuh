@@ -121,12 +121,14 @@ __global__ void __launch_bounds__(256) permute_gather_mx_kernel(GatherMxArgs a) 
     uint4* d = reinterpret_cast<uint4*>(a.dst_codes + static_cast<int64_t>(r) * a.H);
     if (t >= 0) {
       const uint4* s = reinterpret_cast<const uint4*>(a.src_codes + static_cast<int64_t>(t) * a.H);
-      for (int v = lane; v < vecs; v += 32) d[v] = __ldg(s + v);
+      if (a.dst_codes)
+        for (int v = lane; v < vecs; v += 32) d[v] = __ldg(s + v);
       for (int w = lane; w < W; w += 32)
         *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) =
             *reinterpret_cast<const uint32_t*>(a.src_scales + sf_offset(t, 4 * w, KB));
     } else {
-      for (int v = lane; v < vecs; v += 32) d[v] = make_uint4(0, 0, 0, 0);
+      if (a.dst_codes)
+        for (int v = lane; v < vecs; v += 32) d[v] = make_uint4(0, 0, 0, 0);
       for (int w = lane; w < W; w += 32)
         *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) = 0u;
     }
@@ -223,45 +225,47 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(
   scales[sf_offset(r, kb, KB)] = static_cast<uint8_t>(sb);
 }
 
-// NVFP4 quantization of the fc2 input h (bf16, expert-major rows): the row's
-// expert e comes from the segment offsets; global scale g_h[e]; pad rows
-// (past counts[e] in their segment) get zero codes and scales.  `dense` > 0
-// quantizes `dense` token-order rows with g_h[0] instead (shared expert).
+// NVFP4 quantization of the fc2 input h (bf16, expert-major rows), over the
+// rows that hold a token: valid row v (in expert order) is row
+// offsets[e] + v - cnt_prefix[e] of expert e, whose global scale is g_h[e].
+// Pad rows are left as they are (their outputs are masked).  One warp per
+// row.  `dense` > 0 quantizes `dense` token-order rows with g_h[0] instead.
 __global__ void __launch_bounds__(256) quantize_h_nvfp4_kernel(
     const __nv_bfloat16* __restrict__ h, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, int cols, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ counts, int E, const float* __restrict__ g_h, int dense) {
-  extern __shared__ int32_t s_off[];  // [E + 1]
-  if (!dense)
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
-  __syncthreads();
+  __shared__ int32_t s_cpre[1025];
   const int KB = cols / 16;
-  const int64_t rows = dense ? dense : s_off[E];
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t blk = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; blk < rows * KB;
-       blk += stride) {
-    const int64_t r = blk / KB;
-    const int kb = static_cast<int>(blk - r * KB);
+  int64_t n_rows = dense;
+  if (!dense) {
+    block_scan_padded(counts, E, 1, s_cpre);
+    n_rows = s_cpre[E];
+  }
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t vr = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       vr < n_rows; vr += warps) {
+    int64_t r = vr;
     int e = 0;
-    bool pad = false;
     if (!dense) {
-      int lo = 0, hi = E;  // s_off[lo] <= r < s_off[lo+1]
+      int lo = 0, hi = E;  // s_cpre[lo] <= vr < s_cpre[lo + 1]
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (s_off[mid] <= r) lo = mid; else hi = mid;
+        if (s_cpre[mid] <= vr) lo = mid; else hi = mid;
       }
       e = lo;
-      pad = (r - s_off[e]) >= counts[e];
+      r = __ldg(offsets + e) + (vr - s_cpre[e]);
     }
-    uint32_t packed[2] = {0u, 0u};
-    uint32_t sb = 0u;
-    if (!pad) {
+    const float g = __ldg(g_h + e);
+    for (int kb = lane; kb < KB; kb += 32) {
       float v[16];
       load_bf16x16(h + r * cols + kb * 16, v);
-      sb = nv_quantize_block16(v, g_h[e], packed);
+      uint32_t packed[2];
+      const uint32_t sb = nv_quantize_block16(v, g, packed);
+      *reinterpret_cast<uint2*>(codes + r * (cols / 2) + kb * 8) =
+          make_uint2(packed[0], packed[1]);
+      scales[sf_offset(r, kb, KB)] = static_cast<uint8_t>(sb);
     }
-    *reinterpret_cast<uint2*>(codes + r * (cols / 2) + kb * 8) = make_uint2(packed[0], packed[1]);
-    scales[sf_offset(r, kb, KB)] = static_cast<uint8_t>(sb);
   }
 }
 
@@ -280,12 +284,14 @@ __global__ void __launch_bounds__(256) permute_gather_nv_kernel(GatherMxArgs a) 
     if (t >= 0) {
       const uint4* s =
           reinterpret_cast<const uint4*>(a.src_codes + static_cast<int64_t>(t) * row_bytes);
-      for (int v = lane; v < vecs; v += 32) d[v] = __ldg(s + v);
+      if (a.dst_codes)
+        for (int v = lane; v < vecs; v += 32) d[v] = __ldg(s + v);
       for (int w = lane; w < W; w += 32)
         *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) =
             *reinterpret_cast<const uint32_t*>(a.src_scales + sf_offset(t, 4 * w, KB));
     } else {
-      for (int v = lane; v < vecs; v += 32) d[v] = make_uint4(0, 0, 0, 0);
+      if (a.dst_codes)
+        for (int v = lane; v < vecs; v += 32) d[v] = make_uint4(0, 0, 0, 0);
       for (int w = lane; w < W; w += 32)
         *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) = 0u;
     }

@@ -19,6 +19,7 @@ constexpr int kMaxExpertsPerm = 1024;
 // (TransformerEngine PR "DeepSeekV3Layer", Description, DeepSeekV3MoE bullet.)
 // ---------------------------------------------------------------------------
 constexpr int kSelMaxPerLane = 32;  // E <= 1024
+constexpr int kMaxSplits = 4;       // router GEMM K splits summed by the selection
 constexpr int kSelWarps = 4;
 
 struct SelArgs {
@@ -60,9 +61,16 @@ __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(SelArgs a)
     if (e < a.E) {
       float l;
       if (a.n_splits > 0) {
-        // fixed summation order over the K splits: deterministic logits
-        l = a.partials[row + e];
-        for (int sp = 1; sp < a.n_splits; ++sp) l += a.partials[sp * split_stride + row + e];
+        // fixed summation order over the K splits (at most kMaxSplits): deterministic
+        // logits; all partial loads are issued before the additions
+        float part[kMaxSplits];
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplits; ++sp)
+          part[sp] = sp < a.n_splits ? a.partials[sp * split_stride + row + e] : 0.f;
+        l = part[0];
+#pragma unroll
+        for (int sp = 1; sp < kMaxSplits; ++sp)
+          if (sp < a.n_splits) l += part[sp];
         a.logits_out[row + e] = l;
       } else {
         l = a.logits[row + e];
@@ -165,80 +173,61 @@ __global__ void __launch_bounds__(256) permute_hist_kernel(PermArgs a) {
   }
   __syncthreads();
   for (int e = threadIdx.x; e < a.E; e += blockDim.x)
-    a.hist[static_cast<int64_t>(blockIdx.x) * a.E + e] = h[e];
+    a.hist[static_cast<int64_t>(e) * a.ntiles + blockIdx.x] = h[e];
 }
 
-// One block of 1024 threads.  Phase 1: a warp per expert turns that expert's
-// column of tile counts into exclusive tile bases (lanes over tiles, shuffle
-// scan).  Phase 2: thread e pads counts[e] and a block scan gives offsets.
-__global__ void __launch_bounds__(1024) permute_scan_kernel(PermArgs a) {
-  __shared__ int32_t warp_sums[32];
-  __shared__ int32_t s_cnt[kMaxExpertsPerm];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  for (int e = w; e < a.E; e += 32) {
-    int run = 0;
-    for (int b0 = 0; b0 < a.ntiles; b0 += 32) {
-      const int b = b0 + lane;
-      int32_t* p = a.hist + static_cast<int64_t>(b) * a.E + e;
-      const int v = (b < a.ntiles) ? *p : 0;
-      int incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-      }
-      if (b < a.ntiles) *p = run + incl - v;  // the tile's base rank for this expert
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) s_cnt[e] = run;
-  }
-  __syncthreads();
-  const int e = tid;
-  const int cnt = (e < a.E) ? s_cnt[e] : 0;
-  if (e < a.E) a.counts[e] = cnt;
-  const int padded = (e < a.E) ? (cnt + a.P - 1) / a.P * a.P : 0;
-  int incl = padded;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) warp_sums[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    const int ws = warp_sums[lane];
-    int wi = ws;
+// A warp per expert: exclusive scan of the expert's tile counts (hist row
+// [e][0..ntiles), contiguous) into tile bases, and counts[e].
+__global__ void __launch_bounds__(256) permute_scan_kernel(PermArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (e >= a.E) return;
+  int32_t* row = a.hist + static_cast<int64_t>(e) * a.ntiles;
+  int run = 0;
+  for (int b0 = 0; b0 < a.ntiles; b0 += 32) {
+    const int b = b0 + lane;
+    const int v = (b < a.ntiles) ? row[b] : 0;
+    int incl = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += v;
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
     }
-    warp_sums[lane] = wi - ws;
+    if (b < a.ntiles) row[b] = run + incl - v;  // the tile's base rank for this expert
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
-  __syncthreads();
-  const int off = warp_sums[w] + incl - padded;
-  if (e < a.E) {
-    a.offsets[e] = off;
-    for (int r = off + cnt; r < off + padded; ++r) a.row_token[r] = -1;
-  }
-  __shared__ int32_t s_total;
-  if (e == a.E - 1) {
-    a.offsets[a.E] = off + padded;
-    s_total = off + padded;
-  }
-  __syncthreads();
-  // rows past the last segment
-  for (int r = s_total + e; r < a.r_cap; r += blockDim.x) a.row_token[r] = -1;
+  if (lane == 0) a.counts[e] = run;
 }
 
-// One warp per tile, walking its entries in order.  The tile's indices and
-// the per-expert bases (tile base + segment offset) are loaded up front, so
-// the ordered walk touches shared memory only.
-__global__ void __launch_bounds__(32) permute_rank_kernel(PermArgs a) {
-  extern __shared__ int32_t run[];  // [E]: next free slot per expert
-  const int lane = threadIdx.x;
+// One block per tile.  Every block derives the padded segment offsets; block
+// 0 publishes them; all blocks mark pad rows and rows past the last segment
+// with -1 (a grid-stride pass over r_cap); then warp 0 walks the tile's
+// entries in order and assigns stable slots.
+__global__ void __launch_bounds__(256) permute_rank_kernel(PermArgs a) {
+  __shared__ int32_t s_off[kMaxExpertsPerm + 1];
+  __shared__ int32_t run[kMaxExpertsPerm];
+  block_scan_padded(a.counts, a.E, a.P, s_off);
+  const int tid = threadIdx.x;
+  if (blockIdx.x == 0)
+    for (int e = tid; e <= a.E; e += blockDim.x) a.offsets[e] = s_off[e];
+  const int total = s_off[a.E];
+  const int64_t gstride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + tid; r < a.r_cap; r += gstride) {
+    bool pad = r >= total;
+    if (!pad) {
+      int lo = 0, hi = a.E;  // s_off[lo] <= r < s_off[lo + 1]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_off[mid] <= r) lo = mid; else hi = mid;
+      }
+      pad = (r - s_off[lo]) >= a.counts[lo];
+    }
+    if (pad) a.row_token[r] = -1;
+  }
+  if (tid >= 32) return;
+  const int lane = tid;
   for (int e = lane; e < a.E; e += 32)
-    run[e] = a.offsets[e] + a.hist[static_cast<int64_t>(blockIdx.x) * a.E + e];
+    run[e] = s_off[e] + a.hist[static_cast<int64_t>(e) * a.ntiles + blockIdx.x];
   const int base = blockIdx.x * kPermTile;
   int ev[kPermTile / 32];
 #pragma unroll

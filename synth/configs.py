@@ -15,8 +15,8 @@ The six workloads are the routed-MoE shapes the method is exercised on:
   decode size (T=128) and a prefill size (T=8192).
 
 ``pad_multiple`` is the row multiple each expert segment is padded to in the
-expert-major layout.  The block-scaled paths keep scale factors in 128-row
-chunks, so they pad to 128; the bf16 path has no such constraint and pads to 8.
+expert-major layout: 64 for the block-scaled paths (whose scale chunks the
+GEMM addresses in 64-row steps), 8 for bf16.
 """
 
 from dataclasses import dataclass, field, asdict
@@ -74,15 +74,15 @@ CONFIGS = {
     "dsv3_mxfp8_shared_T4096": MoEShape(
         name="dsv3_mxfp8_shared_T4096", T=4096, H=7168, I=2048, E=256, n_group=8,
         topk_group=4, top_k=8, rsf=2.5, I_shared=2048, dtype="mxfp8",
-        pad_multiple=128, router_std=-1.0),
+        pad_multiple=64, router_std=-1.0),
     "dsv4_nvfp4_decode_T128": MoEShape(
         name="dsv4_nvfp4_decode_T128", T=128, H=7168, I=3072, E=384, n_group=8,
         topk_group=4, top_k=6, rsf=2.5, I_shared=0, dtype="nvfp4",
-        pad_multiple=128, router_std=-1.0),
+        pad_multiple=64, router_std=-1.0),
     "dsv4_nvfp4_prefill_T8192": MoEShape(
         name="dsv4_nvfp4_prefill_T8192", T=8192, H=7168, I=3072, E=384, n_group=8,
         topk_group=4, top_k=6, rsf=2.5, I_shared=0, dtype="nvfp4",
-        pad_multiple=128, router_std=-1.0),
+        pad_multiple=64, router_std=-1.0),
 }
 
 # The workload the throughput benchmark times: the mid-size bf16 layer.

@@ -93,7 +93,21 @@ def test_calls_reject_null_and_small_workspace(M):
                            ctypes.c_void_p((1 << 20) + 8), nb, None) == 1
     w = M.MoEWeights()
     assert lib.moe_grouped_mlp(ctypes.byref(c), ctypes.byref(w), fake, None, fake, None, None,
-                               fake, fake, fake, None, fake, nb, None) == 1
+                               fake, fake, None, fake, None, fake, nb, None) == 1
+    # gathered rows (rows == NULL) need row_token
+    wf = M.MoEWeights(w1=fake, w3=fake, w2=fake)
+    assert lib.moe_grouped_mlp(ctypes.byref(c), ctypes.byref(wf), None, None, fake, None, None,
+                               fake, fake, None, fake, None, fake, nb, None) == 1
     assert lib.moe_combine(ctypes.byref(c), None, fake, fake, None, fake, None) == 1
     assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), fake, fake, fake, fake, 0, fake, 16,
                            None) == 3
+
+
+def test_block_scaled_needs_64_row_padding(M):
+    s = synth.get_config("dsv3_mxfp8_shared_T4096").scaled(pad_multiple=32)
+    c = M.config_from_shape(s)
+    sizes = M.binding.MoEWeightSizes()
+    assert M.lib().moe_prepared_weights_size(ctypes.byref(c), ctypes.byref(sizes)) == 2
+    s = s.scaled(pad_multiple=64)
+    assert M.lib().moe_prepared_weights_size(ctypes.byref(M.config_from_shape(s)),
+                                             ctypes.byref(sizes)) == 0

@@ -18,7 +18,7 @@ MX = {
                                                        pad_multiple=128, I_shared=128),
     "ragged_mx": synth.MoEShape(name="ragged_mx", T=300, H=384, I=256, E=8, n_group=2,
                                 topk_group=1, top_k=2, rsf=1.0, I_shared=0, dtype="mxfp8",
-                                pad_multiple=128, router_std=0.05),
+                                pad_multiple=64, router_std=0.05),
     "hot_mx": synth.MoEShape(name="hot_mx", T=700, H=256, I=256, E=4, n_group=2, topk_group=2,
                              top_k=2, rsf=2.5, I_shared=128, dtype="mxfp8", pad_multiple=128,
                              router_std=0.02),
@@ -126,8 +126,9 @@ def test_permute_mxfp8(M, name):
     assert np.array_equal(sf_plain(rs, n, cfg.H // 32), ref_s)
 
 
-def _run_mlp(M, cfg, d, r):
-    """Quantize x, permute with the oracle's maps, grouped MLP on the GPU."""
+def _run_mlp(M, cfg, d, r, gather=False):
+    """Quantize x, permute with the oracle's maps, grouped MLP on the GPU.
+    gather=True: only the scales are permuted and fc1 gathers code rows from x."""
     c = M.config_from_shape(cfg)
     m = O.permute_maps(r["idx"], cfg.E, cfg.pad_multiple)
     nbytes, r_cap = M.moe_workspace_size(c)
@@ -139,27 +140,29 @@ def _run_mlp(M, cfg, d, r):
     counts, offsets = torch.empty(cfg.E, **i32), torch.empty(cfg.E + 1, **i32)
     row_token, token_row = torch.empty(r_cap, **i32), torch.empty(cfg.T * cfg.top_k, **i32)
     M.moe_permute(c, torch.from_numpy(r["idx"]).cuda(), xc, counts, offsets, row_token,
-                  token_row, rows, ws, src_scales=xs, dst_scales=rs)
+                  token_row, None if gather else rows, ws, src_scales=xs, dst_scales=rs)
     p = M.prepare_weights(c, weights_dict(d))
     out_rows = torch.zeros(r_cap, cfg.H, dtype=torch.bfloat16, device="cuda")
     shared_out = (torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
                   if cfg.I_shared else None)
-    M.moe_grouped_mlp(c, p, rows, counts, offsets, out_rows, ws, x=xc, shared_out=shared_out,
-                      row_scales=rs, x_scales=xs)
+    M.moe_grouped_mlp(c, p, None if gather else rows, counts, offsets, out_rows, ws, x=xc,
+                      shared_out=shared_out, row_scales=rs, x_scales=xs,
+                      row_token=row_token if gather else None)
     torch.cuda.synchronize()
     assert M.moe_get_device_status(ws) == 0
     return m, out_rows, shared_out
 
 
+@pytest.mark.parametrize("gather", [False, True], ids=["rows", "gather"])
 @pytest.mark.parametrize("name", list(MX))
-def test_grouped_mlp_mxfp8(M, name):
+def test_grouped_mlp_mxfp8(M, name, gather):
     cfg = MX[name]
     d = synth.gen_all(cfg, "cuda")
     if cfg.I_shared:
         d.update(zip(("ws1", "ws3", "ws2"), synth.gen_shared_weights(cfg, "cuda")))
     h = {k: f64(v) for k, v in d.items()}
     r = _routing(cfg)
-    m, out_rows, shared_out = _run_mlp(M, cfg, d, r)
+    m, out_rows, shared_out = _run_mlp(M, cfg, d, r, gather)
     xq = O.quantize_dequantize(h["x"], "mxfp8")
     xr = O.gather_rows(xq, m["row_token"])
     got = f64(out_rows)
@@ -172,6 +175,20 @@ def test_grouped_mlp_mxfp8(M, name):
     if cfg.I_shared:
         _, so = O.expert_forward(xq, h["ws1"], h["ws3"], h["ws2"], "mxfp8")
         assert rel_frob(f64(shared_out), so) < 2e-2
+
+
+@pytest.mark.parametrize("name", list(MX))
+def test_gathered_rows_give_the_same_bits_mxfp8(M, name):
+    """fc1 reading its rows from x through row_token computes exactly what it
+    computes on the permuted copy (same data, same MMA order)."""
+    cfg = MX[name]
+    d = synth.gen_all(cfg, "cuda")
+    if cfg.I_shared:
+        d.update(zip(("ws1", "ws3", "ws2"), synth.gen_shared_weights(cfg, "cuda")))
+    r = _routing(cfg)
+    _, a, _ = _run_mlp(M, cfg, d, r, False)
+    _, b, _ = _run_mlp(M, cfg, d, r, True)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
 @pytest.mark.parametrize("name", list(MX))

@@ -21,7 +21,7 @@ NV = {
                               router_std=0.02),
     "ragged_nv": synth.MoEShape(name="ragged_nv", T=300, H=512, I=256, E=8, n_group=2,
                                 topk_group=1, top_k=2, rsf=1.0, I_shared=0, dtype="nvfp4",
-                                pad_multiple=128, router_std=0.05),
+                                pad_multiple=64, router_std=0.05),
 }
 
 
@@ -132,8 +132,10 @@ def test_permute_nvfp4(M, name):
     assert np.array_equal(sf_plain(rs, n, cfg.H // 16), ref_s)
 
 
+@pytest.mark.parametrize("gather", [False, True], ids=["rows", "gather"])
 @pytest.mark.parametrize("name", list(NV))
-def test_grouped_mlp_nvfp4(M, name):
+def test_grouped_mlp_nvfp4(M, name, gather):
+    """gather=True: only the scales are permuted and fc1 gathers code rows from x."""
     cfg = NV[name]
     c = M.config_from_shape(cfg)
     d = synth.gen_all(cfg, "cuda")
@@ -149,13 +151,14 @@ def test_grouped_mlp_nvfp4(M, name):
     counts, offsets = torch.empty(cfg.E, **i32), torch.empty(cfg.E + 1, **i32)
     row_token, token_row = torch.empty(r_cap, **i32), torch.empty(cfg.T * cfg.top_k, **i32)
     M.moe_permute(c, torch.from_numpy(r["idx"]).cuda(), xc, counts, offsets, row_token,
-                  token_row, rows, ws, src_scales=xs, dst_scales=rs)
+                  token_row, None if gather else rows, ws, src_scales=xs, dst_scales=rs)
     p = M.prepare_weights(c, weights_dict(d))
     out_rows = torch.zeros(r_cap, cfg.H, dtype=torch.bfloat16, device="cuda")
     shared_out = (torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
                   if cfg.I_shared else None)
-    M.moe_grouped_mlp(c, p, rows, counts, offsets, out_rows, ws, x=xc, shared_out=shared_out,
-                      row_scales=rs, x_scales=xs, x_global=xg)
+    M.moe_grouped_mlp(c, p, None if gather else rows, counts, offsets, out_rows, ws, x=xc,
+                      shared_out=shared_out, row_scales=rs, x_scales=xs, x_global=xg,
+                      row_token=row_token if gather else None)
     torch.cuda.synchronize()
     assert M.moe_get_device_status(ws) == 0
     gx = O.nvfp4_global_scale(np.abs(h["x"]).max())

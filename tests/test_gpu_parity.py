@@ -153,8 +153,10 @@ def test_combine(M, name):
 
 
 # ---------------------------------------------------------------- grouped MLP
+@pytest.mark.parametrize("gather", [False, True], ids=["rows", "gather"])
 @pytest.mark.parametrize("name", BF16_CONFIGS + list(EDGE))
-def test_grouped_mlp(M, name):
+def test_grouped_mlp(M, name, gather):
+    """gather=True: fc1 reads token rows from x through row_token (rows=None)."""
     cfg = _cfg(name)
     c = M.config_from_shape(cfg)
     d = gen_device_inputs(cfg)
@@ -172,8 +174,12 @@ def test_grouped_mlp(M, name):
     out_rows = torch.zeros(r_cap, cfg.H, dtype=torch.bfloat16, device="cuda")
     shared_out = (torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
                   if cfg.I_shared else None)
-    M.moe_grouped_mlp(c, M.prepare_weights(c, weights_dict(d)), rows, counts, offsets, out_rows,
-                      ws, x=d["x"], shared_out=shared_out)
+    rt = np.full(r_cap, -1, dtype=np.int32)
+    rt[:n] = m["row_token"]
+    row_token = torch.from_numpy(rt).to("cuda")
+    M.moe_grouped_mlp(c, M.prepare_weights(c, weights_dict(d)), None if gather else rows, counts,
+                      offsets, out_rows, ws, x=d["x"], shared_out=shared_out,
+                      row_token=row_token if gather else None)
     torch.cuda.synchronize()
     assert M.moe_get_device_status(ws) == 0
     got = f64(out_rows)
