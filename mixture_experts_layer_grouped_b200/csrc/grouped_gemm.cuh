@@ -330,9 +330,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
                           pol_w);
           }
           uint8_t* sb = sa + C::NA * C::A_BYTES;
+          // fixed-count loops with a predicate (straight-line async copies)
           if (!gather)
-            for (int bx = 0; bx < nbox; ++bx)
-              tma_load_2d(sb + bx * kBoxRows * 128, &p.b[t.grp], &full[stage],
+#pragma unroll
+            for (int bx = 0; bx < TILE_N / kBoxRows; ++bx)
+              if (bx < nbox) tma_load_2d(sb + bx * kBoxRows * 128, &p.b[t.grp], &full[stage],
                           kt * (DT == kBF16 ? kBK : 128), t.row0 + bx * kBoxRows, pol_x);
           if (DT != kBF16) {
             // scale chunks of this k-step (SF_KCH consecutive chunks per 128-row chunk):
@@ -348,7 +350,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             else if (MODE == kFc2 && slab1)
               bulk_load(ssf + cb_bytes, p.sfa0[t.grp] + (ca + kb4) * C::SF_CHUNK, cb_bytes,
                         &full[stage], pol_w);
-            for (int cb = 0; cb < nsfb; ++cb) {
+#pragma unroll
+            for (int cb = 0; cb < C::SFB_CHUNKS; ++cb) if (cb < nsfb) {
               const int64_t cbi = (static_cast<int64_t>(t.row0) / 128 + cb) * kb4 + kt * C::SF_KCH;
               bulk_load(ssf + (C::NA + cb) * cb_bytes, p.sfb[t.grp] + cbi * C::SF_CHUNK, cb_bytes,
                         &full[stage], pol_x);
@@ -381,7 +384,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         const Tile t = decode_tile<MODE, TILE_N>(u, p, prefix, units_routed);
         const int n_mma = (t.n_tok + 15) & ~15;
         const uint32_t idesc = idesc_bf16(kBM, n_mma);
-        const int nsfb = ((t.row0 & 127) + t.n_tok + 127) / 128;
         // token j's scale sits at chunk row (row0 % 128) + j: shift the TMEM base
         const uint32_t sfb_shift = static_cast<uint32_t>((t.row0 & 127) >> 5);
         const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
@@ -417,7 +419,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
               tmem_cp_sf_chunk(sf_a0 + 4 * kk, sdesc_sf_chunk(ssf + kk * C::SF_CHUNK));
               if (C::NA == 2)
                 tmem_cp_sf_chunk(sf_a1 + 4 * kk, sdesc_sf_chunk(ssf + cb_bytes + kk * C::SF_CHUNK));
-              for (int cb = 0; cb < nsfb; ++cb)
+              // every token chunk slot is copied, also past the tile's nsfb: a
+              // fixed count keeps the copies straight-line (a data-dependent loop
+              // around tcgen05.cp measured several times slower); the extra
+              // slots hold scales of columns past the tile's tokens, never stored
+#pragma unroll
+              for (int cb = 0; cb < C::SFB_CHUNKS; ++cb)
                 tmem_cp_sf_chunk(sf_b + 4 * (kk * C::SFB_CHUNKS + cb),
                                  sdesc_sf_chunk(ssf + (C::NA + cb) * cb_bytes + kk * C::SF_CHUNK));
             }
@@ -439,7 +446,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             const uint32_t sf_b = sf_a0 + 4 * C::NA;
             tmem_cp_sf_chunk(sf_a0, sdesc_sf_chunk(ssf));
             if (C::NA == 2) tmem_cp_sf_chunk(sf_a1, sdesc_sf_chunk(ssf + C::SF_CHUNK));
-            for (int cb = 0; cb < nsfb; ++cb)
+#pragma unroll
+            for (int cb = 0; cb < C::SFB_CHUNKS; ++cb)  // fixed count, as in the NVFP4 branch
               tmem_cp_sf_chunk(sf_b + 4 * cb, sdesc_sf_chunk(ssf + (C::NA + cb) * C::SF_CHUNK));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
