@@ -424,7 +424,7 @@ def run_ours(args, cfg):
         "gpu_launches": ({"bf16": 9, "mxfp8": 10, "nvfp4": 14}[cfg.dtype] + (1 if cfg.dtype == "nvfp4" and cfg.I_shared else 0)) * args.steps,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"], "samples": clocks["samples"]},
-        "tile_n": int(os.environ.get("MOE_GEMM_TILE_N", "256")),
+        "gemm_pairs": os.environ.get("MOE_GEMM_PAIRS", "1") != "0",
     }
     print(json.dumps(line), flush=True)
 

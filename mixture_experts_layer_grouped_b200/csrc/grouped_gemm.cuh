@@ -61,6 +61,10 @@ struct GemmParams {
   const uint8_t* sfa0[2];   // scales of a0's rows
   const uint8_t* sfa1[2];   // scales of a1's rows
   const uint8_t* sfb[2];    // scales of the token rows
+  // CTA pairs: the same scale buffers as 2-D maps of 512-byte chunks (uint32 x 128)
+  CUtensorMap sfa0_map[2];
+  CUtensorMap sfa1_map[2];
+  CUtensorMap sfb_map[2];
   int32_t kb4[2];           // chunk columns per row chunk (K/128 MXFP8, K/64 NVFP4)
   // NVFP4 global scales: acc * 1 / (ga[e * ga_stride] * gw[e * gw_stride])
   const float* ga[2];
@@ -88,11 +92,13 @@ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-template <int MODE, int TILE_N, int DT = kBF16>
+template <int MODE, int TILE_N, int DT = kBF16, bool PAIR = false>
 struct GemmCfg {
   static constexpr int NA = (MODE == kRouter) ? 1 : 2;
   static constexpr int A_BYTES = kBM * 128;
-  static constexpr int B_BYTES = TILE_N * 128;
+  // a CTA pair splits the token rows of a tile: each CTA holds TILE_N / 2
+  static constexpr int B_ROWS = PAIR ? TILE_N / 2 : TILE_N;
+  static constexpr int B_BYTES = B_ROWS * 128;
   static constexpr int SF_CHUNK = 512;                          // one 128x4 scale chunk
   static constexpr int SF_KCH = (DT == kNVF4) ? 4 : 1;          // scale chunks per k-step
   // token row chunks of scales: a tile starts at a row that is a multiple of 64
@@ -103,7 +109,12 @@ struct GemmCfg {
   static constexpr int SFB_CHUNKS = (TILE_N + 64 + 127) / 128;
   static constexpr int SF_BYTES = (DT != kBF16) ? (NA + SFB_CHUNKS) * SF_KCH * SF_CHUNK : 0;
   static constexpr int STAGE_BYTES = (NA * A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
-  static constexpr int RING = (DT == kNVF4) ? 198 * 1024 : kRingBytes;
+  static constexpr int STG_WARP = 32 * 34 * 2;                 // per warp 32 x 34 bf16
+  static constexpr int STG_BYTES = kEpiWarps * STG_WARP;
+  static constexpr int BAR_BYTES = 256;
+  // CTA pairs take every byte the epilogue staging, barriers and tile prefix leave
+  static constexpr int RING = PAIR ? (232448 - 1024 - STG_BYTES - BAR_BYTES - 4 * (kMaxExperts + 1))
+                                   : ((DT == kNVF4) ? 198 * 1024 : kRingBytes);
   static constexpr int STAGES = (RING / STAGE_BYTES) > 8 ? 8 : (RING / STAGE_BYTES);
   static constexpr int ACC_COLS = NA * TILE_N;  // TMEM columns of one tile
   static constexpr int SF_COLS = (DT != kBF16) ? 4 * SF_KCH * (NA + SFB_CHUNKS) : 0;
@@ -113,10 +124,8 @@ struct GemmCfg {
   // the copies of stage s+1 do not overwrite columns stage s's MMAs still read
   static constexpr int SF_BUFS = (SF_COLS > 0 && ACC_BUFS * ACC_COLS + 2 * SF_COLS <= 512) ? 2 : 1;
   static constexpr uint32_t TMEM_COLS = pow2_at_least(ACC_BUFS * ACC_COLS + SF_BUFS * SF_COLS);
-  static constexpr int SLAB_ROWS = (MODE == kFc2) ? 2 * kBM : kBM;  // features per tile
-  static constexpr int STG_WARP = 32 * 34 * 2;                 // per warp 32 x 34 bf16
-  static constexpr int STG_BYTES = kEpiWarps * STG_WARP;
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int SLAB_ROWS = (MODE == kFc2) ? 2 * kBM : kBM;  // features per CTA tile
+  static constexpr int SLAB_SPAN = PAIR ? 2 * SLAB_ROWS : SLAB_ROWS;  // features per tile
   static constexpr int SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES + 4 * (kMaxExperts + 1);
   static_assert(TMEM_COLS <= 512, "TMEM overflow");
@@ -126,12 +135,15 @@ struct GemmCfg {
 
 struct Tile {
   int grp, e, slab, row0, n_tok, k_begin, k_end, a_row, split;
+  int f0;  // first output feature of this CTA's rows within the expert
 };
 
-template <int MODE, int TILE_N>
+// `rank` is the CTA's rank in its pair (0 without pairs): its A rows start
+// SLAB_ROWS into the tile's SLAB_SPAN features.
+template <int MODE, int TILE_N, bool PAIR = false>
 __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const int* prefix,
-                                            int units_routed) {
-  using C = GemmCfg<MODE, TILE_N, kBF16>;
+                                            int units_routed, int rank = 0) {
+  using C = GemmCfg<MODE, TILE_N, kBF16, PAIR>;
   Tile t;
   if (u < units_routed) {
     const int ns = p.g[0].n_slabs;
@@ -147,7 +159,8 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
     t.e = lo;
     t.row0 = __ldg(p.offsets + lo) + chunk * TILE_N;
     t.n_tok = min(TILE_N, __ldg(p.counts + lo) - chunk * TILE_N);
-    t.a_row = lo * p.g[0].a_rows_per_expert + t.slab * C::SLAB_ROWS;
+    t.f0 = t.slab * C::SLAB_SPAN + rank * C::SLAB_ROWS;
+    t.a_row = lo * p.g[0].a_rows_per_expert + t.f0;
     t.split = 0;
     t.k_begin = 0;
     t.k_end = p.g[0].k_tiles;
@@ -163,7 +176,8 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
     t.e = 0;
     t.row0 = chunk * TILE_N;
     t.n_tok = min(TILE_N, p.dense_rows - t.row0);
-    t.a_row = t.slab * C::SLAB_ROWS;
+    t.f0 = t.slab * C::SLAB_SPAN + rank * C::SLAB_ROWS;
+    t.a_row = t.f0;
     const int kps = (G.k_tiles + G.k_splits - 1) / G.k_splits;
     t.k_begin = t.split * kps;
     t.k_end = min(G.k_tiles, t.k_begin + kps);
@@ -171,13 +185,52 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
   return t;
 }
 
+// One-CTA or CTA-pair (cta_group::2) forms of the MMA issuer's instructions.
+template <bool PAIR>
+__device__ __forceinline__ void mma_bf16_x(uint32_t d, uint64_t a, uint64_t b, uint32_t id,
+                                           uint32_t acc) {
+  if constexpr (PAIR) mma_bf16_pair(d, a, b, id, acc); else mma_bf16(d, a, b, id, acc);
+}
+template <bool PAIR>
+__device__ __forceinline__ void mma_mxf8_x(uint32_t d, uint64_t a, uint64_t b, uint32_t id,
+                                           uint32_t sfa, uint32_t sfb, uint32_t acc) {
+  if constexpr (PAIR) mma_mxf8_pair(d, a, b, id, sfa, sfb, acc);
+  else mma_mxf8(d, a, b, id, sfa, sfb, acc);
+}
+template <bool PAIR>
+__device__ __forceinline__ void mma_nvf4_x(uint32_t d, uint64_t a, uint64_t b, uint32_t id,
+                                           uint32_t sfa, uint32_t sfb, uint32_t acc) {
+  if constexpr (PAIR) mma_nvf4_pair(d, a, b, id, sfa, sfb, acc);
+  else mma_nvf4(d, a, b, id, sfa, sfb, acc);
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_cp_sf_chunk_x(uint32_t taddr, uint64_t sdesc) {
+  if constexpr (PAIR) tmem_cp_sf_chunk_pair(taddr, sdesc); else tmem_cp_sf_chunk(taddr, sdesc);
+}
+// Arrive on `bar` once the issued tcgen05 work completes; pairs arrive on the
+// barrier of both CTAs (two commits, no multicast form).
+template <bool PAIR>
+__device__ __forceinline__ void commit_x(uint64_t* bar) {
+  if constexpr (PAIR) {
+    mma_commit_pair(cluster_addr(bar, 0));
+    mma_commit_pair(cluster_addr(bar, 1));
+  } else {
+    mma_commit(bar);
+  }
+}
+
 // silu(g) = g * sigmoid(g); fast exp and division (well inside bf16 rounding).
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-template <int MODE, int TILE_N, int DT>
+// PAIR: the kernel runs as clusters of two CTAs; rank 0 issues M = 256 MMAs
+// over both CTAs' shared memory (cta_group::2), each CTA loads its own 128
+// weight rows and half of the tile's token rows, and the loads of both count
+// on rank 0's full barrier.
+template <int MODE, int TILE_N, int DT, bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     const __grid_constant__ GemmParams p) {
-  using C = GemmCfg<MODE, TILE_N, DT>;
+  using C = GemmCfg<MODE, TILE_N, DT, PAIR>;
+  static_assert(!PAIR || MODE != kRouter, "CTA pairs serve fc1 and fc2");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -194,6 +247,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
 
   const int warp = warp_id();
   const int lane = lane_id();
+  const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const int n_groups = PAIR ? gridDim.x / 2 : gridDim.x;  // CTAs or CTA pairs
+  const int group_id = PAIR ? blockIdx.x / 2 : blockIdx.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -202,7 +258,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kEpiWarps);
+      // pairs: both CTAs' epilogue warps release rank 0's accumulator barrier
+      mbar_init(&acc_empty[b], PAIR ? 2 * kEpiWarps : kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -216,8 +273,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    // (one cta_group per kernel: pair kernels use only cta_group::2 tcgen05 forms)
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   if (warp == 2) {
     // prefix[e] = number of TILE_N-token chunks of experts < e
@@ -240,7 +303,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     }
   }
   tc_fence_before();
-  __syncthreads();
+  // pairs: the peer's barriers and TMEM must exist before any cross-CTA access
+  if (PAIR) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -252,8 +316,72 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
   const int units = units_routed + units_dense;
 
   // gathered token rows: the whole producer warp issues the row gathers
-  const bool warp_loads = (MODE == kFc1) && p.row_token != nullptr;
-  if (warp == 0) {
+  const bool warp_loads = !PAIR && (MODE == kFc1) && p.row_token != nullptr;
+  if (PAIR && warp == 0) {
+    // ---------------- TMA producer of a CTA pair (lane 0 of each CTA) ----------
+    // Both CTAs walk the same tiles.  Each loads its 128 rows of every weight
+    // operand, its half of the token rows (N/2 each) and all token scale chunks
+    // (each CTA's TMEM needs every token's scales), and every load completes on
+    // rank 0's full barrier, whose expected bytes count both CTAs.
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_last();
+      constexpr uint32_t cb_bytes = C::SF_KCH * C::SF_CHUNK;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = group_id; u < units && ok; u += n_groups) {
+        const Tile t = decode_tile<MODE, TILE_N, PAIR>(u, p, prefix, units_routed, rank);
+        const int half = ((t.n_tok + 15) & ~15) / 2;  // token rows per CTA (multiple of 8)
+        const int nbox = (half + kBoxRows - 1) / kBoxRows;
+        const int nsfb = ((t.row0 & 127) + t.n_tok + 127) / 128;
+        // identical in both CTAs; weight and scale rows past the expert read the
+        // next expert's or the map's zero fill, and only feed masked outputs
+        const uint32_t bytes = C::NA * C::A_BYTES + nbox * kBoxRows * 128 +
+                               (DT != kBF16 ? (C::NA + nsfb) * cb_bytes : 0);
+        const int kt_all = p.g[t.grp].k_tiles;
+        const int tile_base = (t.a_row / kBM) * kt_all;
+        const int kb4 = p.kb4[t.grp];
+        for (int kt = t.k_begin; kt < t.k_end; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          const uint32_t fb = cluster_addr(&full[stage], 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);
+          uint8_t* sa = ring + stage * C::STAGE_BYTES;
+          tma_load_3d_pair(sa, &p.a0[t.grp], fb, 0, 0, tile_base + kt, pol_w);
+          if (MODE == kFc1)
+            tma_load_3d_pair(sa + C::A_BYTES, &p.a1[t.grp], fb, 0, 0, tile_base + kt, pol_w);
+          else
+            tma_load_3d_pair(sa + C::A_BYTES, &p.a0[t.grp], fb, 0, 0, tile_base + kt + kt_all,
+                             pol_w);
+          uint8_t* sb = sa + C::NA * C::A_BYTES;
+          const int col = kt * (DT == kBF16 ? kBK : 128);
+#pragma unroll
+          for (int bx = 0; bx < C::B_ROWS / kBoxRows; ++bx)
+            if (bx < nbox)
+              tma_load_2d_pair(sb + bx * kBoxRows * 128, &p.b[t.grp], fb, col,
+                               t.row0 + rank * half + bx * kBoxRows, pol_x);
+          if (DT != kBF16) {
+            uint8_t* ssf = sb + C::B_BYTES;
+            const int ca = (t.a_row / 128) * kb4 + kt * C::SF_KCH;
+            tma_load_2d_pair(ssf, &p.sfa0_map[t.grp], fb, 0, ca, pol_w);
+            if (MODE == kFc1)
+              tma_load_2d_pair(ssf + cb_bytes, &p.sfa1_map[t.grp], fb, 0, ca, pol_w);
+            else
+              tma_load_2d_pair(ssf + cb_bytes, &p.sfa0_map[t.grp], fb, 0, ca + kb4, pol_w);
+#pragma unroll
+            for (int cb = 0; cb < C::SFB_CHUNKS; ++cb)
+              if (cb < nsfb)
+                tma_load_2d_pair(ssf + (C::NA + cb) * cb_bytes, &p.sfb_map[t.grp], fb, 0,
+                                 (t.row0 / 128 + cb) * kb4 + kt * C::SF_KCH, pol_x);
+          }
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // No drain here: rank 0's MMA issuer waits for every stage either CTA loads
+      // (or gives up after its own bounded wait), and the closing cluster barrier
+      // keeps both CTAs resident until then.
+    }
+  } else if (warp == 0) {
     // ---------------- TMA producer (lane 0, or the whole warp when gathering) ----
     if (lane == 0 || warp_loads) {
       const uint64_t pol_w = l2_policy_evict_first();
@@ -374,16 +502,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    // (pairs: rank 0 only; its MMAs span both CTAs)
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const Tile t = decode_tile<MODE, TILE_N>(u, p, prefix, units_routed);
+      constexpr int M_MMA = PAIR ? 2 * kBM : kBM;
+      for (int u = group_id; u < units && ok; u += n_groups) {
+        const Tile t = decode_tile<MODE, TILE_N, PAIR>(u, p, prefix, units_routed, 0);
         const int n_mma = (t.n_tok + 15) & ~15;
-        const uint32_t idesc = idesc_bf16(kBM, n_mma);
+        const uint32_t idesc = idesc_bf16(M_MMA, n_mma);
         // token j's scale sits at chunk row (row0 % 128) + j: shift the TMEM base
         const uint32_t sfb_shift = static_cast<uint32_t>((t.row0 & 127) >> 5);
         const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
@@ -402,8 +532,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t accum = (kt > t.k_begin || kk) ? 1u : 0u;
               // advance 16 bf16 = 32 bytes along K inside the swizzle atom
-              mma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
-              if (C::NA == 2) mma_bf16(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+              mma_bf16_x<PAIR>(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
+              if (C::NA == 2) mma_bf16_x<PAIR>(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, idesc, accum);
             }
           } else if (DT == kNVF4) {
             // scale factors: chunk kk of each operand feeds MMA kk (one 32-bit word
@@ -416,27 +546,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             const uint32_t sf_b = sf_a0 + 4 * C::SF_KCH * C::NA;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              tmem_cp_sf_chunk(sf_a0 + 4 * kk, sdesc_sf_chunk(ssf + kk * C::SF_CHUNK));
+              tmem_cp_sf_chunk_x<PAIR>(sf_a0 + 4 * kk, sdesc_sf_chunk(ssf + kk * C::SF_CHUNK));
               if (C::NA == 2)
-                tmem_cp_sf_chunk(sf_a1 + 4 * kk, sdesc_sf_chunk(ssf + cb_bytes + kk * C::SF_CHUNK));
+                tmem_cp_sf_chunk_x<PAIR>(sf_a1 + 4 * kk, sdesc_sf_chunk(ssf + cb_bytes + kk * C::SF_CHUNK));
               // every token chunk slot is copied, also past the tile's nsfb: a
               // fixed count keeps the copies straight-line (a data-dependent loop
               // around tcgen05.cp measured several times slower); the extra
               // slots hold scales of columns past the tile's tokens, never stored
 #pragma unroll
               for (int cb = 0; cb < C::SFB_CHUNKS; ++cb)
-                tmem_cp_sf_chunk(sf_b + 4 * (kk * C::SFB_CHUNKS + cb),
+                tmem_cp_sf_chunk_x<PAIR>(sf_b + 4 * (kk * C::SFB_CHUNKS + cb),
                                  sdesc_sf_chunk(ssf + (C::NA + cb) * cb_bytes + kk * C::SF_CHUNK));
             }
-            const uint32_t id = idesc_nvf4(kBM, n_mma);
+            const uint32_t id = idesc_nvf4(M_MMA, n_mma);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t accum = (kt > t.k_begin || kk) ? 1u : 0u;
               const uint32_t sfb = sf_b + 4 * kk * C::SFB_CHUNKS + sfb_shift;
               // advance 64 e2m1 = 32 bytes along K
-              mma_nvf4(d0, da0 + 2 * kk, db + 2 * kk, id, sf_a0 + 4 * kk, sfb, accum);
+              mma_nvf4_x<PAIR>(d0, da0 + 2 * kk, db + 2 * kk, id, sf_a0 + 4 * kk, sfb, accum);
               if (C::NA == 2)
-                mma_nvf4(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, id, sf_a1 + 4 * kk, sfb, accum);
+                mma_nvf4_x<PAIR>(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, id, sf_a1 + 4 * kk, sfb, accum);
             }
           } else {
             // scale factors of this stage: smem -> TMEM (in order with the MMAs below)
@@ -444,32 +574,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             const uint32_t sf_a0 = tmem_base + C::SF_TMEM + (C::SF_BUFS == 2 ? (kt & 1) : 0) * C::SF_COLS;
             const uint32_t sf_a1 = sf_a0 + 4;
             const uint32_t sf_b = sf_a0 + 4 * C::NA;
-            tmem_cp_sf_chunk(sf_a0, sdesc_sf_chunk(ssf));
-            if (C::NA == 2) tmem_cp_sf_chunk(sf_a1, sdesc_sf_chunk(ssf + C::SF_CHUNK));
+            tmem_cp_sf_chunk_x<PAIR>(sf_a0, sdesc_sf_chunk(ssf));
+            if (C::NA == 2) tmem_cp_sf_chunk_x<PAIR>(sf_a1, sdesc_sf_chunk(ssf + C::SF_CHUNK));
 #pragma unroll
             for (int cb = 0; cb < C::SFB_CHUNKS; ++cb)  // fixed count, as in the NVFP4 branch
-              tmem_cp_sf_chunk(sf_b + 4 * cb, sdesc_sf_chunk(ssf + (C::NA + cb) * C::SF_CHUNK));
+              tmem_cp_sf_chunk_x<PAIR>(sf_b + 4 * cb, sdesc_sf_chunk(ssf + (C::NA + cb) * C::SF_CHUNK));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t accum = (kt > t.k_begin || kk) ? 1u : 0u;
-              const uint32_t id = idesc_mxf8(kBM, n_mma, kk);
+              const uint32_t id = idesc_mxf8(M_MMA, n_mma, kk);
               const uint32_t byte = static_cast<uint32_t>(kk) << 30;
               // advance 32 e4m3 = 32 bytes along K; k-block kk of the scale words
               const uint32_t sfb = (sf_b + sfb_shift) | byte;
-              mma_mxf8(d0, da0 + 2 * kk, db + 2 * kk, id, sf_a0 | byte, sfb, accum);
+              mma_mxf8_x<PAIR>(d0, da0 + 2 * kk, db + 2 * kk, id, sf_a0 | byte, sfb, accum);
               if (C::NA == 2)
-                mma_mxf8(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, id, sf_a1 | byte, sfb, accum);
+                mma_mxf8_x<PAIR>(d0 + TILE_N, da1 + 2 * kk, db + 2 * kk, id, sf_a1 | byte, sfb, accum);
             }
           }
-          mma_commit(&empty[stage]);
+          commit_x<PAIR>(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        mma_commit(&acc_full[acc]);
+        commit_x<PAIR>(&acc_full[acc]);
         if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
       }
       // Drain: all issued MMAs complete before TMEM is released.
-      mma_commit(drain);
+      if constexpr (PAIR) mma_commit_pair(cluster_addr(drain, 0)); else mma_commit(drain);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 20000000ull) {
       }
@@ -481,14 +611,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     uint8_t* my_stg = stg + (warp - 2) * C::STG_WARP;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
-      const Tile t = decode_tile<MODE, TILE_N>(u, p, prefix, units_routed);
+    for (int u = group_id; u < units; u += n_groups) {
+      const Tile t = decode_tile<MODE, TILE_N, PAIR>(u, p, prefix, units_routed, rank);
       if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
       const GemmGroup& G = p.g[t.grp];
       const uint32_t lane_addr =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::ACC_COLS;
-      const int f_base = t.slab * C::SLAB_ROWS + quarter * 32;
+      const int f_base = t.f0 + quarter * 32;
       // NVFP4: undo the global encode scales of both operands
       float alpha = 1.0f;
       if (DT == kNVF4)
@@ -592,7 +722,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));  // rank 0's barrier
+        else mbar_arrive(&acc_empty[acc]);
+      }
       if (MODE == kFc1 && DT == kNVF4) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
@@ -604,10 +737,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
   }
 
   tc_fence_before();
-  __syncthreads();
+  // pairs: neither CTA leaves while the other may still touch its shared memory,
+  // barriers or TMEM
+  if (PAIR) cluster_sync_all(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 

@@ -229,6 +229,26 @@ moe_status make_tiled_map(CUtensorMap* m, const void* base, uint64_t rows, uint6
   return MOE_OK;
 }
 
+// 2-D map over a block-scale buffer as rows of 512-byte chunks (uint32 x 128):
+// a box of `box_rows` consecutive chunks; chunks past n_chunks read as zeros.
+moe_status make_sf_map(CUtensorMap* m, const void* base, uint64_t n_chunks, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MOE_ERR_CUDA;
+  if (reinterpret_cast<uintptr_t>(base) % 16 || n_chunks < 1) return MOE_ERR_INVALID_ARG;
+  cuuint64_t dims[2] = {128, n_chunks};
+  cuuint64_t strides[1] = {512};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fprintf(stderr, "moe_b200: cuTensorMapEncodeTiled (scales) failed (%d)\n", static_cast<int>(r));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -236,28 +256,53 @@ int sm_count() {
   return n;
 }
 
-template <int MODE, int TILE_N, int DT>
+// One persistent CTA per SM, or (PAIR) one two-CTA cluster per SM pair, as
+// many as can be resident at once, capped by the number of tiles.
+template <int MODE, int TILE_N, int DT, bool PAIR = false>
 moe_status launch_gemm(const GemmParams& p, int max_units, cudaStream_t s) {
-  using C = GemmCfg<MODE, TILE_N, DT>;
-  MOE_CUDA(cudaFuncSetAttribute(grouped_gemm_kernel<MODE, TILE_N, DT>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-  int grid = sm_count();
-  if (max_units < grid) grid = max_units;
-  if (grid < 1) return MOE_OK;
-  grouped_gemm_kernel<MODE, TILE_N, DT><<<grid, kGemmThreads, C::SMEM_BYTES, s>>>(p);
-  return launch_check();
-}
-
-// Token chunk of the expert GEMMs: 256 (each weight slab streams once per
-// 256 tokens of its expert; one accumulator set) unless MOE_GEMM_TILE_N=128
-// asks for 128 (double-buffered accumulators, slabs re-streamed per 128).
-int expert_tile_n() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("MOE_GEMM_TILE_N");
-    v = (e && atoi(e) == 128) ? 128 : 256;
+  using C = GemmCfg<MODE, TILE_N, DT, PAIR>;
+  auto kern = grouped_gemm_kernel<MODE, TILE_N, DT, PAIR>;
+  MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  if (!PAIR) {
+    int grid = sm_count();
+    if (max_units < grid) grid = max_units;
+    if (grid < 1) return MOE_OK;
+    kern<<<grid, kGemmThreads, C::SMEM_BYTES, s>>>(p);
+    return launch_check();
   }
-  return v;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // resident clusters, once per device for this kernel
+  static int cached[64];
+  static std::mutex mu;
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  int n = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) {
+      n = cached[dev];
+    } else {
+      cfg.gridDim = dim3(2 * (sm_count() / 2));
+      MOE_CUDA(cudaOccupancyMaxActiveClusters(&n, kern, &cfg));
+      if (dev >= 0 && dev < 64) cached[dev] = n;
+    }
+  }
+  if (n < 1) return MOE_ERR_UNSUPPORTED;
+  int clusters = n < max_units ? n : max_units;
+  if (clusters < 1) return MOE_OK;
+  cfg.gridDim = dim3(2 * clusters);
+  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, p));
+  return launch_check();
 }
 
 int32_t* status_ptr(void* ws) { return static_cast<int32_t*>(ws); }
@@ -387,7 +432,9 @@ struct MlpQuant {
   const int32_t* row_token;  // with rows == nullptr: fc1 gathers token rows from x
 };
 
-template <int TILE_N, int DT>
+// PAIR: fc1 and fc2 run as two-CTA clusters (M = 256 MMAs; each CTA holds
+// half of a tile's token rows), which leaves room for a deeper load ring.
+template <int TILE_N, int DT, bool PAIR>
 moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const void* rows,
                              const void* x, const MlpQuant& q, const int32_t* counts,
                              const int32_t* offsets, void* out_rows, void* shared_out, void* ws,
@@ -409,6 +456,11 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
   const uint64_t H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
   const int max_chunks = c.E + (c.T * c.top_k) / TILE_N + 1;
   const int dense_chunks = (c.T + TILE_N - 1) / TILE_N;
+  constexpr int span1 = GemmCfg<kFc1, TILE_N, DT, PAIR>::SLAB_SPAN;  // features per fc1 tile
+  constexpr int span2 = GemmCfg<kFc2, TILE_N, DT, PAIR>::SLAB_SPAN;  // features per fc2 tile
+  constexpr uint32_t sf_box = DT == kNVF4 ? 4 : 1;                    // scale chunks per k-step
+  const uint64_t Rp128 = static_cast<uint64_t>(pad128(L.r_cap)) / 128;
+  const uint64_t Tp128 = static_cast<uint64_t>(pad128(c.T)) / 128;
   // fc1 + SwiGLU: one 128-feature slab of W1 and of W3 per tile
   {
     GemmParams p;
@@ -431,8 +483,9 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
       p.a1[1] = p.a1[0];
       p.b[1] = p.b[0];
     }
-    p.g[0] = GemmGroup{c.I, c.I, c.I / kBM, c.H / kstep, 1, h, c.I, 0};
-    p.g[1] = GemmGroup{0, c.I_shared, c.I_shared / kBM, c.H / kstep, 1, hs, c.I_shared, 0};
+    p.g[0] = GemmGroup{c.I, c.I, (c.I + span1 - 1) / span1, c.H / kstep, 1, h, c.I, 0};
+    p.g[1] = GemmGroup{0, c.I_shared, (c.I_shared + span1 - 1) / span1, c.H / kstep, 1, hs,
+                       c.I_shared, 0};
     if (qz) {
       p.sfa0[0] = static_cast<const uint8_t*>(w.w1_scales);
       p.sfa1[0] = static_cast<const uint8_t*>(w.w3_scales);
@@ -441,6 +494,21 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
       p.sfa1[1] = static_cast<const uint8_t*>(w.ws3_scales);
       p.sfb[1] = static_cast<const uint8_t*>(q.x_scales);
       p.kb4[0] = p.kb4[1] = c.H / kb4_div;
+      if (PAIR) {
+        const uint64_t kb4 = c.H / kb4_div;
+        MOE_TRY(make_sf_map(&p.sfa0_map[0], w.w1_scales, E * I / 128 * kb4, sf_box));
+        MOE_TRY(make_sf_map(&p.sfa1_map[0], w.w3_scales, E * I / 128 * kb4, sf_box));
+        MOE_TRY(make_sf_map(&p.sfb_map[0], q.row_scales, Rp128 * kb4, sf_box));
+        if (sh) {
+          MOE_TRY(make_sf_map(&p.sfa0_map[1], w.ws1_scales, Is / 128 * kb4, sf_box));
+          MOE_TRY(make_sf_map(&p.sfa1_map[1], w.ws3_scales, Is / 128 * kb4, sf_box));
+          MOE_TRY(make_sf_map(&p.sfb_map[1], q.x_scales, Tp128 * kb4, sf_box));
+        } else {
+          p.sfa0_map[1] = p.sfa0_map[0];
+          p.sfa1_map[1] = p.sfa1_map[0];
+          p.sfb_map[1] = p.sfb_map[0];
+        }
+      }
     }
     if (mx) {
       p.q_out[0] = static_cast<uint8_t*>(h);
@@ -466,7 +534,7 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     p.dense_rows = sh ? c.T : 0;
     p.status = status_ptr(ws);
     const int units = max_chunks * p.g[0].n_slabs + (sh ? dense_chunks * p.g[1].n_slabs : 0);
-    MOE_TRY((launch_gemm<kFc1, TILE_N, DT>(p, units, s)));
+    MOE_TRY((launch_gemm<kFc1, TILE_N, DT, PAIR>(p, units, s)));
   }
   // NVFP4: h's per-expert global scales from the amax fc1 gathered, then h codes
   void* h_in = h;
@@ -502,7 +570,7 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     }
     p.a1[0] = p.a0[0];
     p.a1[1] = p.a0[1];
-    const int slabs = (c.H + 2 * kBM - 1) / (2 * kBM);
+    const int slabs = (c.H + span2 - 1) / span2;
     p.g[0] = GemmGroup{c.H, c.H, slabs, c.I / kstep, 1, out_rows, c.H, 0};
     p.g[1] = GemmGroup{0, c.H, slabs, (sh ? c.I_shared : kstep) / kstep, 1, shared_out, c.H, 0};
     if (qz) {
@@ -512,6 +580,19 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
       p.sfb[1] = wsb + L.h_shared_sf;
       p.kb4[0] = c.I / kb4_div;
       p.kb4[1] = sh ? c.I_shared / kb4_div : 1;
+      if (PAIR) {
+        MOE_TRY(make_sf_map(&p.sfa0_map[0], w.w2_scales, E * H / 128 * (I / kb4_div), sf_box));
+        MOE_TRY(make_sf_map(&p.sfb_map[0], wsb + L.h_sf, Rp128 * (I / kb4_div), sf_box));
+        if (sh) {
+          MOE_TRY(make_sf_map(&p.sfa0_map[1], w.ws2_scales, H / 128 * (Is / kb4_div), sf_box));
+          MOE_TRY(make_sf_map(&p.sfb_map[1], wsb + L.h_shared_sf, Tp128 * (Is / kb4_div), sf_box));
+        } else {
+          p.sfa0_map[1] = p.sfa0_map[0];
+          p.sfb_map[1] = p.sfb_map[0];
+        }
+        p.sfa1_map[0] = p.sfa0_map[0];
+        p.sfa1_map[1] = p.sfa0_map[1];
+      }
     }
     if (nv) {
       p.ga[0] = g_h;
@@ -529,26 +610,41 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     p.dense_rows = sh ? c.T : 0;
     p.status = status_ptr(ws);
     const int units = max_chunks * slabs + (sh ? dense_chunks * slabs : 0);
-    MOE_TRY((launch_gemm<kFc2, TILE_N, DT>(p, units, s)));
+    MOE_TRY((launch_gemm<kFc2, TILE_N, DT, PAIR>(p, units, s)));
   }
   return MOE_OK;
+}
+
+// CTA pairs for fc1 and fc2 (bf16, MXFP8) unless fc1 gathers its rows from x
+// (rows == NULL) or MOE_GEMM_PAIRS=0 asks for one-CTA tiles.  NVFP4 keeps
+// one-CTA tiles: its scale chunks leave a pair's ring at three stages, like a
+// single CTA's, and the split tiles then measured slower (prefill grouped MLP
+// 3964 -> 4247 us, decode 1510 -> 1594 us on one B200).
+bool use_pairs(const moe_config& c, const void* rows) {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MOE_GEMM_PAIRS");
+    v = (e && atoi(e) == 0) ? 0 : 1;
+  }
+  return v == 1 && rows != nullptr && c.dtype != MOE_NVFP4;
 }
 
 moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void* rows,
                           const void* x, const MlpQuant& q, const int32_t* counts,
                           const int32_t* offsets, void* out_rows, void* shared_out, void* ws,
                           cudaStream_t s) {
-  if (is_mx(c))
-    return grouped_mlp_tiles<192, kMXF8>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
-                                         ws, s);
+  const bool pairs = use_pairs(c, rows);
+#define MOE_MLP(TN, DT)                                                                        \
+  return pairs ? grouped_mlp_tiles<TN, DT, true>(c, w, rows, x, q, counts, offsets, out_rows,  \
+                                                 shared_out, ws, s)                            \
+               : grouped_mlp_tiles<TN, DT, false>(c, w, rows, x, q, counts, offsets, out_rows, \
+                                                  shared_out, ws, s)
+  if (is_mx(c)) MOE_MLP(192, kMXF8);
   if (is_nv(c))
-    return grouped_mlp_tiles<192, kNVF4>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
-                                         ws, s);
-  if (expert_tile_n() == 128)
-    return grouped_mlp_tiles<128, kBF16>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
-                                         ws, s);
-  return grouped_mlp_tiles<256, kBF16>(c, w, rows, x, q, counts, offsets, out_rows, shared_out,
-                                       ws, s);
+    return grouped_mlp_tiles<192, kNVF4, false>(c, w, rows, x, q, counts, offsets, out_rows,
+                                                shared_out, ws, s);
+  MOE_MLP(256, kBF16);
+#undef MOE_MLP
 }
 
 moe_status do_combine(const moe_config& c, const void* out_rows, const int32_t* token_row,
