@@ -140,10 +140,10 @@ struct Tile {
 
 // `rank` is the CTA's rank in its pair (0 without pairs): its A rows start
 // SLAB_ROWS into the tile's SLAB_SPAN features.
-template <int MODE, int TILE_N, bool PAIR = false>
+template <int MODE, int TILE_N, int DT, bool PAIR>
 __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const int* prefix,
                                             int units_routed, int rank = 0) {
-  using C = GemmCfg<MODE, TILE_N, kBF16, PAIR>;
+  using C = GemmCfg<MODE, TILE_N, DT, PAIR>;
   Tile t;
   if (u < units_routed) {
     const int ns = p.g[0].n_slabs;
@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       uint32_t phase = 0;
       bool ok = true;
       for (int u = group_id; u < units && ok; u += n_groups) {
-        const Tile t = decode_tile<MODE, TILE_N, PAIR>(u, p, prefix, units_routed, rank);
+        const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed, rank);
         const int half = ((t.n_tok + 15) & ~15) / 2;  // token rows per CTA (multiple of 8)
         const int nbox = (half + kBoxRows - 1) / kBoxRows;
         const int nsfb = ((t.row0 & 127) + t.n_tok + 127) / 128;
@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       for (int s = 0; s < C::STAGES; ++s) last_phase[s] = -1;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const Tile t = decode_tile<MODE, TILE_N>(u, p, prefix, units_routed);
+        const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed);
         const bool gather = (MODE == kFc1) && t.grp == 0 && p.row_token != nullptr;
         // gathered rows: lane l owns tile rows [8l, 8l + 8); rows past the MMA's N
         // are not loaded, and rows between the tile's tokens and N repeat its first
@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       bool ok = true;
       constexpr int M_MMA = PAIR ? 2 * kBM : kBM;
       for (int u = group_id; u < units && ok; u += n_groups) {
-        const Tile t = decode_tile<MODE, TILE_N, PAIR>(u, p, prefix, units_routed, 0);
+        const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed, 0);
         const int n_mma = (t.n_tok + 15) & ~15;
         const uint32_t idesc = idesc_bf16(M_MMA, n_mma);
         // token j's scale sits at chunk row (row0 % 128) + j: shift the TMEM base
@@ -612,7 +612,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int u = group_id; u < units; u += n_groups) {
-      const Tile t = decode_tile<MODE, TILE_N, PAIR>(u, p, prefix, units_routed, rank);
+      const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed, rank);
       if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
       const GemmGroup& G = p.g[t.grp];
