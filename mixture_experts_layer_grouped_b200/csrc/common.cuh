@@ -566,3 +566,17 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t cluster_bar) {
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// Programmatic dependent launch.  Every library kernel calls pdl_wait() before
+// it reads or writes global memory: it returns once the preceding kernel in the
+// stream has completed and its writes are visible (at once when the kernel was
+// launched without the programmatic-serialization attribute).  pdl_trigger()
+// lets the next kernel's CTAs start launching; they still wait in pdl_wait().
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace moe

@@ -282,6 +282,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       tmem_relinquish();
     }
   }
+  // everything above touches only this CTA's shared memory and TMEM; from here
+  // on the kernel reads what the previous kernel wrote (token counts, rows)
+  pdl_wait();
+  pdl_trigger();
   if (warp == 2) {
     // prefix[e] = number of TILE_N-token chunks of experts < e
     const int E = p.E;

@@ -188,6 +188,27 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Launch with programmatic dependent launch allowed: the kernel's CTAs may
+// start while the previous kernel in the stream is finishing (every library
+// kernel waits in pdl_wait() before it touches global memory), which hides the
+// gap between the many short kernels of one layer.
+template <typename... KArgs, typename... Args>
+moe_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                      Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
+  return MOE_OK;
+}
+
 // 2-D K-major tile map over [rows, inner] elements with a 128-byte swizzle.
 // The box is (128 bytes of K) x box_rows.
 moe_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
@@ -267,20 +288,21 @@ moe_status launch_gemm(const GemmParams& p, int max_units, cudaStream_t s) {
     int grid = sm_count();
     if (max_units < grid) grid = max_units;
     if (grid < 1) return MOE_OK;
-    kern<<<grid, kGemmThreads, C::SMEM_BYTES, s>>>(p);
-    return launch_check();
+    return launch_pdl(kern, dim3(grid), dim3(kGemmThreads), C::SMEM_BYTES, s, p);
   }
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // as in launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;  // cluster shape only for the occupancy query
   // resident clusters, once per device for this kernel
   static int cached[64];
   static std::mutex mu;
@@ -301,6 +323,7 @@ moe_status launch_gemm(const GemmParams& p, int max_units, cudaStream_t s) {
   int clusters = n < max_units ? n : max_units;
   if (clusters < 1) return MOE_OK;
   cfg.gridDim = dim3(2 * clusters);
+  cfg.numAttrs = 2;
   MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, p));
   return launch_check();
 }
@@ -361,13 +384,13 @@ moe_status do_route(const moe_config& c, const void* x, const void* w_router, co
   a.rsf = c.routed_scaling_factor;
   const int per = (c.E + 31) / 32;
   const dim3 grid((c.T + kSelWarps - 1) / kSelWarps), block(kSelWarps * 32);
-  if (per <= 1) route_select_kernel<1><<<grid, block, 0, s>>>(a);
-  else if (per <= 2) route_select_kernel<2><<<grid, block, 0, s>>>(a);
-  else if (per <= 4) route_select_kernel<4><<<grid, block, 0, s>>>(a);
-  else if (per <= 8) route_select_kernel<8><<<grid, block, 0, s>>>(a);
-  else if (per <= 12) route_select_kernel<12><<<grid, block, 0, s>>>(a);
-  else if (per <= 16) route_select_kernel<16><<<grid, block, 0, s>>>(a);
-  else route_select_kernel<32><<<grid, block, 0, s>>>(a);
+  if (per <= 1) MOE_TRY(launch_pdl(route_select_kernel<1>, dim3(grid), dim3(block), 0, s, a));
+  else if (per <= 2) MOE_TRY(launch_pdl(route_select_kernel<2>, dim3(grid), dim3(block), 0, s, a));
+  else if (per <= 4) MOE_TRY(launch_pdl(route_select_kernel<4>, dim3(grid), dim3(block), 0, s, a));
+  else if (per <= 8) MOE_TRY(launch_pdl(route_select_kernel<8>, dim3(grid), dim3(block), 0, s, a));
+  else if (per <= 12) MOE_TRY(launch_pdl(route_select_kernel<12>, dim3(grid), dim3(block), 0, s, a));
+  else if (per <= 16) MOE_TRY(launch_pdl(route_select_kernel<16>, dim3(grid), dim3(block), 0, s, a));
+  else MOE_TRY(launch_pdl(route_select_kernel<32>, dim3(grid), dim3(block), 0, s, a));
   return launch_check();
 }
 
@@ -391,11 +414,11 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
   a.r_cap = L.r_cap;
   a.ntiles = L.ntiles;
   const size_t hsm = static_cast<size_t>(c.E) * 4;
-  permute_hist_kernel<<<L.ntiles, 256, hsm, s>>>(a);
+  MOE_TRY(launch_pdl(permute_hist_kernel, dim3(L.ntiles), dim3(256), hsm, s, a));
   MOE_TRY(launch_check());
-  permute_scan_kernel<<<(c.E + 7) / 8, 256, 0, s>>>(a);
+  MOE_TRY(launch_pdl(permute_scan_kernel, dim3((c.E + 7) / 8), dim3(256), 0, s, a));
   MOE_TRY(launch_check());
-  permute_rank_kernel<<<L.ntiles, 256, 0, s>>>(a);
+  MOE_TRY(launch_pdl(permute_rank_kernel, dim3(L.ntiles), dim3(256), 0, s, a));
   MOE_TRY(launch_check());
   if (is_mx(c) || is_nv(c)) {
     GatherMxArgs g;
@@ -407,8 +430,8 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
     g.offsets = offsets;
     g.E = c.E;
     g.H = c.H;
-    if (is_nv(c)) permute_gather_nv_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
-    else permute_gather_mx_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
+    if (is_nv(c)) MOE_TRY(launch_pdl(permute_gather_nv_kernel, dim3(sm_count() * 4), dim3(256), 0, s, g));
+    else MOE_TRY(launch_pdl(permute_gather_mx_kernel, dim3(sm_count() * 4), dim3(256), 0, s, g));
     return launch_check();
   }
   if (!dst_rows) return MOE_OK;  // rows are gathered later by the grouped GEMM
@@ -419,7 +442,7 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
   g.offsets = offsets;
   g.E = c.E;
   g.row_bytes = c.H * 2;
-  permute_gather_kernel<<<sm_count() * 4, 256, 0, s>>>(g);
+  MOE_TRY(launch_pdl(permute_gather_kernel, dim3(sm_count() * 4), dim3(256), 0, s, g));
   return launch_check();
 }
 
@@ -540,16 +563,16 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
   void* h_in = h;
   void* hs_in = hs;
   if (nv) {
-    amax_to_global_kernel<<<(c.E + 1 + 255) / 256, 256, 0, s>>>(g_h, c.E + 1);
+    MOE_TRY(launch_pdl(amax_to_global_kernel, dim3((c.E + 1 + 255) / 256), dim3(256), 0, s, g_h, c.E + 1));
     MOE_TRY(launch_check());
-    quantize_h_nvfp4_kernel<<<sm_count() * 4, 256, 0, s>>>(
+    MOE_TRY(launch_pdl(quantize_h_nvfp4_kernel, dim3(sm_count() * 4), dim3(256), 0, s, 
         static_cast<const __nv_bfloat16*>(h), wsb + L.h_q, wsb + L.h_sf, c.I, offsets, counts,
-        c.E, g_h, 0);
+        c.E, g_h, 0));
     MOE_TRY(launch_check());
     if (sh) {
-      quantize_h_nvfp4_kernel<<<sm_count() * 2, 256, 0, s>>>(
+      MOE_TRY(launch_pdl(quantize_h_nvfp4_kernel, dim3(sm_count() * 2), dim3(256), 0, s, 
           static_cast<const __nv_bfloat16*>(hs), wsb + L.h_shared_q, wsb + L.h_shared_sf,
-          c.I_shared, offsets, counts, c.E, g_h + c.E, c.T);
+          c.I_shared, offsets, counts, c.E, g_h + c.E, c.T));
       MOE_TRY(launch_check());
     }
     h_in = wsb + L.h_q;
@@ -660,15 +683,15 @@ moe_status do_combine(const moe_config& c, const void* out_rows, const int32_t* 
   a.k = c.top_k;
   const int threads = (c.H / 8) < 256 ? (c.H / 8) : 256;
   switch (c.top_k) {
-    case 1: combine_kernel<1><<<c.T, threads, 0, s>>>(a); break;
-    case 2: combine_kernel<2><<<c.T, threads, 0, s>>>(a); break;
-    case 3: combine_kernel<3><<<c.T, threads, 0, s>>>(a); break;
-    case 4: combine_kernel<4><<<c.T, threads, 0, s>>>(a); break;
-    case 5: combine_kernel<5><<<c.T, threads, 0, s>>>(a); break;
-    case 6: combine_kernel<6><<<c.T, threads, 0, s>>>(a); break;
-    case 7: combine_kernel<7><<<c.T, threads, 0, s>>>(a); break;
-    case 8: combine_kernel<8><<<c.T, threads, 0, s>>>(a); break;
-    default: combine_kernel<0><<<c.T, threads, 0, s>>>(a); break;
+    case 1: MOE_TRY(launch_pdl(combine_kernel<1>, dim3(c.T), dim3(threads), 0, s, a)); break;
+    case 2: MOE_TRY(launch_pdl(combine_kernel<2>, dim3(c.T), dim3(threads), 0, s, a)); break;
+    case 3: MOE_TRY(launch_pdl(combine_kernel<3>, dim3(c.T), dim3(threads), 0, s, a)); break;
+    case 4: MOE_TRY(launch_pdl(combine_kernel<4>, dim3(c.T), dim3(threads), 0, s, a)); break;
+    case 5: MOE_TRY(launch_pdl(combine_kernel<5>, dim3(c.T), dim3(threads), 0, s, a)); break;
+    case 6: MOE_TRY(launch_pdl(combine_kernel<6>, dim3(c.T), dim3(threads), 0, s, a)); break;
+    case 7: MOE_TRY(launch_pdl(combine_kernel<7>, dim3(c.T), dim3(threads), 0, s, a)); break;
+    case 8: MOE_TRY(launch_pdl(combine_kernel<8>, dim3(c.T), dim3(threads), 0, s, a)); break;
+    default: MOE_TRY(launch_pdl(combine_kernel<0>, dim3(c.T), dim3(threads), 0, s, a)); break;
   }
   return launch_check();
 }
@@ -941,22 +964,21 @@ moe_status moe_quantize(int32_t dtype, const void* in, int32_t rows, int32_t col
     const int64_t n = static_cast<int64_t>(rows) * cols;
     MOE_CUDA(cudaMemsetAsync(global_scale, 0, 4, st));
     const unsigned nb = static_cast<unsigned>((n / 8 + 255) / 256 < 2048 ? (n / 8 + 255) / 256 : 2048);
-    amax_groups_kernel<<<dim3(nb, 1), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), n,
-                                                    global_scale);
+    MOE_TRY(launch_pdl(amax_groups_kernel, dim3(dim3(nb, 1)), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(in), n,
+                                                    global_scale));
     MOE_TRY(launch_check());
-    amax_to_global_kernel<<<1, 32, 0, st>>>(global_scale, 1);
+    MOE_TRY(launch_pdl(amax_to_global_kernel, dim3(1), dim3(32), 0, st, global_scale, 1));
     MOE_TRY(launch_check());
     const int64_t blocks = static_cast<int64_t>(rows) * (cols / 16);
-    quantize_nvfp4_kernel<<<static_cast<unsigned>((blocks + 255) / 256), 256, 0, st>>>(
+    MOE_TRY(launch_pdl(quantize_nvfp4_kernel, dim3(static_cast<unsigned>((blocks + 255) / 256)), dim3(256), 0, st, 
         static_cast<const __nv_bfloat16*>(in), static_cast<uint8_t*>(codes),
-        static_cast<uint8_t*>(scales), rows, cols, global_scale, 0, 0);
+        static_cast<uint8_t*>(scales), rows, cols, global_scale, 0, 0));
     return launch_check();
   }
   const int64_t blocks = static_cast<int64_t>(rows) * (cols / 32);
-  quantize_mxfp8_rows_kernel<<<static_cast<unsigned>((blocks + 255) / 256), 256, 0,
-                               static_cast<cudaStream_t>(stream)>>>(
+  MOE_TRY(launch_pdl(quantize_mxfp8_rows_kernel, dim3(static_cast<unsigned>((blocks + 255) / 256)), dim3(256), 0, static_cast<cudaStream_t>(stream), 
       static_cast<const __nv_bfloat16*>(in), static_cast<uint8_t*>(codes),
-      static_cast<uint8_t*>(scales), rows, cols);
+      static_cast<uint8_t*>(scales), rows, cols));
   return launch_check();
 }
 

@@ -15,6 +15,8 @@ namespace moe {
 __global__ void __launch_bounds__(256) tile_rows_kernel(const uint4* __restrict__ src,
                                                         uint4* __restrict__ dst, int64_t rows,
                                                         int K) {
+  pdl_wait();
+  pdl_trigger();
   const int kt_n = K / 64;
   const int64_t tile = blockIdx.x;
   const int64_t rs = tile / kt_n;

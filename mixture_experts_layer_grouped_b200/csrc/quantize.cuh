@@ -19,6 +19,8 @@ namespace moe {
 __global__ void __launch_bounds__(256) quantize_mxfp8_rows_kernel(
     const __nv_bfloat16* __restrict__ in, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, int64_t rows, int cols) {
+  pdl_wait();
+  pdl_trigger();
   const int KB = cols / 32;
   const int64_t blk = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (blk >= rows * KB) return;
@@ -60,6 +62,8 @@ __global__ void __launch_bounds__(256) quantize_mxfp8_rows_kernel(
 __global__ void __launch_bounds__(256) quantize_mxfp8_tiles_kernel(
     const __nv_bfloat16* __restrict__ in, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, int64_t rows, int cols) {
+  pdl_wait();
+  pdl_trigger();
   const int KB = cols / 32;
   const int64_t blk = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (blk >= rows * KB) return;
@@ -111,6 +115,8 @@ struct GatherMxArgs {
 };
 
 __global__ void __launch_bounds__(256) permute_gather_mx_kernel(GatherMxArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int rows = a.offsets[a.E];
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -152,6 +158,8 @@ namespace moe {
 // at zero).  Each block reduces a strided slice and issues one atomic.
 __global__ void __launch_bounds__(256) amax_groups_kernel(const __nv_bfloat16* __restrict__ in,
                                                           int64_t group_elems, float* out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[8];
   const int64_t vecs = group_elems / 8;
   const uint4* base = reinterpret_cast<const uint4*>(in + blockIdx.y * group_elems);
@@ -178,6 +186,8 @@ __global__ void __launch_bounds__(256) amax_groups_kernel(const __nv_bfloat16* _
 
 // In place: amax -> global encode scale.
 __global__ void amax_to_global_kernel(float* v, int n) {
+  pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) v[i] = nv_global_scale(v[i]);
 }
@@ -204,6 +214,8 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(
     const __nv_bfloat16* __restrict__ in, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, int64_t rows, int cols, const float* __restrict__ g,
     int64_t rows_per_group, int tiled) {
+  pdl_wait();
+  pdl_trigger();
   const int KB = cols / 16;
   const int64_t blk = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (blk >= rows * KB) return;
@@ -234,6 +246,8 @@ __global__ void __launch_bounds__(256) quantize_h_nvfp4_kernel(
     const __nv_bfloat16* __restrict__ h, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, int cols, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ counts, int E, const float* __restrict__ g_h, int dense) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int32_t s_cpre[1025];
   const int KB = cols / 16;
   int64_t n_rows = dense;
@@ -272,6 +286,8 @@ __global__ void __launch_bounds__(256) quantize_h_nvfp4_kernel(
 // Expert-major gather of NVFP4 rows (packed codes, H/2 bytes per row) and
 // their scale words (4 blocks of 16 per 32-bit word).
 __global__ void __launch_bounds__(256) permute_gather_nv_kernel(GatherMxArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int rows = a.offsets[a.E];
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;

@@ -46,6 +46,8 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
 
 template <int PER>
 __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(SelArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sb[kSelWarps][kSelMaxPerLane * 32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kSelWarps + w;
@@ -159,6 +161,8 @@ struct PermArgs {
 };
 
 __global__ void __launch_bounds__(256) permute_hist_kernel(PermArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t h[];
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) h[e] = 0;
   __syncthreads();
@@ -179,6 +183,8 @@ __global__ void __launch_bounds__(256) permute_hist_kernel(PermArgs a) {
 // A warp per expert: exclusive scan of the expert's tile counts (hist row
 // [e][0..ntiles), contiguous) into tile bases, and counts[e].
 __global__ void __launch_bounds__(256) permute_scan_kernel(PermArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (e >= a.E) return;
@@ -204,6 +210,8 @@ __global__ void __launch_bounds__(256) permute_scan_kernel(PermArgs a) {
 // with -1 (a grid-stride pass over r_cap); then warp 0 walks the tile's
 // entries in order and assigns stable slots.
 __global__ void __launch_bounds__(256) permute_rank_kernel(PermArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int32_t s_off[kMaxExpertsPerm + 1];
   __shared__ int32_t run[kMaxExpertsPerm];
   block_scan_padded(a.counts, a.E, a.P, s_off);
@@ -269,6 +277,8 @@ struct GatherArgs {
 };
 
 __global__ void __launch_bounds__(256) permute_gather_kernel(GatherArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int rows = a.offsets[a.E];
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int vecs = a.row_bytes >> 4;
@@ -311,6 +321,8 @@ __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& raw, fl
 // the loads of all K rows before accumulating them in j order.
 template <int K>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int kk = (K > 0) ? K : a.k;
   int rows[K > 0 ? K : 32];
