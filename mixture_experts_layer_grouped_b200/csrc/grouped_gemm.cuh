@@ -219,8 +219,26 @@ __device__ __forceinline__ void commit_x(uint64_t* bar) {
   }
 }
 
-// silu(g) = g * sigmoid(g); fast exp and division (well inside bf16 rounding).
-__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g).  e^-g comes from the hardware exponential (one
+// multi-function-unit op); 1 / (1 + e^-g) is refined from a bit-pattern seed
+// (relative error below 6%) by three Newton-Raphson steps r <- r (2 - d r) on the
+// FMA pipe, which leaves it within about one fp32 ulp.  Arguments below -80 are
+// clamped there (silu is then below 1e-32 in magnitude either way).  Keeping
+// the epilogue to one multi-function op per element (plus one packed bf16
+// conversion per two) is what bounds its time.
+__device__ __forceinline__ float silu_f(float g) {
+  const float d = 1.0f + __expf(-fmaxf(g, -80.0f));
+  float r = __int_as_float(0x7EF311C3 - __float_as_int(d));
+#pragma unroll
+  for (int i = 0; i < 3; ++i) r = fmaf(r, fmaf(-d, r, 1.0f), r);
+  return g * r;
+}
+
+// bf16 pair (a in the low half) as one 32-bit word, one packed conversion.
+__device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
 
 // PAIR: the kernel runs as clusters of two CTAs; rank 0 issues M = 256 MMAs
 // over both CTAs' shared memory (cta_group::2), each CTA loads its own 128
@@ -619,7 +637,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed, rank);
       if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
-      const GemmGroup& G = p.g[t.grp];
+      // per-tile values in registers: the parameter block is reached through a
+      // generic pointer once indexed by t.grp, and loads through it could not be
+      // hoisted past the epilogue's global stores
+      const GemmGroup G = p.g[t.grp];
+      uint8_t* const q_out = p.q_out[t.grp];
+      uint8_t* const q_sf = p.q_sf[t.grp];
+      float* const amax_out = p.amax_out[t.grp] + t.e * p.amax_stride[t.grp];
       const uint32_t lane_addr =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::ACC_COLS;
       const int f_base = t.f0 + quarter * 32;
@@ -629,6 +653,76 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         alpha = 1.0f / (__ldg(p.ga[t.grp] + t.e * p.ga_stride[t.grp]) *
                         __ldg(p.gw[t.grp] + t.e * p.gw_stride[t.grp]));
       float hmax = 0.f;  // fc1 NVFP4: amax of this warp's bf16 h values
+      if constexpr (MODE == kFc1 && DT != kMXF8) {
+        // h of this warp's chunks (32 tokens each) goes from TMEM straight into
+        // registers as bf16 pairs, the accumulator is released, and only then
+        // are the rows staged and stored: the next tile's MMAs wait for the
+        // TMEM reads and the SwiGLU, not for the stores
+        constexpr int NCH = (TILE_N + 63) / 64;
+        uint32_t hp[NCH][16];
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          const int c0 = member * 32 + 64 * i;
+          if (c0 < t.n_tok) {
+            const int rows_here = min(32, t.n_tok - c0);
+            uint32_t r0[32], r1[32];
+            tmem_ld_32x32b_x32(lane_addr + c0, r0);
+            tmem_ld_32x32b_x32(lane_addr + TILE_N + c0, r1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const uint32_t w = bf16x2_bits(
+                  silu_f(__uint_as_float(r0[j]) * alpha) * (__uint_as_float(r1[j]) * alpha),
+                  silu_f(__uint_as_float(r0[j + 1]) * alpha) * (__uint_as_float(r1[j + 1]) * alpha));
+              if (DT == kNVF4) {  // bf16 -> fp32 is a shift
+                if (j < rows_here) hmax = fmaxf(hmax, fabsf(__uint_as_float(w << 16)));
+                if (j + 1 < rows_here) hmax = fmaxf(hmax, fabsf(__uint_as_float(w & 0xFFFF0000u)));
+              }
+              hp[i][j >> 1] = w;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR) mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));  // rank 0's barrier
+          else mbar_arrive(&acc_empty[acc]);
+        }
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(G.out);
+        const uint4* s4 = reinterpret_cast<const uint4*>(my_stg);
+        uint16_t* s = reinterpret_cast<uint16_t*>(my_stg);
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          const int c0 = member * 32 + 64 * i;
+          if (c0 < t.n_tok) {
+            const int rows_here = min(32, t.n_tok - c0);
+            // staged [32 tokens][32 features], then 16-byte row stores
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              s[j * 32 + lane] = static_cast<uint16_t>(hp[i][j >> 1] & 0xFFFFu);
+              s[(j + 1) * 32 + lane] = static_cast<uint16_t>(hp[i][j >> 1] >> 16);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int c = it * 32 + lane;
+              const int j = c >> 2, part = c & 3;
+              if (j < rows_here && f_base < G.a_valid_rows)
+                *reinterpret_cast<uint4*>(out + static_cast<int64_t>(t.row0 + c0 + j) * G.out_ld +
+                                          f_base + part * 8) = s4[j * 4 + part];
+            }
+            __syncwarp();
+          }
+        }
+        if (DT == kNVF4) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+            hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+          if (lane == 0 && hmax > 0.f && f_base < G.a_valid_rows)
+            atomic_max_nonneg(amax_out, hmax);
+        }
+        if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
+      } else {
       for (int c0 = member * 32; c0 < t.n_tok; c0 += 64) {
         const int rows_here = min(32, t.n_tok - c0);
         uint32_t r0[32], r1[32];
@@ -653,10 +747,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
           // are one MXFP8 block, quantized from registers without cross-lane work.
           constexpr int RS = 34;
           __nv_bfloat16* hs_ = reinterpret_cast<__nv_bfloat16*>(my_stg);
+          uint16_t* hs16 = reinterpret_cast<uint16_t*>(my_stg);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            hs_[j * RS + lane] = __float2bfloat16_rn(silu_f(__uint_as_float(r0[j])) *
-                                                     __uint_as_float(r1[j]));
+          for (int j = 0; j < 32; j += 2) {
+            const uint32_t w = bf16x2_bits(silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j]),
+                                           silu_f(__uint_as_float(r0[j + 1])) *
+                                               __uint_as_float(r1[j + 1]));
+            hs16[j * RS + lane] = static_cast<uint16_t>(w & 0xFFFFu);
+            hs16[(j + 1) * RS + lane] = static_cast<uint16_t>(w >> 16);
+          }
           __syncwarp();
           if (lane < rows_here && f_base < G.a_valid_rows) {
             float v[32];
@@ -679,10 +778,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
                      (static_cast<uint32_t>(to_e4m3(v[4 * i + 2] * inv)) << 16) |
                      (static_cast<uint32_t>(to_e4m3(v[4 * i + 3] * inv)) << 24);
             const int64_t r = t.row0 + c0 + lane;
-            uint4* dst = reinterpret_cast<uint4*>(p.q_out[t.grp] + r * G.out_ld + f_base);
+            uint4* dst = reinterpret_cast<uint4*>(q_out + r * G.out_ld + f_base);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
             dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            p.q_sf[t.grp][sf_offset(r, f_base / 32, static_cast<int>(G.out_ld) / 32)] =
+            q_sf[sf_offset(r, f_base / 32, static_cast<int>(G.out_ld) / 32)] =
                 static_cast<uint8_t>(code);
           }
           __syncwarp();
@@ -705,10 +804,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
               if (DT == kNVF4 && j < rows_here) hmax = fmaxf(hmax, fabsf(__bfloat162float(hb)));
             }
           } else {
+            uint16_t* s16 = reinterpret_cast<uint16_t*>(my_stg);
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              s[j * 32 + lane] =
-                  __float2bfloat16_rn(__uint_as_float(half ? r1[j] : r0[j]) * alpha);
+            for (int j = 0; j < 32; j += 2) {
+              const uint32_t w = bf16x2_bits(__uint_as_float(half ? r1[j] : r0[j]) * alpha,
+                                             __uint_as_float(half ? r1[j + 1] : r0[j + 1]) * alpha);
+              s16[j * 32 + lane] = static_cast<uint16_t>(w & 0xFFFFu);
+              s16[(j + 1) * 32 + lane] = static_cast<uint16_t>(w >> 16);
+            }
           }
           __syncwarp();
 #pragma unroll
@@ -734,9 +837,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
         if (lane == 0 && hmax > 0.f && f_base < G.a_valid_rows)
-          atomic_max_nonneg(p.amax_out[t.grp] + t.e * p.amax_stride[t.grp], hmax);
+          atomic_max_nonneg(amax_out, hmax);
       }
       if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
+      }  // generic epilogue
     }
   }
 
