@@ -580,3 +580,26 @@ __device__ __forceinline__ void pdl_trigger() {
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// One row copy by a warp: 16-byte vectors, the loads of eight vectors per lane
+// issued before their stores (a zero source pointer writes zeros).
+__device__ __forceinline__ void warp_copy_row(uint4* __restrict__ d, const uint4* __restrict__ s,
+                                              int vecs, int lane) {
+  for (int v0 = 0; v0 < vecs; v0 += 32 * 8) {
+    uint4 buf[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int v = v0 + i * 32 + lane;
+      buf[i] = (s && v < vecs) ? __ldg(s + v) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int v = v0 + i * 32 + lane;
+      if (v < vecs) d[v] = buf[i];
+    }
+  }
+}
+
+}  // namespace moe

@@ -127,14 +127,12 @@ __global__ void __launch_bounds__(256) permute_gather_mx_kernel(GatherMxArgs a) 
     uint4* d = reinterpret_cast<uint4*>(a.dst_codes + static_cast<int64_t>(r) * a.H);
     if (t >= 0) {
       const uint4* s = reinterpret_cast<const uint4*>(a.src_codes + static_cast<int64_t>(t) * a.H);
-      if (a.dst_codes)
-        for (int v = lane; v < vecs; v += 32) d[v] = __ldg(s + v);
+      if (a.dst_codes) warp_copy_row(d, s, vecs, lane);
       for (int w = lane; w < W; w += 32)
         *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) =
             *reinterpret_cast<const uint32_t*>(a.src_scales + sf_offset(t, 4 * w, KB));
     } else {
-      if (a.dst_codes)
-        for (int v = lane; v < vecs; v += 32) d[v] = make_uint4(0, 0, 0, 0);
+      if (a.dst_codes) warp_copy_row(d, nullptr, vecs, lane);
       for (int w = lane; w < W; w += 32)
         *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) = 0u;
     }
@@ -300,14 +298,12 @@ __global__ void __launch_bounds__(256) permute_gather_nv_kernel(GatherMxArgs a) 
     if (t >= 0) {
       const uint4* s =
           reinterpret_cast<const uint4*>(a.src_codes + static_cast<int64_t>(t) * row_bytes);
-      if (a.dst_codes)
-        for (int v = lane; v < vecs; v += 32) d[v] = __ldg(s + v);
+      if (a.dst_codes) warp_copy_row(d, s, vecs, lane);
       for (int w = lane; w < W; w += 32)
         *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) =
             *reinterpret_cast<const uint32_t*>(a.src_scales + sf_offset(t, 4 * w, KB));
     } else {
-      if (a.dst_codes)
-        for (int v = lane; v < vecs; v += 32) d[v] = make_uint4(0, 0, 0, 0);
+      if (a.dst_codes) warp_copy_row(d, nullptr, vecs, lane);
       for (int w = lane; w < W; w += 32)
         *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) = 0u;
     }

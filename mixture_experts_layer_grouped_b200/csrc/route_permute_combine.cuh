@@ -285,12 +285,10 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(GatherArgs a) {
   for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
     const int t = a.row_token[r];
     uint4* d = reinterpret_cast<uint4*>(a.dst + static_cast<int64_t>(r) * a.row_bytes);
-    if (t >= 0) {
-      const uint4* s = reinterpret_cast<const uint4*>(a.src + static_cast<int64_t>(t) * a.row_bytes);
-      for (int v = threadIdx.x & 31; v < vecs; v += 32) d[v] = __ldg(s + v);
-    } else {
-      for (int v = threadIdx.x & 31; v < vecs; v += 32) d[v] = make_uint4(0, 0, 0, 0);
-    }
+    const uint4* s =
+        t >= 0 ? reinterpret_cast<const uint4*>(a.src + static_cast<int64_t>(t) * a.row_bytes)
+               : nullptr;
+    warp_copy_row(d, s, vecs, threadIdx.x & 31);
   }
 }
 
