@@ -24,6 +24,18 @@
 // 32-column chunks) and write the outputs.  When the accumulators of
 // one tile use at most half of TMEM they are double-buffered, so the epilogue
 // of tile i overlaps the MMAs of tile i+1.
+//
+// CTA pairs (PAIR): clusters of two CTAs run one tile together with M = 256
+// MMAs (cta_group::2) issued by rank 0.  Each CTA holds its own 128 weight rows
+// and half of the tile's token rows, so a stage carries half the token bytes
+// and the ring gets a fourth stage; the accumulator of a CTA's 128 features
+// sits in its own TMEM.
+//
+// The ring is latency-bound: a stage slot cycles through TMA issue, arrival
+// (about 1.5-2 us under full HBM load), MMA and release, so the bytes of
+// weights in flight per SM set the streaming rate.  Stage layouts therefore
+// favour weight bytes (two 16 KB weight boxes per stage) over TMEM double
+// buffering.
 #pragma once
 
 #include "common.cuh"

@@ -188,6 +188,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Programmatic dependent launch is on unless MOE_PDL=0 (plain stream order,
+// e.g. for profilers that replay kernels one at a time).
+bool pdl_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MOE_PDL");
+    v = (e && atoi(e) == 0) ? 0 : 1;
+  }
+  return v == 1;
+}
+
 // Launch with programmatic dependent launch allowed: the kernel's CTAs may
 // start while the previous kernel in the stream is finishing (every library
 // kernel waits in pdl_wait() before it touches global memory), which hides the
@@ -204,7 +215,7 @@ moe_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
   MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
   return MOE_OK;
 }
@@ -323,7 +334,7 @@ moe_status launch_gemm(const GemmParams& p, int max_units, cudaStream_t s) {
   int clusters = n < max_units ? n : max_units;
   if (clusters < 1) return MOE_OK;
   cfg.gridDim = dim3(2 * clusters);
-  cfg.numAttrs = 2;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, p));
   return launch_check();
 }
@@ -656,17 +667,26 @@ moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void*
                           const void* x, const MlpQuant& q, const int32_t* counts,
                           const int32_t* offsets, void* out_rows, void* shared_out, void* ws,
                           cudaStream_t s) {
-  const bool pairs = use_pairs(c, rows);
-#define MOE_MLP(TN, DT)                                                                        \
-  return pairs ? grouped_mlp_tiles<TN, DT, true>(c, w, rows, x, q, counts, offsets, out_rows,  \
-                                                 shared_out, ws, s)                            \
-               : grouped_mlp_tiles<TN, DT, false>(c, w, rows, x, q, counts, offsets, out_rows, \
-                                                  shared_out, ws, s)
-  if (is_mx(c)) MOE_MLP(192, kMXF8);
-  if (is_nv(c))
-    return grouped_mlp_tiles<192, kNVF4, false>(c, w, rows, x, q, counts, offsets, out_rows,
-                                                shared_out, ws, s);
-  MOE_MLP(256, kBF16);
+  // Decode-sized batches (at most 32 rows per expert on average) take 64-token
+  // tiles: a stage holds far fewer token bytes (a fourth stage fits) and two
+  // accumulators fit TMEM, so each tile's epilogue overlaps the next tile.
+  const bool small = static_cast<int64_t>(c.T) * c.top_k <= 32LL * c.E;
+  const bool pairs = !small && use_pairs(c, rows);
+#define MOE_MLP(TN, DT, PR)                                                                      \
+  return grouped_mlp_tiles<TN, DT, PR>(c, w, rows, x, q, counts, offsets, out_rows, shared_out, \
+                                       ws, s)
+  if (is_mx(c)) {
+    if (small) MOE_MLP(64, kMXF8, false);
+    if (pairs) MOE_MLP(192, kMXF8, true);
+    MOE_MLP(192, kMXF8, false);
+  }
+  if (is_nv(c)) {
+    if (small) MOE_MLP(64, kNVF4, false);
+    MOE_MLP(192, kNVF4, false);
+  }
+  if (small) MOE_MLP(64, kBF16, false);
+  if (pairs) MOE_MLP(256, kBF16, true);
+  MOE_MLP(256, kBF16, false);
 #undef MOE_MLP
 }
 
