@@ -193,6 +193,18 @@ def run_reference(args, cfg):
 
 WEIGHT_BYTES = {"bf16": 2.0, "mxfp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}  # per element
 TENSOR_RATIO = {"bf16": 1.0, "mxfp8": 2.0, "nvfp4": 4.0}  # nominal dense peak vs bf16
+# DRAM bytes (read + written) of one grouped-MLP call's fc1 and fc2 kernels per
+# algorithmic weight byte, from the ncu counters summarised in
+# profiles/grouped_gemm_<workload>.md (full size for the mid workload; the others
+# captured on fewer experts with the same tokens per expert, so the ratio carries
+# over per touched expert).  Valid for the kernels those captures measured.
+TRAFFIC_RATIO = {
+    "mid_bf16_shared_T2048": 1.30,
+    "dsv4_bf16_T4096": 1.03,
+    "dsv3_mxfp8_shared_T4096": 1.12,
+    "dsv4_nvfp4_decode_T128": 1.01,
+    "dsv4_nvfp4_prefill_T8192": 1.13,
+}
 
 
 def grouped_mlp_algorithmic(cfg, touched):
@@ -408,7 +420,12 @@ def run_ours(args, cfg):
                                  % (WEIGHT_BYTES[cfg.dtype] * 3 * cfg.H * cfg.I * cfg.E / 1e6)),
                        launch="CUDA graph of the one-call forward", parallelism=f"replicas{ws_n}"),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved_gbs / hbm, "traffic": None,
+                     "frac": achieved_gbs / hbm,
+                     "traffic": (TRAFFIC_RATIO[cfg.name] * wbytes
+                                 if cfg.name in TRAFFIC_RATIO else None),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
+                                       "fc1 and fc2 launches (profiles/grouped_gemm_*.md), "
+                                       "bytes per grouped-MLP call",
                      "kernel": "moe_grouped_mlp (fc1+SwiGLU and fc2 tcgen05 kernels)",
                      "algorithmic_bytes_per_launch": wbytes, "ms_per_launch": mlp_ms,
                      "tensor_tflops": flops / (mlp_ms * 1e-3) / 1e12,
