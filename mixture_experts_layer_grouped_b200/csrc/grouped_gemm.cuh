@@ -158,15 +158,19 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
   using C = GemmCfg<MODE, TILE_N, DT, PAIR>;
   Tile t;
   if (u < units_routed) {
+    // expert e owns units [prefix[e] * ns, prefix[e + 1] * ns), slab-major: the
+    // token chunks of one weight slab are adjacent, so they run at about the same
+    // time and the slab's later reads hit L2
     const int ns = p.g[0].n_slabs;
-    const int q = u / ns;
-    t.slab = u - q * ns;
     int lo = 0, hi = p.E;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (prefix[mid] <= q) lo = mid; else hi = mid;
+      if (prefix[mid] * ns <= u) lo = mid; else hi = mid;
     }
-    const int chunk = q - prefix[lo];
+    const int nch = prefix[lo + 1] - prefix[lo];
+    const int v = u - prefix[lo] * ns;
+    t.slab = v / nch;
+    const int chunk = v - t.slab * nch;
     t.grp = 0;
     t.e = lo;
     t.row0 = __ldg(p.offsets + lo) + chunk * TILE_N;
