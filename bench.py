@@ -122,6 +122,35 @@ def _dist():
     return ws, rank, local
 
 
+# Replicas: the layer shards by batch with no exchange.  Every rank holds the
+# same weights and runs its own batch of T tokens (drawn with seed = rank); the
+# job's time is the slowest rank's, and its throughput counts every rank's tokens.
+
+def replica_config(cfg, rank):
+    """The seeds a rank draws its token batch with (same shapes)."""
+    return cfg.scaled(seed=rank) if rank else cfg
+
+
+def replica_inputs(cfg, rank, device):
+    """A rank's inputs: its own token batch, the job's router weights and bias
+    (expert weights are drawn from `cfg` as well, in prepare_streaming)."""
+    w_router, bias = synth.gen_router(cfg, device)
+    return synth.gen_x(replica_config(cfg, rank), device), w_router, bias
+
+
+def max_over_ranks(value, dist, device):
+    """The largest of every rank's value (each rank passes its own)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank, n_ranks, ms_max):
+    return n_ranks * tokens_per_rank / (ms_max * 1e-3)
+
+
 # ---------------------------------------------------------------------------
 # reference arm: the CPU oracle
 # ---------------------------------------------------------------------------
@@ -268,8 +297,7 @@ def run_ours(args, cfg):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     c = M.config_from_shape(cfg)
-    d = {"x": synth.gen_x(cfg.scaled(seed=rank) if rank else cfg, dev)}  # each rank its batch
-    d["w_router"], d["bias"] = synth.gen_router(cfg, dev)
+    d = dict(zip(("x", "w_router", "bias"), replica_inputs(cfg, rank, dev)))
     layer = M.MoELayer(c, prepare_streaming(M, cfg, c, dev), d["w_router"], d["bias"],
                        prepared=True)
     x, y = d["x"], torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
@@ -314,12 +342,8 @@ def run_ours(args, cfg):
     clk.__exit__(None, None, None)
     ms = ev0.elapsed_time(ev1) / args.steps
     barrier()
-    ms_max = ms
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    value = ws_n * cfg.T / (ms_max * 1e-3)
+    ms_max = max_over_ranks(ms, dist, dev)
+    value = job_tokens_per_s(cfg.T, ws_n, ms_max)
 
     # ---- e2e: host (pinned) buffers through the same C call, eager
     x_h = x.cpu().pin_memory()
@@ -333,11 +357,8 @@ def run_ours(args, cfg):
     ev1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = ev0.elapsed_time(ev1) / args.steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = ws_n * cfg.T / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    e2e_value = job_tokens_per_s(cfg.T, ws_n, e2e_ms)
 
     # ---- roofline of the dominant call (grouped MLP: fc1+SwiGLU and fc2)
     nbytes, r_cap = M.moe_workspace_size(c)
