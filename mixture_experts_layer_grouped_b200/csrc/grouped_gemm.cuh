@@ -738,6 +738,115 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             atomic_max_nonneg(amax_out, hmax);
         }
         if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
+      } else if constexpr ((MODE == kFc2 && TILE_N <= 192) || (MODE == kFc1 && DT == kMXF8)) {
+        // As above: TMEM -> registers (packed bf16), release the accumulator,
+        // then stage and store.  fc2 keeps both 128-feature halves of its chunks
+        // (up to 192-token tiles: 96 registers; 256-token tiles would spill);
+        // MXFP8 fc1 keeps h, quantized after the release.
+        constexpr int NCH = (TILE_N + 63) / 64;
+        constexpr int NH = (MODE == kFc2) ? 2 : 1;
+        uint32_t hp[NCH][NH][16];
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          const int c0 = member * 32 + 64 * i;
+          if (c0 < t.n_tok) {
+            uint32_t r0[32], r1[32];
+            tmem_ld_32x32b_x32(lane_addr + c0, r0);
+            tmem_ld_32x32b_x32(lane_addr + TILE_N + c0, r1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              if (MODE == kFc2) {
+                hp[i][0][j >> 1] = bf16x2_bits(__uint_as_float(r0[j]) * alpha,
+                                               __uint_as_float(r0[j + 1]) * alpha);
+                hp[i][NH - 1][j >> 1] = bf16x2_bits(__uint_as_float(r1[j]) * alpha,
+                                                    __uint_as_float(r1[j + 1]) * alpha);
+              } else {
+                hp[i][0][j >> 1] =
+                    bf16x2_bits(silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j]),
+                                silu_f(__uint_as_float(r0[j + 1])) * __uint_as_float(r1[j + 1]));
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR) mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));  // rank 0's barrier
+          else mbar_arrive(&acc_empty[acc]);
+        }
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          const int c0 = member * 32 + 64 * i;
+          if (c0 >= t.n_tok) continue;
+          const int rows_here = min(32, t.n_tok - c0);
+          if constexpr (MODE == kFc2) {
+            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(G.out);
+            const uint4* s4 = reinterpret_cast<const uint4*>(my_stg);
+            uint16_t* s16 = reinterpret_cast<uint16_t*>(my_stg);
+#pragma unroll
+            for (int half = 0; half < NH; ++half) {
+              const int f0 = f_base + half * kBM;
+#pragma unroll
+              for (int j = 0; j < 32; j += 2) {
+                s16[j * 32 + lane] = static_cast<uint16_t>(hp[i][half][j >> 1] & 0xFFFFu);
+                s16[(j + 1) * 32 + lane] = static_cast<uint16_t>(hp[i][half][j >> 1] >> 16);
+              }
+              __syncwarp();
+#pragma unroll
+              for (int it = 0; it < 4; ++it) {
+                const int c = it * 32 + lane;
+                const int j = c >> 2, part = c & 3;
+                if (j < rows_here && f0 < G.a_valid_rows)
+                  *reinterpret_cast<uint4*>(out + static_cast<int64_t>(t.row0 + c0 + j) *
+                                                      G.out_ld + f0 + part * 8) = s4[j * 4 + part];
+              }
+              __syncwarp();
+            }
+          } else {
+            // h staged [32 tokens][32 features] (row stride 34 bf16 to spread banks);
+            // then lane j takes token j: the warp's 32 features are one MXFP8 block,
+            // quantized from registers without cross-lane work
+            constexpr int RS = 34;
+            uint16_t* hs16 = reinterpret_cast<uint16_t*>(my_stg);
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              hs16[j * RS + lane] = static_cast<uint16_t>(hp[i][0][j >> 1] & 0xFFFFu);
+              hs16[(j + 1) * RS + lane] = static_cast<uint16_t>(hp[i][0][j >> 1] >> 16);
+            }
+            __syncwarp();
+            if (lane < rows_here && f_base < G.a_valid_rows) {
+              float v[32];
+              float amax = 0.f;
+              const __nv_bfloat162* row =
+                  reinterpret_cast<const __nv_bfloat162*>(hs16 + lane * RS);
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const float2 f = __bfloat1622float2(row[q]);
+                v[2 * q] = f.x;
+                v[2 * q + 1] = f.y;
+                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+              }
+              const uint32_t code = mx_scale_code(amax);
+              const float inv = mx_inv_scale(code);
+              uint32_t w[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                w[q] = static_cast<uint32_t>(to_e4m3(v[4 * q] * inv)) |
+                       (static_cast<uint32_t>(to_e4m3(v[4 * q + 1] * inv)) << 8) |
+                       (static_cast<uint32_t>(to_e4m3(v[4 * q + 2] * inv)) << 16) |
+                       (static_cast<uint32_t>(to_e4m3(v[4 * q + 3] * inv)) << 24);
+              const int64_t r = t.row0 + c0 + lane;
+              uint4* dst = reinterpret_cast<uint4*>(q_out + r * G.out_ld + f_base);
+              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              q_sf[sf_offset(r, f_base / 32, static_cast<int>(G.out_ld) / 32)] =
+                  static_cast<uint8_t>(code);
+            }
+            __syncwarp();
+          }
+        }
+        if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
       } else {
       for (int c0 = member * 32; c0 < t.n_tok; c0 += 64) {
         const int rows_here = min(32, t.n_tok - c0);
