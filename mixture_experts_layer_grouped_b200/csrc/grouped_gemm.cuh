@@ -256,6 +256,55 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Two fp32 values in one 64-bit register pair, for the sm_100 packed f32x2
+// add / mul / fma: one instruction computes both halves, each rounded exactly
+// as its scalar form would be.
+__device__ __forceinline__ uint64_t f32x2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// bf16(silu(g0) * u0) and bf16(silu(g1) * u1) as one word: silu_f's steps for
+// two accumulator columns at once -- the exponentials one by one, then the
+// add, the three Newton-Raphson steps and both products as packed f32x2
+// instructions.  Same operations and roundings as silu_f(g) * u (bit-identical
+// results) in about half the FMA-pipe issue slots, which bound the fc1
+// epilogue and with it the gap between two tiles' MMAs.
+__device__ __forceinline__ uint32_t swiglu_bf16x2(float g0, float g1, float u0, float u1) {
+  const float e0 = __expf(-fmaxf(g0, -80.0f)), e1 = __expf(-fmaxf(g1, -80.0f));
+  const uint64_t one = f32x2_pack(1.0f, 1.0f);
+  const uint64_t d = f32x2_add(one, f32x2_pack(e0, e1));
+  float d0, d1;
+  f32x2_unpack(d, d0, d1);
+  uint64_t r = f32x2_pack(__int_as_float(0x7EF311C3 - __float_as_int(d0)),
+                          __int_as_float(0x7EF311C3 - __float_as_int(d1)));
+  const uint64_t nd = f32x2_pack(-d0, -d1);
+#pragma unroll
+  for (int i = 0; i < 3; ++i) r = f32x2_fma(r, f32x2_fma(nd, r, one), r);
+  float h0, h1;
+  f32x2_unpack(f32x2_mul(f32x2_mul(f32x2_pack(g0, g1), r), f32x2_pack(u0, u1)), h0, h1);
+  return bf16x2_bits(h0, h1);
+}
+
 // PAIR: the kernel runs as clusters of two CTAs; rank 0 issues M = 256 MMAs
 // over both CTAs' shared memory (cta_group::2), each CTA loads its own 128
 // weight rows and half of the tile's token rows, and the loads of both count
@@ -651,11 +700,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     uint32_t acc_phase = 0;
     for (int u = group_id; u < units; u += n_groups) {
       const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed, rank);
-      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status)) break;
-      tc_fence_after();
-      // per-tile values in registers: the parameter block is reached through a
-      // generic pointer once indexed by t.grp, and loads through it could not be
-      // hoisted past the epilogue's global stores
+      // per-tile values in registers, loaded while the MMAs still run: the
+      // parameter block is reached through a generic pointer once indexed by
+      // t.grp, and loads through it could not be hoisted past the epilogue's
+      // global stores
       const GemmGroup G = p.g[t.grp];
       uint8_t* const q_out = p.q_out[t.grp];
       uint8_t* const q_sf = p.q_sf[t.grp];
@@ -668,6 +716,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       if (DT == kNVF4)
         alpha = 1.0f / (__ldg(p.ga[t.grp] + t.e * p.ga_stride[t.grp]) *
                         __ldg(p.gw[t.grp] + t.e * p.gw_stride[t.grp]));
+      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status)) break;
+      tc_fence_after();
       float hmax = 0.f;  // fc1 NVFP4: amax of this warp's bf16 h values
       if constexpr (MODE == kFc1 && DT != kMXF8) {
         // h of this warp's chunks (32 tokens each) goes from TMEM straight into
@@ -687,9 +737,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              const uint32_t w = bf16x2_bits(
-                  silu_f(__uint_as_float(r0[j]) * alpha) * (__uint_as_float(r1[j]) * alpha),
-                  silu_f(__uint_as_float(r0[j + 1]) * alpha) * (__uint_as_float(r1[j + 1]) * alpha));
+              float g0 = __uint_as_float(r0[j]), g1 = __uint_as_float(r0[j + 1]);
+              float u0 = __uint_as_float(r1[j]), u1 = __uint_as_float(r1[j + 1]);
+              if constexpr (DT == kNVF4) {  // bf16: alpha is 1
+                g0 *= alpha; g1 *= alpha; u0 *= alpha; u1 *= alpha;
+              }
+              const uint32_t w = swiglu_bf16x2(g0, g1, u0, u1);
               if (DT == kNVF4) {  // bf16 -> fp32 is a shift
                 if (j < rows_here) hmax = fmaxf(hmax, fabsf(__uint_as_float(w << 16)));
                 if (j + 1 < rows_here) hmax = fmaxf(hmax, fabsf(__uint_as_float(w & 0xFFFF0000u)));
@@ -762,9 +815,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
                 hp[i][NH - 1][j >> 1] = bf16x2_bits(__uint_as_float(r1[j]) * alpha,
                                                     __uint_as_float(r1[j + 1]) * alpha);
               } else {
-                hp[i][0][j >> 1] =
-                    bf16x2_bits(silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j]),
-                                silu_f(__uint_as_float(r0[j + 1])) * __uint_as_float(r1[j + 1]));
+                hp[i][0][j >> 1] = swiglu_bf16x2(__uint_as_float(r0[j]), __uint_as_float(r0[j + 1]),
+                                                 __uint_as_float(r1[j]), __uint_as_float(r1[j + 1]));
               }
             }
           }
