@@ -50,14 +50,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// One bounded test of a phase.  The thread may sleep in it until the phase
+// completes, for at most kSuspendNs: waiting warps then leave their issue slots
+// to the warps that work (a GEMM's idle epilogue warps sleep through the main
+// loop instead of polling beside the producer and MMA warps).
+constexpr uint32_t kSuspendNs = 20000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -590,15 +595,16 @@ __device__ __forceinline__ void pdl_trigger() {
 namespace moe {
 
 // One row copy by a warp: 16-byte vectors, the loads of eight vectors per lane
-// issued before their stores (a zero source pointer writes zeros).
-__device__ __forceinline__ void warp_copy_row(uint4* __restrict__ d, const uint4* __restrict__ s,
-                                              int vecs, int lane) {
+// issued before their stores (a zero source pointer writes zeros).  Plain
+// loads on pointers that may alias the destination: the compiler cannot sink
+// them to their stores, so the eight stay in flight together.
+__device__ __forceinline__ void warp_copy_row(uint4* d, const uint4* s, int vecs, int lane) {
   for (int v0 = 0; v0 < vecs; v0 += 32 * 8) {
     uint4 buf[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int v = v0 + i * 32 + lane;
-      buf[i] = (s && v < vecs) ? __ldg(s + v) : make_uint4(0, 0, 0, 0);
+      buf[i] = (s && v < vecs) ? s[v] : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {

@@ -35,18 +35,23 @@ struct StepLayout {
 };
 
 // Router GEMM tiling: 256-token tiles for long batches (W_r re-read per tile
-// is then negligible), 64 otherwise; K split into at most kMaxSplits parts so
-// that about one wave of tiles covers the SMs.
+// is then negligible), 64 otherwise; K split into at most kMaxSplits parts,
+// the count that minimises the rounds of units over the 148 SMs times the
+// k-steps of one unit (ties to fewer splits: less partial-sum traffic).
 int router_tile_of(const moe_config& c) { return c.T >= 4096 ? 256 : 64; }
 
 int router_splits_of(const moe_config& c) {
   const int tn = router_tile_of(c);
   const int units = ((c.T + tn - 1) / tn) * ((c.E + kBM - 1) / kBM);
   const int k_tiles = c.H / kBK;
-  int s = (148 + units - 1) / units;
-  s = s < kMaxSplits ? s : kMaxSplits;
-  s = s < k_tiles / 4 ? s : k_tiles / 4;
-  return s < 1 ? 1 : s;
+  int best = 1;
+  int64_t best_cost = -1;
+  for (int s = 1; s <= kMaxSplits && s <= (k_tiles / 4 > 0 ? k_tiles / 4 : 1); ++s) {
+    const int64_t rounds = (static_cast<int64_t>(units) * s + 147) / 148;
+    const int64_t cost = rounds * ((k_tiles + s - 1) / s);
+    if (best_cost < 0 || cost < best_cost) { best = s; best_cost = cost; }
+  }
+  return best;
 }
 
 int32_t r_cap_of(const moe_config& c) {
@@ -441,8 +446,18 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
     g.offsets = offsets;
     g.E = c.E;
     g.H = c.H;
-    if (is_nv(c)) MOE_TRY(launch_pdl(permute_gather_nv_kernel, dim3(sm_count() * 4), dim3(256), 0, s, g));
-    else MOE_TRY(launch_pdl(permute_gather_mx_kernel, dim3(sm_count() * 4), dim3(256), 0, s, g));
+    const int row_bytes = is_nv(c) ? c.H / 2 : c.H;
+    const int KB = is_nv(c) ? c.H / 16 : c.H / 32;
+    const int vpl = (row_bytes / 16 + 31) / 32;  // 16-byte vectors per lane
+    const dim3 grid(sm_count() * 4), block(256);
+    if (KB / 4 <= 256 && vpl <= 8)
+      MOE_TRY(launch_pdl(permute_gather_bs_kernel<8>, grid, block, 0, s, g, row_bytes, KB));
+    else if (KB / 4 <= 256 && vpl <= 16)
+      MOE_TRY(launch_pdl(permute_gather_bs_kernel<16>, grid, block, 0, s, g, row_bytes, KB));
+    else if (is_nv(c))
+      MOE_TRY(launch_pdl(permute_gather_nv_kernel, grid, block, 0, s, g));
+    else
+      MOE_TRY(launch_pdl(permute_gather_mx_kernel, grid, block, 0, s, g));
     return launch_check();
   }
   if (!dst_rows) return MOE_OK;  // rows are gathered later by the grouped GEMM
@@ -453,7 +468,12 @@ moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* 
   g.offsets = offsets;
   g.E = c.E;
   g.row_bytes = c.H * 2;
-  MOE_TRY(launch_pdl(permute_gather_kernel, dim3(sm_count() * 4), dim3(256), 0, s, g));
+  const int vpl = (g.row_bytes / 16 + 31) / 32;  // 16-byte vectors per lane
+  const dim3 grid(sm_count() * 4), block(256);
+  if (vpl <= 8) MOE_TRY(launch_pdl(permute_gather_row_kernel<8>, grid, block, 0, s, g));
+  else if (vpl <= 16) MOE_TRY(launch_pdl(permute_gather_row_kernel<16>, grid, block, 0, s, g));
+  else if (vpl <= 32) MOE_TRY(launch_pdl(permute_gather_row_kernel<32>, grid, block, 0, s, g));
+  else MOE_TRY(launch_pdl(permute_gather_kernel, grid, block, 0, s, g));
   return launch_check();
 }
 

@@ -281,6 +281,60 @@ __global__ void __launch_bounds__(256) quantize_h_nvfp4_kernel(
   }
 }
 
+// One-round form of the block-scaled gathers (MXFP8: row_bytes = H, KB = H/32;
+// NVFP4: row_bytes = H/2, KB = H/16) for rows of at most 32 * MAXV vectors and
+// 256 scale words: all loads of a row, codes and scale words, are issued before
+// its first store, and the next row's token index is read one row ahead, so a
+// warp waits about one memory latency per row instead of one per 8 vectors
+// and one per 32 scale words.  (Plain loads: the compiler may not move them
+// past the stores, which could alias, so all of them stay in flight at once;
+// read-only loads let it sink each load to its store and serialize the row.)
+template <int MAXV>
+__global__ void __launch_bounds__(256) permute_gather_bs_kernel(GatherMxArgs a, int row_bytes,
+                                                                int KB) {
+  constexpr int MAXW = 8;
+  pdl_wait();
+  pdl_trigger();
+  const int rows = a.offsets[a.E];
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int vecs = row_bytes >> 4, W = KB / 4;
+  int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int t = r < rows ? a.row_token[r] : -1;
+  for (; r < rows; r += warps) {
+    const int t_next = r + warps < rows ? a.row_token[r + warps] : -1;
+    const uint4* src = (t >= 0 && a.dst_codes)
+                           ? reinterpret_cast<const uint4*>(a.src_codes + static_cast<int64_t>(t) * row_bytes)
+                           : nullptr;
+    uint4 buf[MAXV];
+    uint32_t sw[MAXW];
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = i * 32 + lane;
+      buf[i] = (src && v < vecs) ? src[v] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < MAXW; ++i) {
+      const int w = i * 32 + lane;
+      sw[i] = (t >= 0 && w < W)
+                  ? *reinterpret_cast<const uint32_t*>(a.src_scales + sf_offset(t, 4 * w, KB))
+                  : 0u;
+    }
+    if (a.dst_codes) {
+      uint4* d = reinterpret_cast<uint4*>(a.dst_codes + static_cast<int64_t>(r) * row_bytes);
+#pragma unroll
+      for (int i = 0; i < MAXV; ++i)
+        if (i * 32 + lane < vecs) d[i * 32 + lane] = buf[i];
+    }
+#pragma unroll
+    for (int i = 0; i < MAXW; ++i) {
+      const int w = i * 32 + lane;
+      if (w < W) *reinterpret_cast<uint32_t*>(a.dst_scales + sf_offset(r, 4 * w, KB)) = sw[i];
+    }
+    t = t_next;
+  }
+}
+
 // Expert-major gather of NVFP4 rows (packed codes, H/2 bytes per row) and
 // their scale words (4 blocks of 16 per 32-bit word).
 __global__ void __launch_bounds__(256) permute_gather_nv_kernel(GatherMxArgs a) {

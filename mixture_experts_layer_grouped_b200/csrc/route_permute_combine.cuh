@@ -292,6 +292,39 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(GatherArgs a) {
   }
 }
 
+// One-round form of the row gather for rows of at most 32 * MAXV vectors: all
+// loads of a row are issued before its first store and the next row's token
+// index is read one row ahead (about one memory latency per row and warp).
+// Plain loads keep all of them ahead of the stores (see permute_gather_bs_kernel).
+template <int MAXV>
+__global__ void __launch_bounds__(256) permute_gather_row_kernel(GatherArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  const int rows = a.offsets[a.E];
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int vecs = a.row_bytes >> 4;
+  int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int t = r < rows ? a.row_token[r] : -1;
+  for (; r < rows; r += warps) {
+    const int t_next = r + warps < rows ? a.row_token[r + warps] : -1;
+    const uint4* src =
+        t >= 0 ? reinterpret_cast<const uint4*>(a.src + static_cast<int64_t>(t) * a.row_bytes)
+               : nullptr;
+    uint4 buf[MAXV];
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = i * 32 + lane;
+      buf[i] = (src && v < vecs) ? src[v] : make_uint4(0, 0, 0, 0);
+    }
+    uint4* d = reinterpret_cast<uint4*>(a.dst + static_cast<int64_t>(r) * a.row_bytes);
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i)
+      if (i * 32 + lane < vecs) d[i * 32 + lane] = buf[i];
+    t = t_next;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Combine: y[t] = bf16(sum_j w[t,j] * out_rows[token_row[t*k+j]] + shared[t]),
 // fp32 accumulation in j order.  One warp per token, 8 bf16 per lane-vector.

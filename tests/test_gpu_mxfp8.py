@@ -100,9 +100,20 @@ def _routing(cfg):
     return O.route(f64(logits), f64(bias), cfg.n_group, cfg.topk_group, cfg.top_k, cfg.rsf)
 
 
-@pytest.mark.parametrize("name", list(MX))
+# permute-only shapes for the other gather forms: 14 and 17 code vectors per lane
+MX_WIDE = {
+    "wide_mx": synth.MoEShape(name="wide_mx", T=96, H=7168, I=128, E=16, n_group=4, topk_group=2,
+                              top_k=4, rsf=2.5, I_shared=0, dtype="mxfp8", pad_multiple=64,
+                              router_std=0.02),
+    "wider_mx": synth.MoEShape(name="wider_mx", T=96, H=8448, I=128, E=16, n_group=4,
+                               topk_group=2, top_k=4, rsf=2.5, I_shared=0, dtype="mxfp8",
+                               pad_multiple=64, router_std=0.02),
+}
+
+
+@pytest.mark.parametrize("name", list(MX) + list(MX_WIDE))
 def test_permute_mxfp8(M, name):
-    cfg = MX[name]
+    cfg = MX[name] if name in MX else MX_WIDE[name]
     c = M.config_from_shape(cfg)
     r = _routing(cfg)
     m = O.permute_maps(r["idx"], cfg.E, cfg.pad_multiple)

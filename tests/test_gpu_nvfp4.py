@@ -109,9 +109,20 @@ def _routing(cfg):
     return O.route(f64(logits), f64(bias), cfg.n_group, cfg.topk_group, cfg.top_k, cfg.rsf)
 
 
-@pytest.mark.parametrize("name", list(NV))
+# permute-only shapes for the other gather forms: 7 and 17 code vectors per lane
+NV_WIDE = {
+    "wide_nv": synth.MoEShape(name="wide_nv", T=96, H=7168, I=256, E=16, n_group=4, topk_group=2,
+                              top_k=4, rsf=2.5, I_shared=0, dtype="nvfp4", pad_multiple=64,
+                              router_std=0.02),
+    "wider_nv": synth.MoEShape(name="wider_nv", T=96, H=16640, I=256, E=16, n_group=4,
+                               topk_group=2, top_k=4, rsf=2.5, I_shared=0, dtype="nvfp4",
+                               pad_multiple=64, router_std=0.02),
+}
+
+
+@pytest.mark.parametrize("name", list(NV) + list(NV_WIDE))
 def test_permute_nvfp4(M, name):
-    cfg = NV[name]
+    cfg = NV[name] if name in NV else NV_WIDE[name]
     c = M.config_from_shape(cfg)
     r = _routing(cfg)
     m = O.permute_maps(r["idx"], cfg.E, cfg.pad_multiple)

@@ -37,6 +37,18 @@ EDGE = {
 }
 
 
+# permute-only shapes whose rows take the other gather forms: 28 and 33
+# 16-byte vectors per lane (the 32-vector one-round kernel and the looping one)
+WIDE = {
+    "rows_h7168": synth.MoEShape(name="edge_rows_h7168", T=96, H=7168, I=128, E=16, n_group=4,
+                                 topk_group=2, top_k=4, rsf=2.5, I_shared=0, dtype="bf16",
+                                 pad_multiple=8, router_std=0.02),
+    "rows_h8448": synth.MoEShape(name="edge_rows_h8448", T=96, H=8448, I=128, E=16, n_group=4,
+                                 topk_group=2, top_k=4, rsf=2.5, I_shared=0, dtype="bf16",
+                                 pad_multiple=8, router_std=0.02),
+}
+
+
 @pytest.fixture(scope="module")
 def M():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
@@ -46,6 +58,8 @@ def M():
 
 
 def _cfg(name):
+    if name in WIDE:
+        return WIDE[name]
     return EDGE[name] if name in EDGE else synth.get_config(name)
 
 
@@ -99,8 +113,10 @@ def test_router_gemm(M, name):
 
 # ---------------------------------------------------------------- permute
 @pytest.mark.parametrize("name", ["tiny_bf16_T64", "mid_bf16_shared_T2048", "dsv4_bf16_T4096"]
-                         + list(EDGE))
+                         + list(EDGE) + list(WIDE))
 def test_permute_bit_exact(M, name):
+    """Counts, offsets, slots and every gather form against the oracle's maps
+    and rows."""
     cfg = _cfg(name)
     c = M.config_from_shape(cfg)
     _, bias = synth.gen_router(cfg, "cuda")
