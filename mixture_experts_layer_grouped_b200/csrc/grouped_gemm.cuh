@@ -791,18 +791,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             atomic_max_nonneg(amax_out, hmax);
         }
         if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
-      } else if constexpr ((MODE == kFc2 && TILE_N <= 192) || (MODE == kFc1 && DT == kMXF8)) {
+      } else if constexpr (MODE == kFc2 || (MODE == kFc1 && DT == kMXF8)) {
         // As above: TMEM -> registers (packed bf16), release the accumulator,
         // then stage and store.  fc2 keeps both 128-feature halves of its chunks
-        // (up to 192-token tiles: 96 registers; 256-token tiles would spill);
-        // MXFP8 fc1 keeps h, quantized after the release.
+        // (128 registers for 256-token tiles, which therefore read 16 columns
+        // at a time: 16 raw registers live instead of 64, within the 168 a
+        // thread gets); MXFP8 fc1 keeps h, quantized after the release.
         constexpr int NCH = (TILE_N + 63) / 64;
         constexpr int NH = (MODE == kFc2) ? 2 : 1;
         uint32_t hp[NCH][NH][16];
 #pragma unroll
         for (int i = 0; i < NCH; ++i) {
           const int c0 = member * 32 + 64 * i;
-          if (c0 < t.n_tok) {
+          if (MODE == kFc2 && TILE_N > 192 && c0 < t.n_tok) {
+#pragma unroll
+            for (int q = 0; q < 2 * NH; ++q) {  // (half, 16-column part)
+              uint32_t r[16];
+              tmem_ld_32x32b_x16(lane_addr + (q >> 1) * TILE_N + c0 + (q & 1) * 16, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 16; j += 2)
+                hp[i][q >> 1][(q & 1) * 8 + (j >> 1)] =
+                    bf16x2_bits(__uint_as_float(r[j]) * alpha, __uint_as_float(r[j + 1]) * alpha);
+            }
+          } else if (c0 < t.n_tok) {
             uint32_t r0[32], r1[32];
             tmem_ld_32x32b_x32(lane_addr + c0, r0);
             tmem_ld_32x32b_x32(lane_addr + TILE_N + c0, r1);
