@@ -85,6 +85,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Wait until the 32-bit counter at p reaches `target` (acquire, GPU scope),
+// sleeping between polls; the same limit and abort handling as mbar_wait.
+__device__ __forceinline__ bool counter_wait(const int32_t* p, int32_t target, volatile int* abort,
+                                             int32_t* status, uint64_t limit_ns = 2000000000ull) {
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if (v >= target) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      set_status(status, MOE_ERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(200);
+  }
+}
+
+// Orders this thread's earlier generic-proxy accesses (an acquire above) before
+// its later async-proxy (TMA) accesses to global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // --------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // --------------------------------------------------------------------------

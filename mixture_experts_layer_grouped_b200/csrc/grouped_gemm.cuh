@@ -96,6 +96,14 @@ struct GemmParams {
   int32_t E;               // routed experts (0: no routed group)
   int32_t dense_rows;      // rows of the dense group (0: none)
   int32_t* status;
+  // fc1 -> fc2 hand-off per token chunk (null: none).  Chunk ids number the
+  // TILE_N-token chunks of the routed experts in order, then the dense group's.
+  // fc1 adds one per epilogue warp to chunk_done[id] once the warp's h rows of
+  // the tile are stored; fc2 starts without waiting for fc1 as a whole and
+  // loads a chunk's h only after chunk_done[id] reached chunk_target[group]
+  // (fc1 slabs x epilogue warps per tile).
+  int32_t* chunk_done;
+  int32_t chunk_target[2];
 };
 
 constexpr int pow2_at_least(int v) {
@@ -148,6 +156,7 @@ struct GemmCfg {
 struct Tile {
   int grp, e, slab, row0, n_tok, k_begin, k_end, a_row, split;
   int f0;  // first output feature of this CTA's rows within the expert
+  int chunk_id;  // token chunk over both groups (routed chunks, then dense)
 };
 
 // `rank` is the CTA's rank in its pair (0 without pairs): its A rows start
@@ -173,6 +182,7 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
     const int chunk = v - t.slab * nch;
     t.grp = 0;
     t.e = lo;
+    t.chunk_id = prefix[lo] + chunk;
     t.row0 = __ldg(p.offsets + lo) + chunk * TILE_N;
     t.n_tok = min(TILE_N, __ldg(p.counts + lo) - chunk * TILE_N);
     t.f0 = t.slab * C::SLAB_SPAN + rank * C::SLAB_ROWS;
@@ -190,6 +200,7 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
     t.slab = v - chunk * ns;
     t.grp = 1;
     t.e = 0;
+    t.chunk_id = (p.E > 0 ? prefix[p.E] : 0) + chunk;
     t.row0 = chunk * TILE_N;
     t.n_tok = min(TILE_N, p.dense_rows - t.row0);
     t.f0 = t.slab * C::SLAB_SPAN + rank * C::SLAB_ROWS;
@@ -199,6 +210,17 @@ __device__ __forceinline__ Tile decode_tile(int u, const GemmParams& p, const in
     t.k_end = min(G.k_tiles, t.k_begin + kps);
   }
   return t;
+}
+
+// fc1 epilogue warp, after its rows of a tile are stored: count the warp done
+// on the tile's token chunk.  Every lane fences its own stores at GPU scope,
+// the warp barrier orders the fences before lane 0's counter update, so an fc2
+// producer that acquires the full count sees every h row of the chunk.
+__device__ __forceinline__ void signal_chunk(const GemmParams& p, const Tile& t, int lane) {
+  if (p.chunk_done == nullptr) return;
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) atomicAdd(p.chunk_done + t.chunk_id, 1);
 }
 
 // One-CTA or CTA-pair (cta_group::2) forms of the MMA issuer's instructions.
@@ -366,8 +388,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     }
   }
   // everything above touches only this CTA's shared memory and TMEM; from here
-  // on the kernel reads what the previous kernel wrote (token counts, rows)
-  pdl_wait();
+  // on the kernel reads what the previous kernel wrote (token counts, rows).
+  // An fc2 fed chunk by chunk does not wait for fc1 as a whole: the counts it
+  // reads were final before fc1 let it launch, and its producer waits for each
+  // chunk of h (chunk_done) before loading it.
+  if (!(MODE == kFc2 && p.chunk_done != nullptr)) pdl_wait();
   pdl_trigger();
   if (warp == 2) {
     // prefix[e] = number of TILE_N-token chunks of experts < e
@@ -429,6 +454,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         const int kt_all = p.g[t.grp].k_tiles;
         const int tile_base = (t.a_row / kBM) * kt_all;
         const int kb4 = p.kb4[t.grp];
+        if (MODE == kFc2 && p.chunk_done != nullptr) {
+          if (!counter_wait(p.chunk_done + t.chunk_id, p.chunk_target[t.grp], abort_flag,
+                            p.status)) { ok = false; break; }
+          fence_proxy_async_global();
+        }
         for (int kt = t.k_begin; kt < t.k_end; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           const uint32_t fb = cluster_addr(&full[stage], 0);
@@ -505,6 +535,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         const int n_sfa = (MODE == kRouter) ? 1 : (slab1 ? 2 : 1);
         const uint32_t bytes = C::NA * C::A_BYTES + (gather ? n_load : nbox * kBoxRows) * 128 +
                                (DT != kBF16 ? (n_sfa + nsfb) * C::SF_KCH * C::SF_CHUNK : 0);
+        if (MODE == kFc2 && p.chunk_done != nullptr) {  // lane 0 only (no gather in fc2)
+          if (!counter_wait(p.chunk_done + t.chunk_id, p.chunk_target[t.grp], abort_flag,
+                            p.status)) { ok = false; break; }
+          fence_proxy_async_global();
+        }
         for (int kt = t.k_begin; kt < t.k_end; ++kt) {
           // lane 0 waits and sets the expected bytes; the decision is shared so the
           // warp stays converged
@@ -790,6 +825,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
           if (lane == 0 && hmax > 0.f && f_base < G.a_valid_rows)
             atomic_max_nonneg(amax_out, hmax);
         }
+        signal_chunk(p, t, lane);
         if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
       } else if constexpr (MODE == kFc2 || (MODE == kFc1 && DT == kMXF8)) {
         // As above: TMEM -> registers (packed bf16), release the accumulator,
@@ -910,6 +946,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             __syncwarp();
           }
         }
+        if constexpr (MODE == kFc1) signal_chunk(p, t, lane);
         if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
       } else {
       for (int c0 = member * 32; c0 < t.n_tok; c0 += 64) {

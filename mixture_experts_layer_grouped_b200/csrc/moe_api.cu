@@ -29,8 +29,8 @@ inline int64_t pad128(int64_t v) { return (v + 127) / 128 * 128; }
 // ---------------------------------------------------------------------------
 struct StepLayout {
   // h: fc1 output (bf16; MXFP8: e4m3 codes); h_q: NVFP4 codes of h; h_sf: scales
-  size_t status, hist, h, h_q, h_sf, h_shared, h_shared_q, h_shared_sf, g_h, router_partials,
-      total;
+  size_t status, hist, h, h_q, h_sf, h_shared, h_shared_q, h_shared_sf, g_h, chunk_done,
+      router_partials, total;
   int32_t r_cap, ntiles, router_splits;
 };
 
@@ -52,6 +52,25 @@ int router_splits_of(const moe_config& c) {
     if (best_cost < 0 || cost < best_cost) { best = s; best_cost = cost; }
   }
   return best;
+}
+
+// Upper bound on the token chunks of the grouped GEMMs (tiles of at least 64
+// tokens): each expert's ceil(count / TILE_N) summed over experts, plus the
+// dense group's.
+int max_token_chunks(const moe_config& c) {
+  return c.E + (c.T * c.top_k) / 64 + 1 + (c.T + 63) / 64;
+}
+
+// fc2 starts on the SMs fc1 frees and waits per token chunk (bf16, MXFP8;
+// NVFP4 quantizes h between the two).  MOE_FC2_EARLY=0 makes fc2 wait for fc1
+// as a whole instead.
+bool fc2_early(const moe_config& c) {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MOE_FC2_EARLY");
+    v = (e && atoi(e) == 0) ? 0 : 1;
+  }
+  return v == 1 && c.dtype != MOE_NVFP4;
 }
 
 int32_t r_cap_of(const moe_config& c) {
@@ -80,6 +99,7 @@ StepLayout step_layout(const moe_config& c) {
   L.h_shared_q = o; o = align_up(o + (nv ? Tp * Is / 2 : 0));
   L.h_shared_sf = o; o = align_up(o + ((mx || nv) ? Tp * Is / blk : 0));
   L.g_h = o; o = align_up(o + (nv ? (static_cast<size_t>(c.E) + 1) * 4 : 0));
+  L.chunk_done = o; o = align_up(o + static_cast<size_t>(max_token_chunks(c)) * 4);
   L.router_splits = router_splits_of(c);
   L.router_partials = o;
   o = align_up(o + static_cast<size_t>(L.router_splits) * c.T * c.E * 4);
@@ -507,6 +527,9 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
   const int kb4_div = nv ? 64 : 128;          // K elements per scale chunk column
   float* g_h = reinterpret_cast<float*>(wsb + L.g_h);
   if (nv) MOE_CUDA(cudaMemsetAsync(g_h, 0, (static_cast<size_t>(c.E) + 1) * 4, s));
+  const bool early = fc2_early(c);
+  int32_t* chunk_done = reinterpret_cast<int32_t*>(wsb + L.chunk_done);
+  int fc1_slabs[2] = {0, 0};
   const uint64_t H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
   const int max_chunks = c.E + (c.T * c.top_k) / TILE_N + 1;
   const int dense_chunks = (c.T + TILE_N - 1) / TILE_N;
@@ -587,7 +610,13 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     p.E = c.E;
     p.dense_rows = sh ? c.T : 0;
     p.status = status_ptr(ws);
+    if (early) {
+      p.chunk_done = chunk_done;
+      MOE_CUDA(cudaMemsetAsync(chunk_done, 0, static_cast<size_t>(max_token_chunks(c)) * 4, s));
+    }
     const int units = max_chunks * p.g[0].n_slabs + (sh ? dense_chunks * p.g[1].n_slabs : 0);
+    fc1_slabs[0] = p.g[0].n_slabs;
+    fc1_slabs[1] = p.g[1].n_slabs;
     MOE_TRY((launch_gemm<kFc1, TILE_N, DT, PAIR>(p, units, s)));
   }
   // NVFP4: h's per-expert global scales from the amax fc1 gathered, then h codes
@@ -663,6 +692,13 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     p.E = c.E;
     p.dense_rows = sh ? c.T : 0;
     p.status = status_ptr(ws);
+    if (early) {
+      // every epilogue warp of every fc1 tile of the chunk counts once
+      const int warps = kEpiWarps * (PAIR ? 2 : 1);
+      p.chunk_done = chunk_done;
+      p.chunk_target[0] = fc1_slabs[0] * warps;
+      p.chunk_target[1] = fc1_slabs[1] * warps;
+    }
     const int units = max_chunks * slabs + (sh ? dense_chunks * slabs : 0);
     MOE_TRY((launch_gemm<kFc2, TILE_N, DT, PAIR>(p, units, s)));
   }

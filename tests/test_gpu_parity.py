@@ -240,6 +240,27 @@ def test_forward_end_to_end(M, name):
     assert layer.device_status() == 0
 
 
+@pytest.mark.parametrize("name", ["mid_bf16_shared_T2048", "hot_chunks", "tiny_mx",
+                                  "ragged_mx"])
+def test_fc2_early_start_same_bits(M, name, tmp_path):
+    """fc2 started chunk by chunk as fc1 finishes them (the default) gives the
+    same bits as fc2 waiting for fc1 as a whole (MOE_FC2_EARLY=0): only the
+    schedule differs, never the arithmetic."""
+    import os
+    import subprocess
+    import sys
+    helper = os.path.join(os.path.dirname(os.path.abspath(__file__)), "forward_once.py")
+    outs = []
+    for early in ("1", "0"):
+        path = str(tmp_path / f"y_{early}.pt")
+        env = dict(os.environ, MOE_FC2_EARLY=early)
+        r = subprocess.run([sys.executable, helper, name, path], env=env, capture_output=True,
+                           text=True, timeout=600)
+        assert r.returncode == 0, r.stderr[-2000:]
+        outs.append(torch.load(path))
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
 @pytest.mark.slow
 def test_forward_dsv4_bf16_sampled(M):
     """Full-size DeepSeek-V4 geometry in bf16: every token routed on the GPU,
