@@ -523,6 +523,44 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
                : "memory");
 }
 
+// Arrive with release semantics at cluster scope (orders the thread's earlier
+// reads and writes of either CTA's shared memory before the arrival).
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+
+// mbar_wait with acquire semantics at cluster scope: pairs with arrivals made
+// by the peer CTA (mbar_arrive_release_cluster), so the peer's earlier writes
+// to this CTA's shared memory are visible afterwards.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort, int32_t* status,
+                                                  uint64_t limit_ns = 2000000000ull) {
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    if (ok) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      set_status(status, MOE_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// 32-bit store to shared memory given by its cluster address (possibly the peer's).
+__device__ __forceinline__ void st_shared_cluster_s32(uint32_t cluster_addr_, int32_t v) {
+  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(cluster_addr_), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(dst_smem)),

@@ -104,6 +104,9 @@ struct GemmParams {
   // (fc1 slabs x epilogue warps per tile).
   int32_t* chunk_done;
   int32_t chunk_target[2];
+  // dynamic tile order (null: CTA i takes tiles i, i + grid, ...): the next
+  // tile index is claimed from this zeroed counter
+  int32_t* unit_counter;
 };
 
 constexpr int pow2_at_least(int v) {
@@ -131,7 +134,7 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = (NA * A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
   static constexpr int STG_WARP = 32 * 34 * 2;                 // per warp 32 x 34 bf16
   static constexpr int STG_BYTES = kEpiWarps * STG_WARP;
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int BAR_BYTES = 512;  // ring / accumulator barriers, then the tile queue
   // CTA pairs take every byte the epilogue staging, barriers and tile prefix leave
   static constexpr int RING = PAIR ? (232448 - 1024 - STG_BYTES - BAR_BYTES - 4 * (kMaxExperts + 1))
                                    : ((DT == kNVF4) ? 198 * 1024 : kRingBytes);
@@ -221,6 +224,75 @@ __device__ __forceinline__ void signal_chunk(const GemmParams& p, const Tile& t,
   __threadfence();
   __syncwarp();
   if (lane == 0) atomicAdd(p.chunk_done + t.chunk_id, 1);
+}
+
+// The sequence of tiles a CTA (or CTA pair) works on.  Static: first, first +
+// stride, ...  Dynamic (p.unit_counter set): the producer thread (rank 0's in
+// a pair) claims the next tile from the global counter when it is ready to
+// load one and publishes the index through a kSched-slot queue in shared
+// memory (in both CTAs of a pair); the other roles (the MMA thread, the eight
+// epilogue warps, rank 1's producer) read it and release the slot.  CTAs that
+// start late or run short tiles simply claim fewer tiles.  Tiles are claimed
+// in list order, so a claimed fc2 tile's fc1 chunk was claimed before by a
+// running fc1 CTA.
+constexpr int kSched = 4;
+
+struct TileQueue {
+  uint64_t* full;      // [kSched], one arrival (the claimer)
+  uint64_t* empty;     // [kSched], one arrival per consumer of both CTAs
+  volatile int* slot_u;
+  int slot;
+  uint32_t phase;
+  int next_static, stride;
+  bool dynamic;
+};
+
+// Producer of rank 0 (or of a single CTA): the next tile, or `units` at the end.
+template <bool PAIR>
+__device__ __forceinline__ int claim_tile(TileQueue& q, const GemmParams& p, int units,
+                                          volatile int* abort, bool& ok) {
+  if (!q.dynamic) {
+    const int u = q.next_static;
+    q.next_static += q.stride;
+    return u;
+  }
+  const bool free_slot = PAIR ? mbar_wait_cluster(&q.empty[q.slot], q.phase ^ 1, abort, p.status)
+                              : mbar_wait(&q.empty[q.slot], q.phase ^ 1, abort, p.status);
+  if (!free_slot) { ok = false; return units; }
+  int u = atomicAdd(p.unit_counter, 1);
+  if (u > units) u = units;
+  q.slot_u[q.slot] = u;
+  if constexpr (PAIR) {
+    st_shared_cluster_s32(cluster_addr(const_cast<int*>(&q.slot_u[q.slot]), 1), u);
+    mbar_arrive_release_cluster(cluster_addr(&q.full[q.slot], 1));
+  }
+  mbar_arrive(&q.full[q.slot]);
+  if (++q.slot == kSched) { q.slot = 0; q.phase ^= 1; }
+  return u;
+}
+
+// Any other role: the next tile, or `units` at the end (or on a time-out).
+// A warp calls it with all lanes (one release per warp), a thread alone with
+// warp_wide = false.
+template <bool PAIR>
+__device__ __forceinline__ int next_tile(TileQueue& q, const GemmParams& p, int units, int rank,
+                                         bool warp_wide, volatile int* abort) {
+  if (!q.dynamic) {
+    const int u = q.next_static;
+    q.next_static += q.stride;
+    return u;
+  }
+  const bool got = (PAIR && rank == 1)
+                       ? mbar_wait_cluster(&q.full[q.slot], q.phase, abort, p.status)
+                       : mbar_wait(&q.full[q.slot], q.phase, abort, p.status);
+  const int u = got ? q.slot_u[q.slot] : units;
+  if (warp_wide) __syncwarp();
+  if (!warp_wide || lane_id() == 0) {
+    if constexpr (PAIR) mbar_arrive_release_cluster(cluster_addr(&q.empty[q.slot], 0));
+    else mbar_arrive(&q.empty[q.slot]);
+  }
+  if (++q.slot == kSched) { q.slot = 0; q.phase ^= 1; }
+  return u;
 }
 
 // One-CTA or CTA-pair (cta_group::2) forms of the MMA issuer's instructions.
@@ -348,6 +420,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // tile queue in the second half of the barrier area
+  uint64_t* sched_full = reinterpret_cast<uint64_t*>(stg + C::STG_BYTES + 256);
+  uint64_t* sched_empty = sched_full + kSched;
+  volatile int* sched_u = reinterpret_cast<volatile int*>(sched_empty + kSched);
   int* prefix = reinterpret_cast<int*>(stg + C::STG_BYTES + C::BAR_BYTES);
 
   const int warp = warp_id();
@@ -367,6 +443,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       mbar_init(&acc_empty[b], PAIR ? 2 * kEpiWarps : kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < kSched; ++i) {
+      mbar_init(&sched_full[i], 1);
+      // consumers: rank 0's MMA thread and epilogue warps, rank 1's producer
+      // and epilogue warps (one CTA: MMA thread and epilogue warps)
+      mbar_init(&sched_empty[i], PAIR ? 2 * (1 + kEpiWarps) : 1 + kEpiWarps);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -426,6 +508,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
                                     p.g[1].k_splits
                               : 0;
   const int units = units_routed + units_dense;
+  TileQueue tq{sched_full, sched_empty, sched_u, 0, 0u, group_id, n_groups,
+               p.unit_counter != nullptr};
 
   // gathered token rows: the whole producer warp issues the row gathers
   const bool warp_loads = !PAIR && (MODE == kFc1) && p.row_token != nullptr;
@@ -442,7 +526,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = group_id; u < units && ok; u += n_groups) {
+      while (ok) {
+        const int u = (rank == 0) ? claim_tile<PAIR>(tq, p, units, abort_flag, ok)
+                                  : next_tile<PAIR>(tq, p, units, rank, false, abort_flag);
+        if (u >= units) break;
         const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed, rank);
         const int half = ((t.n_tok + 15) & ~15) / 2;  // token rows per CTA (multiple of 8)
         const int nbox = (half + kBoxRows - 1) / kBoxRows;
@@ -509,7 +596,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
 #pragma unroll
       for (int s = 0; s < C::STAGES; ++s) last_phase[s] = -1;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      while (ok) {
+        int u = units;
+        if (lane == 0) u = claim_tile<PAIR>(tq, p, units, abort_flag, ok);
+        if (warp_loads) u = __shfl_sync(0xffffffffu, u, 0);
+        if (u >= units) break;
         const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed);
         const bool gather = (MODE == kFc1) && t.grp == 0 && p.row_token != nullptr;
         // gathered rows: lane l owns tile rows [8l, 8l + 8); rows past the MMA's N
@@ -632,7 +723,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       uint32_t acc_phase = 0;
       bool ok = true;
       constexpr int M_MMA = PAIR ? 2 * kBM : kBM;
-      for (int u = group_id; u < units && ok; u += n_groups) {
+      while (ok) {
+        const int u = next_tile<PAIR>(tq, p, units, 0, false, abort_flag);
+        if (u >= units) break;
         const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed, 0);
         const int n_mma = (t.n_tok + 15) & ~15;
         const uint32_t idesc = idesc_bf16(M_MMA, n_mma);
@@ -733,7 +826,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     uint8_t* my_stg = stg + (warp - 2) * C::STG_WARP;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = group_id; u < units; u += n_groups) {
+    while (true) {
+      const int u = next_tile<PAIR>(tq, p, units, rank, true, abort_flag);
+      if (u >= units) break;
       const Tile t = decode_tile<MODE, TILE_N, DT, PAIR>(u, p, prefix, units_routed, rank);
       // per-tile values in registers, loaded while the MMAs still run: the
       // parameter block is reached through a generic pointer once indexed by

@@ -61,6 +61,17 @@ int max_token_chunks(const moe_config& c) {
   return c.E + (c.T * c.top_k) / 64 + 1 + (c.T + 63) / 64;
 }
 
+// fc1 and fc2 CTAs claim their tiles from a counter (MOE_DYNAMIC_TILES=0:
+// CTA i takes tiles i, i + grid, ...).
+bool dynamic_tiles() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MOE_DYNAMIC_TILES");
+    v = (e && atoi(e) == 0) ? 0 : 1;
+  }
+  return v == 1;
+}
+
 // fc2 starts on the SMs fc1 frees and waits per token chunk (bf16, MXFP8;
 // NVFP4 quantizes h between the two).  MOE_FC2_EARLY=0 makes fc2 wait for fc1
 // as a whole instead.
@@ -99,7 +110,8 @@ StepLayout step_layout(const moe_config& c) {
   L.h_shared_q = o; o = align_up(o + (nv ? Tp * Is / 2 : 0));
   L.h_shared_sf = o; o = align_up(o + ((mx || nv) ? Tp * Is / blk : 0));
   L.g_h = o; o = align_up(o + (nv ? (static_cast<size_t>(c.E) + 1) * 4 : 0));
-  L.chunk_done = o; o = align_up(o + static_cast<size_t>(max_token_chunks(c)) * 4);
+  // two tile-claim counters (fc1, fc2), then the per-chunk counters
+  L.chunk_done = o; o = align_up(o + (2 + static_cast<size_t>(max_token_chunks(c))) * 4);
   L.router_splits = router_splits_of(c);
   L.router_partials = o;
   o = align_up(o + static_cast<size_t>(L.router_splits) * c.T * c.E * 4);
@@ -528,7 +540,12 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
   float* g_h = reinterpret_cast<float*>(wsb + L.g_h);
   if (nv) MOE_CUDA(cudaMemsetAsync(g_h, 0, (static_cast<size_t>(c.E) + 1) * 4, s));
   const bool early = fc2_early(c);
-  int32_t* chunk_done = reinterpret_cast<int32_t*>(wsb + L.chunk_done);
+  const bool dyn = dynamic_tiles();
+  int32_t* unit_counters = reinterpret_cast<int32_t*>(wsb + L.chunk_done);
+  int32_t* chunk_done = unit_counters + 2;
+  if (early || dyn)
+    MOE_CUDA(cudaMemsetAsync(unit_counters, 0, (2 + static_cast<size_t>(max_token_chunks(c))) * 4,
+                             s));
   int fc1_slabs[2] = {0, 0};
   const uint64_t H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
   const int max_chunks = c.E + (c.T * c.top_k) / TILE_N + 1;
@@ -610,10 +627,8 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
     p.E = c.E;
     p.dense_rows = sh ? c.T : 0;
     p.status = status_ptr(ws);
-    if (early) {
-      p.chunk_done = chunk_done;
-      MOE_CUDA(cudaMemsetAsync(chunk_done, 0, static_cast<size_t>(max_token_chunks(c)) * 4, s));
-    }
+    if (early) p.chunk_done = chunk_done;
+    if (dyn) p.unit_counter = unit_counters;
     const int units = max_chunks * p.g[0].n_slabs + (sh ? dense_chunks * p.g[1].n_slabs : 0);
     fc1_slabs[0] = p.g[0].n_slabs;
     fc1_slabs[1] = p.g[1].n_slabs;
@@ -699,6 +714,7 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
       p.chunk_target[0] = fc1_slabs[0] * warps;
       p.chunk_target[1] = fc1_slabs[1] * warps;
     }
+    if (dyn) p.unit_counter = unit_counters + 1;
     const int units = max_chunks * slabs + (sh ? dense_chunks * slabs : 0);
     MOE_TRY((launch_gemm<kFc2, TILE_N, DT, PAIR>(p, units, s)));
   }

@@ -1,7 +1,7 @@
 """Helper for the GPU tests: one forward of a named workload on its seeded
 inputs, output saved with torch.save.  Run as a separate process so that
-launch-time switches read from the environment (MOE_FC2_EARLY, ...) take
-effect:  python tests/forward_once.py <workload> <out.pt>"""
+launch-time switches read from the environment (MOE_FC2_EARLY,
+MOE_DYNAMIC_TILES, ...) take effect:  python tests/forward_once.py <workload> <out.pt>"""
 
 import os
 import sys
@@ -14,6 +14,7 @@ sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 import synth  # noqa: E402
 from moe_testlib import weights_dict  # noqa: E402
 import test_gpu_mxfp8  # noqa: E402
+import test_gpu_nvfp4  # noqa: E402
 import test_gpu_parity  # noqa: E402
 
 
@@ -22,6 +23,8 @@ def shape(name):
         return test_gpu_parity.EDGE[name]
     if name in test_gpu_mxfp8.MX:
         return test_gpu_mxfp8.MX[name]
+    if name in test_gpu_nvfp4.NV:
+        return test_gpu_nvfp4.NV[name]
     return synth.get_config(name)
 
 

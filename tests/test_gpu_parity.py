@@ -241,11 +241,12 @@ def test_forward_end_to_end(M, name):
 
 
 @pytest.mark.parametrize("name", ["mid_bf16_shared_T2048", "hot_chunks", "tiny_mx",
-                                  "ragged_mx"])
-def test_fc2_early_start_same_bits(M, name, tmp_path):
-    """fc2 started chunk by chunk as fc1 finishes them (the default) gives the
-    same bits as fc2 waiting for fc1 as a whole (MOE_FC2_EARLY=0): only the
-    schedule differs, never the arithmetic."""
+                                  "ragged_mx", "tiny_nv"])
+def test_schedules_give_same_bits(M, name, tmp_path):
+    """The default schedule (tiles claimed from a counter, fc2 started chunk by
+    chunk as fc1 finishes them) gives the same bits as the static one (CTA i
+    takes tiles i, i + grid, ...; fc2 waits for fc1 as a whole): only the
+    order of tiles differs, never the arithmetic of one."""
     import os
     import subprocess
     import sys
@@ -253,7 +254,7 @@ def test_fc2_early_start_same_bits(M, name, tmp_path):
     outs = []
     for early in ("1", "0"):
         path = str(tmp_path / f"y_{early}.pt")
-        env = dict(os.environ, MOE_FC2_EARLY=early)
+        env = dict(os.environ, MOE_FC2_EARLY=early, MOE_DYNAMIC_TILES=early)
         r = subprocess.run([sys.executable, helper, name, path], env=env, capture_output=True,
                            text=True, timeout=600)
         assert r.returncode == 0, r.stderr[-2000:]
