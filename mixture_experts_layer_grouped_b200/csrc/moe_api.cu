@@ -430,6 +430,7 @@ moe_status do_route(const moe_config& c, const void* x, const void* w_router, co
   a.g = c.topk_group;
   a.k = c.top_k;
   a.rsf = c.routed_scaling_factor;
+  a.gs_magic = static_cast<uint32_t>(((1ull << 32) + (c.E / c.n_group) - 1) / (c.E / c.n_group));
   const int per = (c.E + 31) / 32;
   const dim3 grid((c.T + kSelWarps - 1) / kSelWarps), block(kSelWarps * 32);
   if (per <= 1) MOE_TRY(launch_pdl(route_select_kernel<1>, dim3(grid), dim3(block), 0, s, a));
@@ -520,11 +521,25 @@ struct MlpQuant {
 
 // PAIR: fc1 and fc2 run as two-CTA clusters (M = 256 MMAs; each CTA holds
 // half of a tile's token rows), which leaves room for a deeper load ring.
+// The grouped MLP's counters (tile claims, fc1 -> fc2 chunks) and NVFP4's
+// per-expert amax of h start every call at zero.  A memset between two kernels
+// breaks their programmatic launch overlap, so the one-call forward issues it
+// first, before the routing kernels, and tells the grouped MLP so.
+moe_status zero_mlp_scratch(const moe_config& c, void* ws, cudaStream_t s) {
+  const StepLayout L = step_layout(c);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  MOE_CUDA(cudaMemsetAsync(wsb + L.chunk_done, 0,
+                           (2 + static_cast<size_t>(max_token_chunks(c))) * 4, s));
+  if (c.dtype == MOE_NVFP4)
+    MOE_CUDA(cudaMemsetAsync(wsb + L.g_h, 0, (static_cast<size_t>(c.E) + 1) * 4, s));
+  return MOE_OK;
+}
+
 template <int TILE_N, int DT, bool PAIR>
 moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const void* rows,
                              const void* x, const MlpQuant& q, const int32_t* counts,
                              const int32_t* offsets, void* out_rows, void* shared_out, void* ws,
-                             cudaStream_t s) {
+                             cudaStream_t s, bool scratch_zeroed) {
   const StepLayout L = step_layout(c);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   void* h = wsb + L.h;
@@ -538,14 +553,11 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
   const int kstep = nv ? 256 : (mx ? 128 : kBK);  // K elements per k-step
   const int kb4_div = nv ? 64 : 128;          // K elements per scale chunk column
   float* g_h = reinterpret_cast<float*>(wsb + L.g_h);
-  if (nv) MOE_CUDA(cudaMemsetAsync(g_h, 0, (static_cast<size_t>(c.E) + 1) * 4, s));
+  if (!scratch_zeroed) MOE_TRY(zero_mlp_scratch(c, ws, s));
   const bool early = fc2_early(c);
   const bool dyn = dynamic_tiles();
   int32_t* unit_counters = reinterpret_cast<int32_t*>(wsb + L.chunk_done);
   int32_t* chunk_done = unit_counters + 2;
-  if (early || dyn)
-    MOE_CUDA(cudaMemsetAsync(unit_counters, 0, (2 + static_cast<size_t>(max_token_chunks(c))) * 4,
-                             s));
   int fc1_slabs[2] = {0, 0};
   const uint64_t H = c.H, I = c.I, Is = c.I_shared, E = c.E, T = c.T;
   const int max_chunks = c.E + (c.T * c.top_k) / TILE_N + 1;
@@ -738,7 +750,7 @@ bool use_pairs(const moe_config& c, const void* rows) {
 moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void* rows,
                           const void* x, const MlpQuant& q, const int32_t* counts,
                           const int32_t* offsets, void* out_rows, void* shared_out, void* ws,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool scratch_zeroed = false) {
   // Decode-sized batches (at most 32 rows per expert on average) take 64-token
   // tiles: a stage holds far fewer token bytes (a fourth stage fits) and two
   // accumulators fit TMEM, so each tile's epilogue overlaps the next tile.
@@ -746,7 +758,7 @@ moe_status do_grouped_mlp(const moe_config& c, const moe_weights& w, const void*
   const bool pairs = !small && use_pairs(c, rows);
 #define MOE_MLP(TN, DT, PR)                                                                      \
   return grouped_mlp_tiles<TN, DT, PR>(c, w, rows, x, q, counts, offsets, out_rows, shared_out, \
-                                       ws, s)
+                                       ws, s, scratch_zeroed)
   if (is_mx(c)) {
     if (small) MOE_MLP(64, kMXF8, false);
     if (pairs) MOE_MLP(192, kMXF8, true);
@@ -1113,6 +1125,7 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   int32_t* token_row = reinterpret_cast<int32_t*>(b + F.token_row);
   void* out_rows = b + F.out_rows;
   void* shared_out = c.I_shared > 0 ? b + F.shared_out : nullptr;
+  MOE_TRY(zero_mlp_scratch(c, workspace, s));
   MOE_TRY(do_route(c, xd, w_router, bias, nullptr, logits, topk_idx, topk_w, workspace, s));
   const void* xq = xd;
   MlpQuant q{nullptr, nullptr, nullptr, nullptr};
@@ -1128,7 +1141,7 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   MOE_TRY(do_permute(c, topk_idx, xq, q.x_scales, counts, offsets, row_token, token_row, rows,
                      b + F.rows_sf, workspace, s));
   MOE_TRY(do_grouped_mlp(c, *w, rows, xq, q, counts, offsets, out_rows, shared_out, workspace,
-                         s));
+                         s, /*scratch_zeroed=*/true));
   MOE_TRY(do_combine(c, out_rows, token_row, topk_w, shared_out, yd, s));
   if (xy_on_host) MOE_CUDA(cudaMemcpyAsync(y, yd, xbytes, cudaMemcpyDeviceToHost, s));
   return MOE_OK;

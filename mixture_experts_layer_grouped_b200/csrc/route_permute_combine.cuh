@@ -32,6 +32,7 @@ struct SelArgs {
   float* topk_w;        // [T, k]
   int T, E, G, g, k;
   float rsf;
+  uint32_t gs_magic;  // ceil(2^32 / (E / G)): e / (E / G) == umulhi(e, gs_magic) for e < 1024
 };
 
 // Warp arg-max of (v, i): larger v wins, ties to the smaller i.
@@ -86,15 +87,31 @@ __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(SelArgs a)
     }
   }
   __syncwarp();
-  // group scores (lane q handles group q)
+  // group scores: lpg = 32 / G lanes per group when G divides 32 (else one),
+  // each scanning a strided share of the group's experts for its two largest
+  // values, merged across the group's lanes by shuffles; group q's score ends
+  // in lane q
+  const int lpg = (32 % a.G == 0) ? 32 / a.G : 1;
   float gscore = -INFINITY;
-  if (lane < a.G) {
+  {
+    const int q = lane / lpg, sub = lane - q * lpg;
     float m1 = -INFINITY, m2 = -INFINITY;
-    for (int e = lane * gs; e < (lane + 1) * gs; ++e) {
-      const float v = sb[w][e];
-      if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
+    if (q < a.G) {
+      for (int e = q * gs + sub; e < (q + 1) * gs; e += lpg) {
+        const float v = sb[w][e];
+        if (v > m1) { m2 = m1; m1 = v; } else if (v > m2) { m2 = v; }
+      }
     }
-    gscore = m1 + m2;
+    for (int o = 1; o < lpg; o <<= 1) {  // top-2 of two top-2 pairs (a multiset)
+      const float o1 = __shfl_xor_sync(0xffffffffu, m1, o);
+      const float o2 = __shfl_xor_sync(0xffffffffu, m2, o);
+      const float hi = fmaxf(m1, o1);
+      m2 = fmaxf(fminf(m1, o1), fmaxf(m2, o2));
+      m1 = hi;
+    }
+    const float s_q = m1 + m2;  // in every lane of group q
+    gscore = __shfl_sync(0xffffffffu, s_q, (lane < a.G ? lane : 0) * lpg);
+    if (lane >= a.G) gscore = -INFINITY;
   }
   // keep the best g groups
   uint32_t keep = 0;
@@ -110,7 +127,8 @@ __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(SelArgs a)
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
-    if (e >= a.E || !((keep >> (e / gs)) & 1u)) b[i] = -INFINITY;
+    if (e >= a.E || !((keep >> __umulhi(static_cast<uint32_t>(e), a.gs_magic)) & 1u))
+      b[i] = -INFINITY;
   }
   float sel_s = 0.f;
   int sel_e = 0;
