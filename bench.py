@@ -228,11 +228,11 @@ TENSOR_RATIO = {"bf16": 1.0, "mxfp8": 2.0, "nvfp4": 4.0}  # nominal dense peak v
 # captured on fewer experts with the same tokens per expert, so the ratio carries
 # over per touched expert).  Valid for the kernels those captures measured.
 TRAFFIC_RATIO = {
-    "mid_bf16_shared_T2048": 1.26,
+    "mid_bf16_shared_T2048": 1.20,
     "dsv4_bf16_T4096": 1.03,
-    "dsv3_mxfp8_shared_T4096": 1.10,
+    "dsv3_mxfp8_shared_T4096": 1.08,
     "dsv4_nvfp4_decode_T128": 1.01,
-    "dsv4_nvfp4_prefill_T8192": 1.08,
+    "dsv4_nvfp4_prefill_T8192": 1.06,
 }
 
 
