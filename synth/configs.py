@@ -1,6 +1,6 @@
 """Workload shapes of the routed MoE layer forward.
 
-The six workloads are the routed-MoE shapes the method is exercised on:
+The workloads are the routed-MoE shapes the method is exercised on:
 
 * a tiny bf16 layer (T=64, H=256, I=128, E=16, groups 4/2, top-4);
 * a mid-size bf16 layer with a shared expert and a skewed router
@@ -12,7 +12,9 @@ The six workloads are the routed-MoE shapes the method is exercised on:
   "DeepSeekV3Layer", Performance section: DeepSeek-V3 dims, top-k 8, MXFP8);
 * the DeepSeek-V4 geometry 7168/3072/top-6/E=384 in NVFP4 W4A4 (sglang PR
   "Mistral Large 3 NVFP4 TRTLLM MoE support", Modifications: W4A4 NVFP4), at a
-  decode size (T=128) and a prefill size (T=8192).
+  decode size (T=128) and a prefill size (T=8192);
+* and for serving, the same geometry at a batch between those (T=1024, NVFP4)
+  and in MXFP8 (T=4096).
 
 ``pad_multiple`` is the row multiple each expert segment is padded to in the
 expert-major layout: 64 for the block-scaled paths (whose scale chunks the
@@ -82,6 +84,16 @@ CONFIGS = {
     "dsv4_nvfp4_prefill_T8192": MoEShape(
         name="dsv4_nvfp4_prefill_T8192", T=8192, H=7168, I=3072, E=384, n_group=8,
         topk_group=4, top_k=6, rsf=2.5, I_shared=0, dtype="nvfp4",
+        pad_multiple=64, router_std=-1.0),
+    # serving sizes of the same geometry: a batch between the decode and
+    # prefill sizes (16 routed rows per expert on average), and the MXFP8 form
+    "dsv4_nvfp4_serve_T1024": MoEShape(
+        name="dsv4_nvfp4_serve_T1024", T=1024, H=7168, I=3072, E=384, n_group=8,
+        topk_group=4, top_k=6, rsf=2.5, I_shared=0, dtype="nvfp4",
+        pad_multiple=64, router_std=-1.0),
+    "dsv4_mxfp8_T4096": MoEShape(
+        name="dsv4_mxfp8_T4096", T=4096, H=7168, I=3072, E=384, n_group=8,
+        topk_group=4, top_k=6, rsf=2.5, I_shared=0, dtype="mxfp8",
         pad_multiple=64, router_std=-1.0),
 }
 

@@ -221,27 +221,32 @@ def test_forward_mxfp8_end_to_end(M, name):
 
 
 @pytest.mark.slow
-def test_forward_dsv3_mxfp8_sampled(M):
-    """DeepSeek-V3 dims in MXFP8 with a shared expert, full size: every token
-    routed and computed on the GPU; the oracle checks a seeded sample of
-    tokens (their experts' weights quantized on the host)."""
-    cfg = synth.get_config("dsv3_mxfp8_shared_T4096")
+@pytest.mark.parametrize("name", ["dsv3_mxfp8_shared_T4096", "dsv4_mxfp8_T4096"])
+def test_forward_mxfp8_sampled(M, name):
+    """Full-size MXFP8 layers (DeepSeek-V3 dims with a shared expert, the
+    DeepSeek-V4 geometry without): every token routed and computed on the GPU;
+    the oracle checks a seeded sample of tokens (their experts' weights
+    quantized on the host)."""
+    cfg = synth.get_config(name)
     c = M.config_from_shape(cfg)
     x = synth.gen_x(cfg, "cuda")
     w_r, bias = synth.gen_router(cfg, "cuda")
     sh = synth.gen_shared_weights(cfg, "cuda")
     sz = M.moe_prepared_weights_size(c)
     u8 = dict(dtype=torch.uint8, device="cuda")
-    p = {k: torch.empty(sz[n], **u8) for k, n in
-         (("w1", "w13"), ("w3", "w13"), ("w2", "w2"), ("w1_scales", "w13_scales"),
-          ("w3_scales", "w13_scales"), ("w2_scales", "w2_scales"), ("ws1", "ws13"),
-          ("ws3", "ws13"), ("ws2", "ws2"), ("ws1_scales", "ws13_scales"),
-          ("ws3_scales", "ws13_scales"), ("ws2_scales", "ws2_scales"))}
+    names = [("w1", "w13"), ("w3", "w13"), ("w2", "w2"), ("w1_scales", "w13_scales"),
+             ("w3_scales", "w13_scales"), ("w2_scales", "w2_scales")]
+    if sh is not None:
+        names += [("ws1", "ws13"), ("ws3", "ws13"), ("ws2", "ws2"),
+                  ("ws1_scales", "ws13_scales"), ("ws3_scales", "ws13_scales"),
+                  ("ws2_scales", "ws2_scales")]
+    p = {k: torch.empty(sz[n], **u8) for k, n in names}
     dst = M.binding.weights_struct(p)
     for e in range(cfg.E):  # one expert at a time: the bf16 layer never exists whole
         a, b, cc = synth.gen_expert_weights(cfg, e, "cuda")
         M.moe_prepare_weights(c, 0, e, 1, a, b, cc, dst)
-    M.moe_prepare_weights(c, 1, 0, 1, sh[0], sh[1], sh[2], dst)
+    if sh is not None:
+        M.moe_prepare_weights(c, 1, 0, 1, sh[0], sh[1], sh[2], dst)
     layer = M.MoELayer(c, p, w_r, bias, prepared=True)
     y = layer.forward(x)
     torch.cuda.synchronize()
@@ -251,8 +256,11 @@ def test_forward_dsv3_mxfp8_sampled(M):
     keep = ~near_ties(r)
     sample = np.random.default_rng(1).choice(np.nonzero(keep)[0], 6, replace=False)
     xq = O.quantize_dequantize(xh[sample], "mxfp8")
-    shh = [f64(t) for t in sh]
-    _, so = O.expert_forward(xq, shh[0], shh[1], shh[2], "mxfp8")
+    if sh is not None:
+        shh = [f64(t) for t in sh]
+        _, so = O.expert_forward(xq, shh[0], shh[1], shh[2], "mxfp8")
+    else:
+        so = np.zeros((len(sample), cfg.H))
     ref = np.zeros((len(sample), cfg.H))
     cache = {}
     for i, t in enumerate(sample):

@@ -205,9 +205,9 @@ def test_forward_nvfp4_end_to_end(M, name):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["dsv4_nvfp4_decode_T128"])
+@pytest.mark.parametrize("name", ["dsv4_nvfp4_decode_T128", "dsv4_nvfp4_serve_T1024"])
 def test_forward_dsv4_nvfp4_sampled(M, name):
-    """DeepSeek-V4 geometry in NVFP4 W4A4 at full size (decode batch): every
+    """DeepSeek-V4 geometry in NVFP4 W4A4 at full size (decode and serving batches): every
     token on the GPU, the oracle on a seeded sample of tokens.  h's global
     scale is per expert, over each touched expert's rows, so the oracle runs
     fc1 on all rows of the sampled tokens' experts."""
