@@ -233,6 +233,8 @@ TRAFFIC_RATIO = {
     "dsv3_mxfp8_shared_T4096": 1.08,
     "dsv4_nvfp4_decode_T128": 1.01,
     "dsv4_nvfp4_prefill_T8192": 1.06,
+    "dsv4_nvfp4_serve_T1024": 1.01,
+    "dsv4_mxfp8_T4096": 1.02,
 }
 
 
