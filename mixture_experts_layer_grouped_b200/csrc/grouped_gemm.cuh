@@ -1044,124 +1044,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         if constexpr (MODE == kFc1) signal_chunk(p, t, lane);
         if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
       } else {
-      for (int c0 = member * 32; c0 < t.n_tok; c0 += 64) {
-        const int rows_here = min(32, t.n_tok - c0);
-        uint32_t r0[32], r1[32];
-        tmem_ld_32x32b_x32(lane_addr + c0, r0);
-        if (C::NA == 2) tmem_ld_32x32b_x32(lane_addr + TILE_N + c0, r1);
-        tmem_ld_wait();
-        if (MODE == kRouter) {
-          // thread = expert, register j = token: 32 consecutive fp32 per token
-          float* out = static_cast<float*>(G.out) + t.split * G.split_stride;
-          const int e = f_base + lane;
+        // router logits, the one mode left: thread = expert, register j = token
+        // (32 consecutive fp32 per token), into the tile's K-split partials
+        static_assert(MODE == kRouter, "fc1 and fc2 release their accumulator early");
+        float* out = static_cast<float*>(G.out) + t.split * G.split_stride;
+        const int e = f_base + lane;
+        for (int c0 = member * 32; c0 < t.n_tok; c0 += 64) {
+          const int rows_here = min(32, t.n_tok - c0);
+          uint32_t r0[32];
+          tmem_ld_32x32b_x32(lane_addr + c0, r0);
+          tmem_ld_wait();
           if (e < G.a_valid_rows) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (j < rows_here)
                 out[static_cast<int64_t>(t.row0 + c0 + j) * G.out_ld + e] = __uint_as_float(r0[j]);
           }
-          continue;
         }
-        if (MODE == kFc1 && DT == kMXF8) {
-          // h = bf16(silu(gate) * up) staged as [32 tokens][32 features] (row stride 34
-          // bf16 to spread banks); then lane j takes token j: the warp's 32 features
-          // are one MXFP8 block, quantized from registers without cross-lane work.
-          constexpr int RS = 34;
-          __nv_bfloat16* hs_ = reinterpret_cast<__nv_bfloat16*>(my_stg);
-          uint16_t* hs16 = reinterpret_cast<uint16_t*>(my_stg);
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const uint32_t w = bf16x2_bits(silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j]),
-                                           silu_f(__uint_as_float(r0[j + 1])) *
-                                               __uint_as_float(r1[j + 1]));
-            hs16[j * RS + lane] = static_cast<uint16_t>(w & 0xFFFFu);
-            hs16[(j + 1) * RS + lane] = static_cast<uint16_t>(w >> 16);
-          }
-          __syncwarp();
-          if (lane < rows_here && f_base < G.a_valid_rows) {
-            float v[32];
-            float amax = 0.f;
-            const __nv_bfloat162* row = reinterpret_cast<const __nv_bfloat162*>(hs_ + lane * RS);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float2 f = __bfloat1622float2(row[i]);
-              v[2 * i] = f.x;
-              v[2 * i + 1] = f.y;
-              amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
-            const uint32_t code = mx_scale_code(amax);
-            const float inv = mx_inv_scale(code);
-            uint32_t w[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              w[i] = static_cast<uint32_t>(to_e4m3(v[4 * i] * inv)) |
-                     (static_cast<uint32_t>(to_e4m3(v[4 * i + 1] * inv)) << 8) |
-                     (static_cast<uint32_t>(to_e4m3(v[4 * i + 2] * inv)) << 16) |
-                     (static_cast<uint32_t>(to_e4m3(v[4 * i + 3] * inv)) << 24);
-            const int64_t r = t.row0 + c0 + lane;
-            uint4* dst = reinterpret_cast<uint4*>(q_out + r * G.out_ld + f_base);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            q_sf[sf_offset(r, f_base / 32, static_cast<int>(G.out_ld) / 32)] =
-                static_cast<uint8_t>(code);
-          }
-          __syncwarp();
-          continue;
-        }
-        // bf16 outputs: stage [32 tokens][32 features] per warp, then 16-byte stores
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(G.out);
-        const uint4* s4 = reinterpret_cast<const uint4*>(my_stg);
-        __nv_bfloat16* s = reinterpret_cast<__nv_bfloat16*>(my_stg);
-        const int n_halves = (MODE == kFc2) ? 2 : 1;
-#pragma unroll
-        for (int half = 0; half < n_halves; ++half) {
-          const int f0 = f_base + half * kBM;
-          if (MODE == kFc1) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const __nv_bfloat16 hb = __float2bfloat16_rn(
-                  silu_f(__uint_as_float(r0[j]) * alpha) * (__uint_as_float(r1[j]) * alpha));
-              s[j * 32 + lane] = hb;
-              if (DT == kNVF4 && j < rows_here) hmax = fmaxf(hmax, fabsf(__bfloat162float(hb)));
-            }
-          } else {
-            uint16_t* s16 = reinterpret_cast<uint16_t*>(my_stg);
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const uint32_t w = bf16x2_bits(__uint_as_float(half ? r1[j] : r0[j]) * alpha,
-                                             __uint_as_float(half ? r1[j + 1] : r0[j + 1]) * alpha);
-              s16[j * 32 + lane] = static_cast<uint16_t>(w & 0xFFFFu);
-              s16[(j + 1) * 32 + lane] = static_cast<uint16_t>(w >> 16);
-            }
-          }
-          __syncwarp();
-#pragma unroll
-          for (int it = 0; it < 4; ++it) {
-            const int c = it * 32 + lane;
-            const int j = c >> 2, part = c & 3;
-            if (j < rows_here && f0 < G.a_valid_rows) {
-              const uint4 v = s4[j * 4 + part];
-              *reinterpret_cast<uint4*>(out + static_cast<int64_t>(t.row0 + c0 + j) * G.out_ld +
-                                        f0 + part * 8) = v;
-            }
-          }
-          __syncwarp();
-        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (PAIR) mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));  // rank 0's barrier
-        else mbar_arrive(&acc_empty[acc]);
-      }
-      if (MODE == kFc1 && DT == kNVF4) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
-        if (lane == 0 && hmax > 0.f && f_base < G.a_valid_rows)
-          atomic_max_nonneg(amax_out, hmax);
-      }
-      if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
-      }  // generic epilogue
     }
   }
 
