@@ -72,6 +72,15 @@ bool dynamic_tiles() {
   return v == 1;
 }
 
+// Failure-path test hook: MOE_TEST_FC2_NEVER_READY=1 (read on every call)
+// raises fc2's chunk targets by one, a count fc1 never reaches, so every fc2
+// producer's bounded wait runs out, the kernel records MOE_ERR_TIMEOUT and
+// exits in order.  Nothing sets it outside that test.
+bool test_fc2_never_ready() {
+  const char* e = getenv("MOE_TEST_FC2_NEVER_READY");
+  return e && atoi(e) == 1;
+}
+
 // fc2 starts on the SMs fc1 frees and waits per token chunk (bf16, MXFP8;
 // NVFP4 quantizes h between the two).  MOE_FC2_EARLY=0 makes fc2 wait for fc1
 // as a whole instead.
@@ -723,8 +732,9 @@ moe_status grouped_mlp_tiles(const moe_config& c, const moe_weights& w, const vo
       // every epilogue warp of every fc1 tile of the chunk counts once
       const int warps = kEpiWarps * (PAIR ? 2 : 1);
       p.chunk_done = chunk_done;
-      p.chunk_target[0] = fc1_slabs[0] * warps;
-      p.chunk_target[1] = fc1_slabs[1] * warps;
+      const int never = test_fc2_never_ready() ? 1 : 0;
+      p.chunk_target[0] = fc1_slabs[0] * warps + never;
+      p.chunk_target[1] = fc1_slabs[1] * warps + never;
     }
     if (dyn) p.unit_counter = unit_counters + 1;
     const int units = max_chunks * slabs + (sh ? dense_chunks * slabs : 0);

@@ -262,6 +262,24 @@ def test_schedules_give_same_bits(M, name, tmp_path):
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
 
 
+@pytest.mark.parametrize("name", ["tiny_bf16_T64", "mid_bf16_shared_T2048"])
+def test_bounded_wait_times_out_and_recovers(M, name):
+    """A wait that nothing satisfies (fc2's chunk counts raised past what fc1
+    produces, for one call) ends in order: the status word reads
+    MOE_ERR_TIMEOUT, the context stays usable, and the next call gives the
+    same bits as before.  One-CTA tiles (tiny) and CTA pairs (mid)."""
+    import os
+    import subprocess
+    import sys
+    helper = os.path.join(os.path.dirname(os.path.abspath(__file__)), "timeout_once.py")
+    r = subprocess.run([sys.executable, helper, name], capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = [l for l in r.stdout.splitlines() if l.startswith("status")][-1].split()
+    s0, s1, s2, same = int(line[1]), int(line[2]), int(line[3]), int(line[5])
+    assert (s0, s1, s2, same) == (0, 5, 0, 1), line  # 5 = MOE_ERR_TIMEOUT
+
+
 @pytest.mark.slow
 def test_forward_dsv4_bf16_sampled(M):
     """Full-size DeepSeek-V4 geometry in bf16: every token routed on the GPU,
