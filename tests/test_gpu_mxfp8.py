@@ -254,7 +254,10 @@ def test_forward_mxfp8_sampled(M, name):
     xh, wrh, bh = f64(x), f64(w_r), f64(bias)
     r = O.route(O.router_logits(xh, wrh), bh, cfg.n_group, cfg.topk_group, cfg.top_k, cfg.rsf)
     keep = ~near_ties(r)
-    sample = np.random.default_rng(1).choice(np.nonzero(keep)[0], 6, replace=False)
+    # the oracle quantizes each sampled token's experts on the host (seconds
+    # per DeepSeek-V4-size expert): fewer tokens for the 384-expert layer
+    n_sample = 6 if cfg.E <= 256 else 3
+    sample = np.random.default_rng(1).choice(np.nonzero(keep)[0], n_sample, replace=False)
     xq = O.quantize_dequantize(xh[sample], "mxfp8")
     if sh is not None:
         shh = [f64(t) for t in sh]
