@@ -23,7 +23,12 @@
 // accumulators (tcgen05.ld; two warps per TMEM lane quarter, alternating
 // 32-column chunks) and write the outputs.  When the accumulators of
 // one tile use at most half of TMEM they are double-buffered, so the epilogue
-// of tile i overlaps the MMAs of tile i+1.
+// of tile i overlaps the MMAs of tile i+1; otherwise fc1 and fc2 read their
+// accumulators into registers and release them before storing.
+//
+// Tiles are claimed at run time from a counter (or taken statically), and fc2
+// may start before fc1 ends: its producer waits, per token chunk, for fc1's
+// epilogue warps to have stored that chunk of h (see GemmParams::chunk_done).
 //
 // CTA pairs (PAIR): clusters of two CTAs run one tile together with M = 256
 // MMAs (cta_group::2) issued by rank 0.  Each CTA holds its own 128 weight rows
