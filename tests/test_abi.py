@@ -103,6 +103,21 @@ def test_calls_reject_null_and_small_workspace(M):
                            None) == 3
 
 
+@pytest.mark.parametrize("name", sorted(synth.CONFIGS))
+def test_every_workload_passes_validation(M, name):
+    """Each workload the bench and the tests use is a shape the library accepts,
+    with a workspace and prepared weights of the expected sizes."""
+    s = synth.get_config(name)
+    c = M.config_from_shape(s)
+    nbytes, r_cap = M.moe_workspace_size(c)
+    assert r_cap == s.r_cap and nbytes > 0
+    assert M.moe_forward_workspace_size(c) > nbytes
+    sizes = M.moe_prepared_weights_size(c)
+    per = {"bf16": 2.0, "mxfp8": 1.0, "nvfp4": 0.5}[s.dtype]
+    assert sizes["w13"] == int(s.E * s.I * s.H * per)
+    assert sizes["w2"] == int(s.E * s.H * s.I * per)
+
+
 def test_block_scaled_needs_64_row_padding(M):
     s = synth.get_config("dsv3_mxfp8_shared_T4096").scaled(pad_multiple=32)
     c = M.config_from_shape(s)
