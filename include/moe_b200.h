@@ -108,6 +108,10 @@ const char* moe_status_string(moe_status s);
  * `workspace`; *r_cap = rows of the expert-major buffers (row_token, the
  * permuted rows, the grouped-GEMM outputs): T*top_k + E*(pad_multiple-1)
  * rounded up to pad_multiple.  Either output pointer may be NULL.
+ * A workspace holds per-call state (h, the grouped MLP's tile and chunk
+ * counters, the status word): calls whose kernels may overlap on the GPU
+ * (different streams) need workspaces of their own; calls in one stream may
+ * share one.  Its contents need no initialisation.
  */
 moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes, int32_t* r_cap);
 
