@@ -111,7 +111,8 @@ const char* moe_status_string(moe_status s);
  * A workspace holds per-call state (h, the grouped MLP's tile and chunk
  * counters, the status word): calls whose kernels may overlap on the GPU
  * (different streams) need workspaces of their own; calls in one stream may
- * share one.  Its contents need no initialisation.
+ * share one.  Only its first 4 bytes, the status word, must be zero before
+ * the first call (a call never clears it; moe_get_device_status does).
  */
 moe_status moe_workspace_size(const moe_config* cfg, size_t* bytes, int32_t* r_cap);
 
