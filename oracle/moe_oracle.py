@@ -25,10 +25,15 @@ output rows and of y; the quantized codes of x, of the weights and of h.
 Where the pages leave a step open, the reading taken is stated at the function.
 
 Parity status: every function here is pinned by the CPU tests (brute force on
-tiny inputs, closed forms, library cross-checks, invariants).  Quantization
-noise itself has no external truth to pin against; only the code-level rules
-(round-to-nearest-even, saturation, scale selection) are pinned.
+tiny inputs, closed forms, library cross-checks, invariants, and a hand-worked
+NVFP4 and MXFP8 expert that pins the quantized composition stage by stage).
+Quantization noise itself has no external truth to pin against; only the
+code-level rules (round-to-nearest-even, saturation, scale selection and the
+scope of each global scale) are pinned.
 """
+
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -337,17 +342,39 @@ def nvfp4_dequantize(codes, sb, g):
     return (vals * decode_e4m3(sb)[:, :, None] / np.float64(_F32(g))).reshape(R, K)
 
 
+ROW_BLOCK = 128
+
+
+def by_row_blocks(fn, v, rows=ROW_BLOCK):
+    """fn applied to consecutive blocks of `rows` rows of v, results stacked.
+
+    Every quantizer here is row-local once its global scale is fixed (its
+    blocks of 16 or 32 elements run along a row), so applying it block by
+    block gives exactly the result of one call on the whole matrix.  The blocks
+    run on a thread pool (numpy releases the interpreter lock inside its array
+    operations); that only keeps full-size layers within minutes on the host.
+    """
+    v = np.asarray(v, np.float64)
+    if v.shape[0] <= rows:
+        return fn(v)
+    parts = [v[i:i + rows] for i in range(0, v.shape[0], rows)]
+    with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        return np.concatenate(list(ex.map(fn, parts)), axis=0)
+
+
 def quantize_dequantize(v, dtype, g=None):
-    """The values a quantized tensor stands for, as the MMA consumes them."""
+    """The values a quantized tensor stands for, as the MMA consumes them.
+
+    NVFP4: ``g`` is the tensor's global encode scale; when None it is set from
+    the amax of ``v`` itself (``v`` is then the whole tensor)."""
     if dtype == "bf16":
         return np.asarray(v, np.float64)
     if dtype == "mxfp8":
-        return mxfp8_dequantize(*mxfp8_quantize(v))
+        return by_row_blocks(lambda b: mxfp8_dequantize(*mxfp8_quantize(b)), v)
     if dtype == "nvfp4":
         if g is None:
             g = nvfp4_global_scale(np.abs(np.asarray(v, np.float64)).max())
-        c, s = nvfp4_quantize(v, g)
-        return nvfp4_dequantize(c, s, g)
+        return by_row_blocks(lambda b: nvfp4_dequantize(*nvfp4_quantize(b, g), g), v)
     raise ValueError(dtype)
 
 
@@ -400,27 +427,29 @@ def combine(out_rows, token_row, w, shared_out=None):
 # The whole layer
 # ---------------------------------------------------------------------------
 
-def quantize_weights(W13_or_W2, dtype):
-    """Per-expert weight tensor -> dequantized values (NVFP4: own global scale)."""
-    return quantize_dequantize(W13_or_W2, dtype)
+def prepare_expert_weights(W1, W3, W2, dtype):
+    """An expert's weights as its GEMMs consume them: the bf16 values for
+    bf16; for MXFP8 / NVFP4 the dequantized values of their codes.  W1 and W3
+    are quantized as one stacked fc1 tensor (NVFP4: one global scale for both,
+    from their joint amax), W2 on its own (its own global scale)."""
+    if dtype == "bf16":
+        return (np.asarray(W1, np.float64), np.asarray(W3, np.float64),
+                np.asarray(W2, np.float64))
+    I = W1.shape[0]
+    w13 = quantize_dequantize(np.concatenate([W1, W3], axis=0), dtype)
+    return w13[:I], w13[I:], quantize_dequantize(W2, dtype)
 
 
-def expert_forward(X_deq, W1, W3, W2, dtype, h_global=None):
+def expert_forward(X_deq, W1, W3, W2, dtype, h_global=None, prepared=False):
     """One expert on its rows: dequantized x rows in, bf16 fc2 rows out.
 
-    W1/W3/W2 are the bf16 weight values.  For MXFP8/NVFP4 the weights are
-    quantized here (W1 and W3 share one NVFP4 global scale, as one stacked
-    fc1 tensor), h is rounded to bf16 and then quantized (its NVFP4 global
-    scale is the amax over this expert's rows, the fc2 input of this group of
-    the grouped GEMM, unless ``h_global`` is given).
+    W1/W3/W2 are the bf16 weight values, or (``prepared=True``) the output of
+    prepare_expert_weights.  For MXFP8/NVFP4, h is rounded to bf16 and then
+    quantized; its NVFP4 global scale is set from the amax over this expert's
+    rows (each expert's fc2 input is its own tensor of the grouped GEMM),
+    unless ``h_global`` is given.
     """
-    if dtype == "bf16":
-        w1, w3, w2 = W1, W3, W2
-    else:
-        I = W1.shape[0]
-        w13 = quantize_dequantize(np.concatenate([W1, W3], axis=0), dtype)
-        w1, w3 = w13[:I], w13[I:]
-        w2 = quantize_dequantize(W2, dtype)
+    w1, w3, w2 = (W1, W3, W2) if prepared else prepare_expert_weights(W1, W3, W2, dtype)
     h = expert_fc1(X_deq, w1, w3)
     if dtype == "nvfp4":
         g = nvfp4_global_scale(np.abs(h).max()) if h_global is None else h_global
