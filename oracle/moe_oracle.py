@@ -19,6 +19,11 @@ Sources (page title, then the passage):
   NVFP4 (e2m1 elements, e4m3 scale per 16 along K, fp32 per-tensor global
   scale from amax).
 
+quant_rows.c restates the two row quantizers in plain C (loaded through
+native.py when gcc is available; the CPU tests check it against the numpy
+functions here bit for bit), only so that full-size experts take well under a
+second.
+
 Arithmetic is fp64 on the values each stored tensor holds.  The storage
 roundings that the layer defines are reproduced: bf16 storage of h, of the fc2
 output rows and of y; the quantized codes of x, of the weights and of h.
@@ -362,18 +367,45 @@ def by_row_blocks(fn, v, rows=ROW_BLOCK):
         return np.concatenate(list(ex.map(fn, parts)), axis=0)
 
 
-def quantize_dequantize(v, dtype, g=None):
+def _qdq_native(v, dtype, g):
+    """The same quantize-dequantize through the C restatement in quant_rows.c
+    (checked bit for bit against the numpy functions above), or None."""
+    from . import native
+    L = native.load()
+    if L is None:
+        return None
+    import ctypes
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    if v.ndim != 2:
+        return None
+    out = np.empty_like(v)
+    dp = ctypes.POINTER(ctypes.c_double)
+    if dtype == "mxfp8":
+        L.oracle_mxfp8_qdq_rows(v.ctypes.data_as(dp), out.ctypes.data_as(dp), v.shape[0],
+                                v.shape[1])
+    else:
+        L.oracle_nvfp4_qdq_rows(v.ctypes.data_as(dp), out.ctypes.data_as(dp), v.shape[0],
+                                v.shape[1], float(g))
+    return out
+
+
+def quantize_dequantize(v, dtype, g=None, native=True):
     """The values a quantized tensor stands for, as the MMA consumes them.
 
     NVFP4: ``g`` is the tensor's global encode scale; when None it is set from
-    the amax of ``v`` itself (``v`` is then the whole tensor)."""
+    the amax of ``v`` itself (``v`` is then the whole tensor).  ``native``
+    allows the C restatement of the row quantizers (same results)."""
     if dtype == "bf16":
         return np.asarray(v, np.float64)
+    if dtype == "nvfp4" and g is None:
+        g = nvfp4_global_scale(np.abs(np.asarray(v, np.float64)).max())
+    if native and dtype in ("mxfp8", "nvfp4"):
+        out = _qdq_native(v, dtype, g)
+        if out is not None:
+            return out
     if dtype == "mxfp8":
         return by_row_blocks(lambda b: mxfp8_dequantize(*mxfp8_quantize(b)), v)
     if dtype == "nvfp4":
-        if g is None:
-            g = nvfp4_global_scale(np.abs(np.asarray(v, np.float64)).max())
         return by_row_blocks(lambda b: nvfp4_dequantize(*nvfp4_quantize(b, g), g), v)
     raise ValueError(dtype)
 
