@@ -27,5 +27,6 @@ from .binding import (  # noqa: F401
     moe_quantize,
     scale_bytes,
     prepare_weights,
+    allocate_prepared_weights,
     MoELayer,
 )

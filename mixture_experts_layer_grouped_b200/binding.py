@@ -217,13 +217,12 @@ def moe_prepare_weights(cfg, which, e_begin, e_count, w1, w3, w2, dst, stream=No
         _p(_cuda(w3, bf, "w3")), _p(_cuda(w2, bf, "w2")), ctypes.byref(ws), _stream(stream)))
 
 
-def prepare_weights(cfg, raw: dict, stream=None) -> dict:
-    """Allocate the prepared weight buffers (torch) and fill them from the
-    row-major bf16 tensors in ``raw`` (keys w1, w3, w2 and, with a shared
-    expert, ws1, ws3, ws2)."""
-    dev = raw["w1"].device
+def allocate_prepared_weights(cfg, device="cuda") -> dict:
+    """Empty device buffers for the prepared weights of a layer (sizes from
+    moe_prepared_weights_size), keyed by the moe_weights field names; fill
+    them with moe_prepare_weights, all experts at once or a range at a time."""
     sz = moe_prepared_weights_size(cfg)
-    u8 = dict(dtype=torch.uint8, device=dev)
+    u8 = dict(dtype=torch.uint8, device=device)
     out = {"w1": torch.empty(sz["w13"], **u8), "w3": torch.empty(sz["w13"], **u8),
            "w2": torch.empty(sz["w2"], **u8)}
     if sz["w13_scales"]:
@@ -239,11 +238,19 @@ def prepare_weights(cfg, raw: dict, stream=None) -> dict:
             out["ws3_scales"] = torch.empty(sz["ws13_scales"], **u8)
             out["ws2_scales"] = torch.empty(sz["ws2_scales"], **u8)
         if sz["ws_globals"]:
-            out["ws13_global"] = torch.empty(1, dtype=torch.float32, device=dev)
-            out["ws2_global"] = torch.empty(1, dtype=torch.float32, device=dev)
+            out["ws13_global"] = torch.empty(1, dtype=torch.float32, device=device)
+            out["ws2_global"] = torch.empty(1, dtype=torch.float32, device=device)
     if sz["w_globals"]:
-        out["w13_global"] = torch.empty(cfg.E, dtype=torch.float32, device=dev)
-        out["w2_global"] = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+        out["w13_global"] = torch.empty(cfg.E, dtype=torch.float32, device=device)
+        out["w2_global"] = torch.empty(cfg.E, dtype=torch.float32, device=device)
+    return out
+
+
+def prepare_weights(cfg, raw: dict, stream=None) -> dict:
+    """Allocate the prepared weight buffers (torch) and fill them from the
+    row-major bf16 tensors in ``raw`` (keys w1, w3, w2 and, with a shared
+    expert, ws1, ws3, ws2)."""
+    out = allocate_prepared_weights(cfg, raw["w1"].device)
     dst = weights_struct(out)
     moe_prepare_weights(cfg, 0, 0, cfg.E, raw["w1"], raw["w3"], raw["w2"], dst, stream)
     if cfg.I_shared > 0:

@@ -89,9 +89,8 @@ def test_route_selection_from_identical_logits(M, name):
 
 @pytest.mark.parametrize("name", ALL_CONFIGS)
 def test_router_gemm(M, name):
+    """Every workload at its full T (the 8192-token prefill splits K three ways)."""
     cfg = _cfg(name)
-    if cfg.T > 4096:
-        cfg = cfg.scaled(T=4096)
     c = M.config_from_shape(cfg)
     x = synth.gen_x(cfg, "cuda")
     w_r, bias = synth.gen_router(cfg, "cuda")
@@ -241,7 +240,7 @@ def test_forward_end_to_end(M, name):
 
 
 @pytest.mark.parametrize("name", ["mid_bf16_shared_T2048", "hot_chunks", "tiny_mx",
-                                  "ragged_mx", "tiny_nv"])
+                                  "ragged_mx", "tiny_nv", "hot_nv"])
 def test_schedules_give_same_bits(M, name, tmp_path):
     """The default schedule (tiles claimed from a counter, fc2 started chunk by
     chunk as fc1 finishes them) gives the same bits as the static one (CTA i
@@ -278,37 +277,6 @@ def test_bounded_wait_times_out_and_recovers(M, name):
     line = [l for l in r.stdout.splitlines() if l.startswith("status")][-1].split()
     s0, s1, s2, same = int(line[1]), int(line[2]), int(line[3]), int(line[5])
     assert (s0, s1, s2, same) == (0, 5, 0, 1), line  # 5 = MOE_ERR_TIMEOUT
-
-
-@pytest.mark.slow
-def test_forward_dsv4_bf16_sampled(M):
-    """Full-size DeepSeek-V4 geometry in bf16: every token routed on the GPU,
-    the oracle's expert math on a seeded sample of tokens."""
-    cfg = synth.get_config("dsv4_bf16_T4096")
-    d = gen_device_inputs(cfg)
-    out = run_steps(cfg, d)
-    assert out["status"] == 0
-    x, wr, bias = f64(d["x"]), f64(d["w_router"]), f64(d["bias"])
-    logits = O.router_logits(x, wr)
-    r = O.route(logits, bias, cfg.n_group, cfg.topk_group, cfg.top_k, cfg.rsf)
-    keep, bad = check_routing(r, out["topk_idx"].cpu().numpy(), out["topk_w"].cpu().numpy(),
-                              cfg.rsf)
-    assert not bad
-    rng = np.random.default_rng(0)
-    sample = rng.choice(np.nonzero(keep)[0], 12, replace=False)
-    y = f64(out["y"])
-    ref = np.zeros((len(sample), cfg.H))
-    cache = {}
-    for i, t in enumerate(sample):
-        acc = np.zeros(cfg.H)
-        for j in range(cfg.top_k):
-            e = int(r["idx"][t, j])
-            if e not in cache:
-                cache[e] = tuple(f64(d[k][e]) for k in ("w1", "w3", "w2"))
-            _, o = O.expert_forward(x[t:t + 1], *cache[e], "bf16")
-            acc += r["w"][t, j] * o[0]
-        ref[i] = O.round_bf16(acc)
-    assert rel_frob(y[sample], ref) < 1e-2
 
 
 def test_device_status_reports_bad_index(M):
