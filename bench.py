@@ -1,9 +1,11 @@
 """Throughput of the routed MoE layer forward on B200.
 
 One step = one whole forward of the layer (router GEMM + grouped top-k,
-permute, grouped fc1+SwiGLU / fc2, combine) over one batch of T synthetic
-tokens of the mid-size bf16 workload (T=2048, H=2048, I=1024, E=64, groups
-8/4, top-6, shared expert I=1024), weights resident in HBM.
+quantize, permute, grouped fc1+SwiGLU / fc2, combine) over one batch of T
+synthetic tokens, weights resident in HBM.  The default workload is the
+largest single-GPU one: the DeepSeek-V4 routed-expert geometry in NVFP4 W4A4
+at prefill size (T=8192, H=7168, I=3072, E=384, groups 8/4, top-6); --config
+picks another.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -11,8 +13,8 @@ With N > 1 (torchrun) every rank runs an independent replica on its own batch
 (tokens are independent, so the layer shards by batch with no exchange): weak
 scaling, whole-job tokens/s = N*T*K / max-over-ranks time.
 
---impl reference times the CPU oracle (fp64 numpy) on a bounded token sample
-of the same workload, on rank 0 only.
+--impl reference times the CPU oracle (fp64) on a bounded token sample of the
+same workload, on rank 0 only.
 """
 
 import argparse
@@ -155,61 +157,89 @@ def job_tokens_per_s(tokens_per_rank, n_ranks, ms_max):
 # reference arm: the CPU oracle
 # ---------------------------------------------------------------------------
 
-def _oracle_inputs(cfg, T):
-    from oracle import moe_oracle as O
-    x = O.from_bf16(synth.gen_x(cfg, "cpu", T=T))
-    wr, bias = synth.gen_router(cfg, "cpu")
-    w1 = np.empty((cfg.E, cfg.I, cfg.H))
-    w3 = np.empty_like(w1)
-    w2 = np.empty((cfg.E, cfg.H, cfg.I))
-    for e in range(cfg.E):
-        a, b, c = synth.gen_expert_weights(cfg, e, "cpu")
-        w1[e], w3[e], w2[e] = O.from_bf16(a), O.from_bf16(b), O.from_bf16(c)
-    sh = synth.gen_shared_weights(cfg, "cpu")
-    sh = tuple(O.from_bf16(t) for t in sh) if sh is not None else None
-    return x, O.from_bf16(wr), bias.numpy().astype(np.float64), w1, w3, w2, sh
-
-
-def _blas_threads():
+def _host_cores():
+    """Threads the oracle uses: numpy's BLAS pool and the OpenMP pool of its C
+    row quantizers, each as wide as the host."""
+    n = os.cpu_count() or 1
     try:
         from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
+        b = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max([n] + b)
     except Exception:
-        return os.cpu_count() or 1
+        return n
 
 
-def time_oracle(cfg, sample_tokens, steps, warmup):
-    """Oracle forward on a token sample; returns (tokens/s, seconds per step)."""
+def oracle_tokens(cfg, seconds, device):
+    """Tokens in the oracle's sample so that one pass takes about `seconds` on
+    the host: a one-token pass is timed first (its time goes mostly into
+    preparing the weights of the experts the token touches, so a pass grows
+    about linearly with the tokens until every expert is touched)."""
+    _, t1, _ = time_oracle(cfg, 1, 1, 0, device)
+    n = int(seconds / max(t1, 1e-6))
+    if n >= 2 * cfg.E // max(1, cfg.top_k):   # every expert touched: only the GEMMs grow
+        n = 128
+    return max(1, min(128, cfg.T, n))
+
+
+def oracle_sample(cfg, n_tokens, device):
+    """The oracle's inputs: the first n_tokens tokens of the workload's batch
+    (the GPU arm's draws), the router, and host copies of the bf16 weights of
+    exactly the experts those tokens are routed to."""
     from oracle import moe_oracle as O
-    x, wr, bias, w1, w3, w2, sh = _oracle_inputs(cfg, sample_tokens)
-    scfg = cfg.scaled(T=sample_tokens)
+    xh = O.from_bf16(synth.gen_x(cfg, device)[:n_tokens])
+    wr, bias = synth.gen_router(cfg, device)
+    wrh, bh = O.from_bf16(wr), bias.cpu().numpy().astype(np.float64)
+    r = O.route(O.router_logits(xh, wrh), bh, cfg.n_group, cfg.topk_group, cfg.top_k, cfg.rsf)
+    experts = sorted(set(r["idx"].ravel().tolist()))
+    W = {e: tuple(t.cpu() for t in synth.gen_expert_weights(cfg, e, device)) for e in experts}
+    sh = synth.gen_shared_weights(cfg, device)
+    sh = tuple(O.from_bf16(t) for t in sh) if sh is not None else None
+    return xh, wrh, bh, W, sh
+
+
+def time_oracle(cfg, n_tokens, steps, warmup, device):
+    """The oracle's forward (as it stands: weights quantized inside, fp64
+    arithmetic) on an n_tokens sample; returns (tokens/s, seconds per pass,
+    experts touched)."""
+    from oracle import moe_oracle as O
+    xh, wrh, bh, W, sh = oracle_sample(cfg, n_tokens, device)
+    scfg = cfg.scaled(T=n_tokens)
+    w = [(lambda e, k=k: O.from_bf16(W[e][k])) for k in range(3)]
+
+    def one():
+        O.forward(scfg, xh, wrh, bh, w[0], w[1], w[2], shared=sh)
+
     for _ in range(warmup):
-        O.forward(scfg, x, wr, bias, w1, w3, w2, shared=sh)
+        one()
     t0 = time.perf_counter()
     for _ in range(steps):
-        O.forward(scfg, x, wr, bias, w1, w3, w2, shared=sh)
+        one()
     dt = (time.perf_counter() - t0) / max(steps, 1)
-    return sample_tokens / dt, dt
+    return n_tokens / dt, dt, len(W)
+
+
+def _oracle_note(cfg, n_tokens, n_experts):
+    return (f"oracle forward (fp64; weights of the {n_experts} experts the sample touches "
+            f"quantized inside each pass, as the oracle stands) on the first {n_tokens} tokens of "
+            f"the {cfg.name} batch, per pass")
 
 
 def run_reference(args, cfg):
     ws, rank, _ = _dist()
     if rank != 0:
         return
-    tokens = args.ref_tokens
-    tps, dt = time_oracle(cfg, tokens, args.steps, args.warmup)
-    cores = _blas_threads()
-    sample = (f"oracle forward (fp64 numpy) on a {tokens}-token sample of the workload "
-              f"(all {cfg.E} experts' weights), per step")
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    # the whole --steps K --warmup W run stays within a few minutes
+    n = args.ref_tokens or oracle_tokens(cfg, 150.0 / max(1, args.steps + args.warmup), dev)
+    tps, dt, ne = time_oracle(cfg, n, args.steps, args.warmup, dev)
     line = {
         "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": _workload(cfg, "host oracle; no GPU"),
-        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "config": _workload(cfg, "host oracle; no GPU kernels"),
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": _host_cores(), "kind": "oracle",
+                         "sample": _oracle_note(cfg, n, ne)},
         "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -222,20 +252,46 @@ def run_reference(args, cfg):
 
 WEIGHT_BYTES = {"bf16": 2.0, "mxfp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}  # per element
 TENSOR_RATIO = {"bf16": 1.0, "mxfp8": 2.0, "nvfp4": 4.0}  # nominal dense peak vs bf16
-# DRAM bytes (read + written) of one grouped-MLP call's fc1 and fc2 kernels per
-# algorithmic weight byte, from the ncu counters summarised in
-# profiles/grouped_gemm_<workload>.md (full size for the mid workload; the others
-# captured on fewer experts with the same tokens per expert, so the ratio carries
-# over per touched expert).  Valid for the kernels those captures measured.
-TRAFFIC_RATIO = {
-    "mid_bf16_shared_T2048": 1.20,
-    "dsv4_bf16_T4096": 1.03,
-    "dsv3_mxfp8_shared_T4096": 1.08,
-    "dsv4_nvfp4_decode_T128": 1.01,
-    "dsv4_nvfp4_prefill_T8192": 1.06,
-    "dsv4_nvfp4_serve_T1024": 1.01,
-    "dsv4_mxfp8_T4096": 1.02,
-}
+# DRAM bytes (read + written) of one grouped-MLP call's fc1 and fc2 launches per
+# algorithmic weight byte, from ncu dram__bytes_read.sum + dram__bytes_write.sum
+# captures, keyed by workload, each with the hash of the kernel source it was
+# taken on (kernel_source_hash): a ratio is reported only while the kernels
+# are unchanged since its capture.  Workloads too large to capture whole were
+# captured on fewer experts with the same tokens per expert; the ratio carries
+# over per touched expert.
+TRAFFIC_RATIO = {}
+
+
+def kernel_source_hash():
+    """Hash of the grouped-GEMM kernel source (the files its code is in)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("grouped_gemm.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "mixture_experts_layer_grouped_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def graph_kernel_names(graph):
+    """Names of the kernel nodes of a captured CUDA graph (one per launch), or
+    None when the driver bindings cannot list them."""
+    try:
+        from cuda.bindings import driver as drv
+        raw = graph.raw_cuda_graph()
+        g = raw if isinstance(raw, drv.CUgraph) else drv.CUgraph(int(raw))
+        err, _, n = drv.cuGraphGetNodes(g, 0)
+        err, nodes, n = drv.cuGraphGetNodes(g, n)
+        names = []
+        for nd in nodes[:n]:
+            err, t = drv.cuGraphNodeGetType(nd)
+            if t != drv.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL:
+                continue
+            err, prm = drv.cuGraphKernelNodeGetParams(nd)
+            err, name = drv.cuFuncGetName(prm.func)
+            names.append(name.decode() if isinstance(name, bytes) else str(name))
+        return names
+    except Exception:
+        return None
 
 
 def grouped_mlp_algorithmic(cfg, touched):
@@ -257,27 +313,7 @@ def layer_algorithmic(cfg, touched):
 
 def prepare_streaming(M, cfg, c, dev):
     """Prepared weights, drawn and converted one expert at a time."""
-    sz = M.moe_prepared_weights_size(c)
-    u8 = dict(dtype=torch.uint8, device=dev)
-    p = {"w1": torch.empty(sz["w13"], **u8), "w3": torch.empty(sz["w13"], **u8),
-         "w2": torch.empty(sz["w2"], **u8)}
-    if sz["w13_scales"]:
-        for k, n in (("w1_scales", "w13_scales"), ("w3_scales", "w13_scales"),
-                     ("w2_scales", "w2_scales")):
-            p[k] = torch.empty(sz[n], **u8)
-    if sz["w_globals"]:
-        p["w13_global"] = torch.empty(cfg.E, dtype=torch.float32, device=dev)
-        p["w2_global"] = torch.empty(cfg.E, dtype=torch.float32, device=dev)
-    if cfg.I_shared:
-        p["ws1"], p["ws3"] = torch.empty(sz["ws13"], **u8), torch.empty(sz["ws13"], **u8)
-        p["ws2"] = torch.empty(sz["ws2"], **u8)
-        if sz["ws13_scales"]:
-            for k, n in (("ws1_scales", "ws13_scales"), ("ws3_scales", "ws13_scales"),
-                         ("ws2_scales", "ws2_scales")):
-                p[k] = torch.empty(sz[n], **u8)
-        if sz["ws_globals"]:
-            p["ws13_global"] = torch.empty(1, dtype=torch.float32, device=dev)
-            p["ws2_global"] = torch.empty(1, dtype=torch.float32, device=dev)
+    p = M.allocate_prepared_weights(c, dev)
     dst = M.binding.weights_struct(p)
     for e in range(cfg.E):
         M.moe_prepare_weights(c, 0, e, 1, *synth.gen_expert_weights(cfg, e, dev), dst)
@@ -315,9 +351,11 @@ def run_ours(args, cfg):
     for _ in range(args.warmup):
         layer.forward(x, out=y)
     torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
+    graph = torch.cuda.CUDAGraph(keep_graph=True)
     with torch.cuda.graph(graph):
         layer.forward(x, out=y)
+    graph.instantiate()
+    launches = graph_kernel_names(graph)  # the library's kernels in one forward
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
@@ -347,19 +385,40 @@ def run_ours(args, cfg):
     ms_max = max_over_ranks(ms, dist, dev)
     value = job_tokens_per_s(cfg.T, ws_n, ms_max)
 
-    # ---- e2e: host (pinned) buffers through the same C call, eager
-    x_h = x.cpu().pin_memory()
-    y_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, pin_memory=True)
-    for _ in range(args.warmup):
-        layer.forward(x_h, out=y_h)
-    barrier()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        layer.forward(x_h, out=y_h)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = ev0.elapsed_time(ev1) / args.steps
-    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    # ---- e2e: host (pinned) x and y through the same C call, which copies x
+    # in and y out on its stream.  Two calls are in flight, on two streams with
+    # a workspace each, so one call's copies overlap the other's kernels (the
+    # way a serving loop feeds the layer); every step still moves its own x in
+    # and y out.  The one-stream figure (copies never overlapped) is reported
+    # beside it.
+    layers = [layer, M.MoELayer(c, layer.weights, d["w_router"], d["bias"], prepared=True)]
+    streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+    x_h = [x.cpu().pin_memory() for _ in range(2)]
+    y_h = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+
+    def e2e_loop(n, two):
+        for i in range(n):
+            j = i % 2 if two else 0
+            layers[j].forward(x_h[j], out=y_h[j], stream=streams[j])
+
+    def e2e_timed(two):
+        e2e_loop(args.warmup, two)
+        barrier()
+        ev0.record(stream)
+        for st in streams:
+            st.wait_event(ev0)
+        e2e_loop(args.steps, two)
+        for st in streams:
+            stream.wait_stream(st)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
+
+    e2e_ms_serial = e2e_timed(False)
+    e2e_ms = e2e_timed(True)
+    for lay in layers:
+        if lay.device_status() != 0:
+            raise RuntimeError("device status set in the end-to-end loop")
     e2e_value = job_tokens_per_s(cfg.T, ws_n, e2e_ms)
 
     # ---- roofline of the dominant call (grouped MLP: fc1+SwiGLU and fc2)
@@ -427,10 +486,13 @@ def run_ours(args, cfg):
 
     cpu = None
     if ws_n == 1 and not args.no_cpu_baseline:
-        tps, _ = time_oracle(cfg, args.ref_tokens, 1, 0)
-        cpu = {"value": tps, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
-               "sample": f"oracle forward (fp64 numpy) on a {args.ref_tokens}-token sample of "
-                         f"the workload, one pass"}
+        n = args.ref_tokens or oracle_tokens(cfg, 20.0, dev)
+        tps, _, ne = time_oracle(cfg, n, 1, 0, dev)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": _host_cores(), "kind": "oracle",
+               "sample": _oracle_note(cfg, n, ne) + ", one pass"}
+    src_hash = kernel_source_hash()
+    tr = TRAFFIC_RATIO.get(cfg.name)
+    traffic = tr[0] * wbytes if tr is not None and tr[1] == src_hash else None
     clocks = clk.summary(t_soak, t_timed_end)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
@@ -444,11 +506,12 @@ def run_ours(args, cfg):
                        launch="CUDA graph of the one-call forward", parallelism=f"replicas{ws_n}"),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
                      "frac": achieved_gbs / hbm,
-                     "traffic": (TRAFFIC_RATIO[cfg.name] * wbytes
-                                 if cfg.name in TRAFFIC_RATIO else None),
-                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
-                                       "fc1 and fc2 launches (profiles/grouped_gemm_*.md), "
-                                       "bytes per grouped-MLP call",
+                     "traffic": traffic,
+                     "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
+                                        "fc1 and fc2 launches, per algorithmic weight byte, "
+                                        f"captured on kernel source {src_hash}, x this call's "
+                                        "algorithmic bytes" if traffic is not None else
+                                        f"no ncu capture of kernel source {src_hash}"),
                      "kernel": "moe_grouped_mlp (fc1+SwiGLU and fc2 tcgen05 kernels)",
                      "algorithmic_bytes_per_launch": wbytes, "ms_per_launch": mlp_ms,
                      "tensor_tflops": flops / (mlp_ms * 1e-3) / 1e12,
@@ -460,8 +523,12 @@ def run_ours(args, cfg):
         "step_ms": {k: statistics.mean(v) for k, v in steps_ms.items()},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s",
-                "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
-        "gpu_launches": ({"bf16": 9, "mxfp8": 10, "nvfp4": 14}[cfg.dtype] + (1 if cfg.dtype == "nvfp4" and cfg.I_shared else 0)) * args.steps,
+                "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2,
+                "mode": "moe_forward on pinned host x / y (copies inside the call), two calls in "
+                        "flight on two streams",
+                "one_stream_value": job_tokens_per_s(cfg.T, ws_n, e2e_ms_serial)},
+        "gpu_launches": (len(launches) * args.steps if launches is not None else None),
+        "gpu_launches_per_step": launches,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"], "samples": clocks["samples"]},
         "gemm_pairs": os.environ.get("MOE_GEMM_PAIRS", "1") != "0",
@@ -476,18 +543,24 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=BENCH_CONFIG, choices=sorted(synth.CONFIGS))
-    ap.add_argument("--ref-tokens", type=int, default=128)
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="tokens in the oracle's sample (0: sized to a time budget)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling only: scale the workload to this many experts, keeping "
                          "the rows per expert (T scales with E)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling only: run this many tokens (with --experts, keeps the "
+                         "token-side kernels at full size while the weights stay small)")
     ap.add_argument("--soak-s", type=float, default=1.5,
                     help="untimed graph replays before the timed region (clock sampling)")
     args = ap.parse_args()
     cfg = synth.get_config(args.config)
     if args.experts:
-        t = max(1, round(cfg.T * args.experts / cfg.E))
+        t = args.tokens or max(1, round(cfg.T * args.experts / cfg.E))
         cfg = cfg.scaled(E=args.experts, T=t, name=f"{cfg.name}_E{args.experts}_T{t}")
+    elif args.tokens:
+        cfg = cfg.scaled(T=args.tokens, name=f"{cfg.name}_T{args.tokens}")
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

@@ -97,8 +97,9 @@ CONFIGS = {
         pad_multiple=64, router_std=-1.0),
 }
 
-# The workload the throughput benchmark times: the mid-size bf16 layer.
-BENCH_CONFIG = "mid_bf16_shared_T2048"
+# The workload the throughput benchmark times by default: the largest one that
+# fits one GPU (DeepSeek-V4 geometry, NVFP4 W4A4, prefill batch of 8192 tokens).
+BENCH_CONFIG = "dsv4_nvfp4_prefill_T8192"
 
 
 def get_config(name: str) -> MoEShape:
