@@ -207,28 +207,35 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * moe_permute without a workspace.  The pages have no counterpart to this
- * call; it exists for callers that cannot allocate device memory: code that
- * runs under an engine or framework that owns every device allocation (a
- * plugin handed only its input and output buffers), and code that must not
- * call cudaMalloc because cudaMalloc can synchronize the device.
+ * moe_permute without a workspace, for bf16 layers.  The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory: code that runs under an engine or framework that owns every device
+ * allocation (a plugin handed only its input and output buffers), and code
+ * that must not call cudaMalloc because cudaMalloc can synchronize the device.
  *
- * Same arguments, outputs and results as moe_permute, minus the workspace.
+ * Arguments and results are those of moe_permute for a MOE_BF16 config, with
+ * these differences:
+ *   - dtype must be MOE_BF16 (MOE_ERR_UNSUPPORTED otherwise): the call gathers
+ *     bf16 rows only;
+ *   - dst_rows and src_rows are required (MOE_ERR_INVALID_ARG when NULL);
+ *   - src_scales and dst_scales must be NULL (MOE_ERR_INVALID_ARG otherwise);
+ *   - there is no workspace and no status word: an expert index outside
+ *     [0, E) is dropped (its token_row is -1), as in moe_permute, but is not
+ *     reported.
  * The histogram scratch is a fixed 1 MiB int32 array compiled into the
  * library (static __device__ storage, held on every GPU that loads the
  * library until the process exits), so ceil(T*top_k/256) * E must be at most
  * 262144; larger shapes return MOE_ERR_WORKSPACE with a message on stderr and
  * launch nothing.  The call allocates and frees nothing.
  *
- *   - The first call on each device looks up the array's device address
+ *   - The first call in each CUDA context (per device, and again after a
+ *     device reset) looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture on the device.
  *   - Every call on a device shares the one array.  Nothing in it needs to
  *     start at zero (each call writes every entry before reading it), but
  *     calls whose kernels overlap on the GPU -- on different streams, or from
  *     different host threads -- race on it and give wrong results.
- *   - There is no status word: an expert index outside [0, E) is dropped
- *     (its token_row is -1), as in moe_permute, but is not reported.
  */
 moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx,
                                const void* src_rows, const void* src_scales,

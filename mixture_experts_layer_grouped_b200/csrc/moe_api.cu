@@ -1190,20 +1190,51 @@ namespace {
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 int32_t* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kNoAllocMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the current CUDA context (ids are never reused, so a context
+// re-created after a device reset gets a new one); 0 if it cannot be read.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &a, 12000, cudaEnableDefault, &qa) !=
+            cudaSuccess || qa != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPointByVersion("cuCtxGetId", &b, 12000, cudaEnableDefault, &qb) !=
+            cudaSuccess || qb != cudaDriverEntryPointSuccess)
+      return 0;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    get_id = reinterpret_cast<CtxGetIdFn>(b);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of the scratch array on the current device.  Host code must
 // not use the array's name as a pointer: on the host it is only a stand-in
-// for the symbol.  The address is looked up once per device, with that device
-// current, and cached.
+// for the symbol.  The address is looked up with the device current, once
+// per device and CUDA context (again after a device reset re-creates the
+// context), and cached.
 moe_status noalloc_scratch(int32_t** out) {
   int dev = 0;
   MOE_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_UNSUPPORTED;
+  // 0 before the device's context exists; the symbol lookup then creates it
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     MOE_CUDA(cudaGetSymbolAddress(&p, moe_noalloc_permute_scratch));
     g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+    g_noalloc_ctx[dev] = current_context_id();
   }
   *out = g_noalloc_ptr[dev];
   return MOE_OK;
@@ -1216,10 +1247,9 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
                                           int32_t* counts, int32_t* offsets, int32_t* row_token,
                                           int32_t* token_row, void* dst_rows, void* dst_scales,
                                           void* stream) {
-  (void)src_scales;
-  (void)dst_scales;
   MOE_TRY(check_config(cfg));
   if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;  // gathers bf16 rows only
+  if (src_scales || dst_scales) return MOE_ERR_INVALID_ARG;  // bf16 rows carry no scales
   if (!topk_idx || !src_rows || !counts || !offsets || !row_token || !token_row || !dst_rows)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(src_rows) || !aligned16(dst_rows)) return MOE_ERR_INVALID_ARG;

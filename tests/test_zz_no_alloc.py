@@ -6,11 +6,12 @@ its input and output buffers, or code that must not call cudaMalloc because it
 can synchronize the whole device.  moe_permute_noalloc serves them: its
 histogram scratch is a fixed array compiled into the library instead of a
 caller-provided workspace.  These tests check, through the C ABI, that it
-returns exactly what moe_permute returns (the permute's outputs are integer
-maps and copied rows, so the tolerance is bit-exact), on two calls in a row
-with different routings so that stale scratch contents from the first call
-would show in the second, and that shapes too large for the built-in scratch
-are refused before anything is launched.
+returns exactly what moe_permute returns and what the oracle's maps and
+gather give (the permute's outputs are integer maps and copied rows, so the
+tolerance is bit-exact), on two calls in a row with different routings so
+that stale scratch contents from the first call would show in the second, and
+that what it does not serve (shapes too large for the built-in scratch, block
+scales, block-scaled types) is refused before anything is launched.
 
 This file is collected last so that a run stopping at its first failure has
 already run every other test.
@@ -23,6 +24,7 @@ import pytest
 import torch
 
 import synth
+from oracle import moe_oracle as O
 
 
 def _outputs(cfg, r_cap):
@@ -61,6 +63,15 @@ def test_permute_noalloc_matches_permute_on_two_calls(name):
             assert torch.equal(got[k], ref[k]), (call, k)
         assert torch.equal(got["rows"][:n].view(torch.int16), ref["rows"][:n].view(torch.int16))
         assert M.moe_get_device_status(ws) == 0
+        # and both are the oracle's maps and rows
+        m = O.permute_maps(idx.cpu().numpy(), cfg.E, cfg.pad_multiple)
+        assert np.array_equal(got["counts"].cpu().numpy(), m["counts"])
+        assert np.array_equal(got["offsets"].cpu().numpy(), m["offsets"])
+        rt = got["row_token"].cpu().numpy()
+        assert np.array_equal(rt[:n], m["row_token"]) and np.all(rt[n:] == -1)
+        assert np.array_equal(got["token_row"].cpu().numpy(), m["token_row"])
+        ref_rows = O.gather_rows(x.cpu().view(torch.int16).numpy(), m["row_token"])
+        assert np.array_equal(got["rows"][:n].cpu().view(torch.int16).numpy(), ref_rows)
 
 
 def test_permute_noalloc_refuses_shapes_beyond_its_scratch():
@@ -73,3 +84,23 @@ def test_permute_noalloc_refuses_shapes_beyond_its_scratch():
     code = M.lib().moe_permute_noalloc(ctypes.byref(c), fake, fake, None, fake, fake, fake, fake,
                                        fake, None, None)
     assert code == 3  # MOE_ERR_WORKSPACE
+
+
+def test_permute_noalloc_refuses_scales_and_block_scaled_types():
+    import mixture_experts_layer_grouped_b200 as M
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the argument checks fail first
+    s = synth.get_config("tiny_bf16_T64")
+    c = M.config_from_shape(s)
+    args = [fake] * 7
+    # src_scales or dst_scales given: bf16 rows carry no scales
+    assert M.lib().moe_permute_noalloc(ctypes.byref(c), fake, fake, fake, *args[:4], fake, None,
+                                       None) == 1
+    assert M.lib().moe_permute_noalloc(ctypes.byref(c), fake, fake, None, *args[:4], fake, fake,
+                                       None) == 1
+    # dst_rows is required
+    assert M.lib().moe_permute_noalloc(ctypes.byref(c), fake, fake, None, *args[:4], None, None,
+                                       None) == 1
+    for dt in ("mxfp8", "nvfp4"):
+        cq = M.config_from_shape(s.scaled(dtype=dt, pad_multiple=64, H=256, I=256))
+        assert M.lib().moe_permute_noalloc(ctypes.byref(cq), fake, fake, fake, *args[:4], fake,
+                                           fake, None) == 2  # MOE_ERR_UNSUPPORTED
