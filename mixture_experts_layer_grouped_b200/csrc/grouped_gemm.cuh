@@ -415,6 +415,36 @@ __device__ __forceinline__ uint32_t swiglu_bf16x2(float g0, float g1, float u0, 
   return bf16x2_bits(h0, h1);
 }
 
+// Scale chunks of one stage, shared memory -> TMEM (in order with the MMAs
+// issued after them).  NVFP4: chunk kk of each weight operand and token chunk
+// cb of MMA kk (at sf_b + 4 * (kk * SFB + cb)); MXFP8: one chunk per operand
+// and token chunk.  Only the first NB token chunks are copied: a tile whose
+// token rows lie in one 128-row chunk reads no other (NB = 1); NB is a
+// compile-time count so that the copies stay straight-line (a data-dependent
+// loop around tcgen05.cp measured several times slower).
+template <bool PAIR, int NA, int SFB, int NB>
+__device__ __forceinline__ void sf_copies_nvf4(uint32_t sf_a0, uint32_t sf_a1, uint32_t sf_b,
+                                               uint32_t ssf, uint32_t cb_bytes) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    tmem_cp_sf_chunk_x<PAIR>(sf_a0 + 4 * kk, sdesc_sf_chunk(ssf + kk * 512));
+    if (NA == 2) tmem_cp_sf_chunk_x<PAIR>(sf_a1 + 4 * kk, sdesc_sf_chunk(ssf + cb_bytes + kk * 512));
+#pragma unroll
+    for (int cb = 0; cb < NB; ++cb)
+      tmem_cp_sf_chunk_x<PAIR>(sf_b + 4 * (kk * SFB + cb),
+                               sdesc_sf_chunk(ssf + (NA + cb) * cb_bytes + kk * 512));
+  }
+}
+template <bool PAIR, int NA, int NB>
+__device__ __forceinline__ void sf_copies_mxf8(uint32_t sf_a0, uint32_t sf_a1, uint32_t sf_b,
+                                               uint32_t ssf) {
+  tmem_cp_sf_chunk_x<PAIR>(sf_a0, sdesc_sf_chunk(ssf));
+  if (NA == 2) tmem_cp_sf_chunk_x<PAIR>(sf_a1, sdesc_sf_chunk(ssf + 512));
+#pragma unroll
+  for (int cb = 0; cb < NB; ++cb)
+    tmem_cp_sf_chunk_x<PAIR>(sf_b + 4 * cb, sdesc_sf_chunk(ssf + (NA + cb) * 512));
+}
+
 // PAIR: the kernel runs as clusters of two CTAs; rank 0 issues M = 256 MMAs
 // over both CTAs' shared memory (cta_group::2), each CTA loads its own 128
 // weight rows and half of the tile's token rows, and the loads of both count
@@ -747,6 +777,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         const uint32_t idesc = idesc_bf16(M_MMA, n_mma);
         // token j's scale sits at chunk row (row0 % 128) + j: shift the TMEM base
         const uint32_t sfb_shift = static_cast<uint32_t>((t.row0 & 127) >> 5);
+        // the MMA reads token scales of rows (row0 % 128) .. + n_mma - 1
+        const bool one_chunk = (t.row0 & 127) + n_mma <= 128;
         const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
@@ -775,20 +807,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             const uint32_t sf_a0 = tmem_base + C::SF_TMEM + (C::SF_BUFS == 2 ? (kt & 1) : 0) * C::SF_COLS;
             const uint32_t sf_a1 = sf_a0 + 4 * C::SF_KCH;
             const uint32_t sf_b = sf_a0 + 4 * C::SF_KCH * C::NA;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              tmem_cp_sf_chunk_x<PAIR>(sf_a0 + 4 * kk, sdesc_sf_chunk(ssf + kk * C::SF_CHUNK));
-              if (C::NA == 2)
-                tmem_cp_sf_chunk_x<PAIR>(sf_a1 + 4 * kk, sdesc_sf_chunk(ssf + cb_bytes + kk * C::SF_CHUNK));
-              // every token chunk slot is copied, also past the tile's nsfb: a
-              // fixed count keeps the copies straight-line (a data-dependent loop
-              // around tcgen05.cp measured several times slower); the extra
-              // slots hold scales of columns past the tile's tokens, never stored
-#pragma unroll
-              for (int cb = 0; cb < C::SFB_CHUNKS; ++cb)
-                tmem_cp_sf_chunk_x<PAIR>(sf_b + 4 * (kk * C::SFB_CHUNKS + cb),
-                                 sdesc_sf_chunk(ssf + (C::NA + cb) * cb_bytes + kk * C::SF_CHUNK));
-            }
+            // a multi-chunk tile copies every token chunk slot, also past the ones
+            // its rows reach (those slots feed only columns that are never stored)
+            if (one_chunk)
+              sf_copies_nvf4<PAIR, C::NA, C::SFB_CHUNKS, 1>(sf_a0, sf_a1, sf_b, ssf, cb_bytes);
+            else
+              sf_copies_nvf4<PAIR, C::NA, C::SFB_CHUNKS, C::SFB_CHUNKS>(sf_a0, sf_a1, sf_b, ssf,
+                                                                       cb_bytes);
             const uint32_t id = idesc_nvf4(M_MMA, n_mma);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -805,11 +830,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             const uint32_t sf_a0 = tmem_base + C::SF_TMEM + (C::SF_BUFS == 2 ? (kt & 1) : 0) * C::SF_COLS;
             const uint32_t sf_a1 = sf_a0 + 4;
             const uint32_t sf_b = sf_a0 + 4 * C::NA;
-            tmem_cp_sf_chunk_x<PAIR>(sf_a0, sdesc_sf_chunk(ssf));
-            if (C::NA == 2) tmem_cp_sf_chunk_x<PAIR>(sf_a1, sdesc_sf_chunk(ssf + C::SF_CHUNK));
-#pragma unroll
-            for (int cb = 0; cb < C::SFB_CHUNKS; ++cb)  // fixed count, as in the NVFP4 branch
-              tmem_cp_sf_chunk_x<PAIR>(sf_b + 4 * cb, sdesc_sf_chunk(ssf + (C::NA + cb) * C::SF_CHUNK));
+            if (one_chunk) sf_copies_mxf8<PAIR, C::NA, 1>(sf_a0, sf_a1, sf_b, ssf);
+            else sf_copies_mxf8<PAIR, C::NA, C::SFB_CHUNKS>(sf_a0, sf_a1, sf_b, ssf);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t accum = (kt > t.k_begin || kk) ? 1u : 0u;
