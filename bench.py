@@ -347,9 +347,12 @@ def run_ours(args, cfg):
         torch.cuda.synchronize()
 
     clk = ClockSampler(local).__enter__()
-    # warm-up (eager), then capture one forward into a CUDA graph
+    # warm-up (eager; an NVTX range per forward lets a profiler pick out the
+    # kernels of one call), then capture one forward into a CUDA graph
     for _ in range(args.warmup):
+        torch.cuda.nvtx.range_push("moe_forward")
         layer.forward(x, out=y)
+        torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph(keep_graph=True)
     with torch.cuda.graph(graph):

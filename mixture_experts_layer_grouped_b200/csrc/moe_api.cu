@@ -452,6 +452,34 @@ moe_status do_route(const moe_config& c, const void* x, const void* w_router, co
   return launch_check();
 }
 
+// Histogram, padded offsets and the two row maps (no row is copied).
+moe_status do_permute_maps(const moe_config& c, const int32_t* topk_idx, int32_t* counts,
+                           int32_t* offsets, int32_t* row_token, int32_t* token_row, void* ws,
+                           cudaStream_t s) {
+  const StepLayout L = step_layout(c);
+  PermArgs a;
+  a.topk_idx = topk_idx;
+  a.hist = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + L.hist);
+  a.counts = counts;
+  a.offsets = offsets;
+  a.row_token = row_token;
+  a.token_row = token_row;
+  a.status = status_ptr(ws);
+  a.n = c.T * c.top_k;
+  a.k = c.top_k;
+  a.E = c.E;
+  a.P = c.pad_multiple;
+  a.r_cap = L.r_cap;
+  a.ntiles = L.ntiles;
+  const size_t hsm = static_cast<size_t>(c.E) * 4;
+  MOE_TRY(launch_pdl(permute_hist_kernel, dim3(L.ntiles), dim3(256), hsm, s, a));
+  MOE_TRY(launch_check());
+  MOE_TRY(launch_pdl(permute_scan_kernel, dim3((c.E + 7) / 8), dim3(256), 0, s, a));
+  MOE_TRY(launch_check());
+  MOE_TRY(launch_pdl(permute_rank_kernel, dim3(L.ntiles), dim3(256), 0, s, a));
+  return launch_check();
+}
+
 moe_status do_permute(const moe_config& c, const int32_t* topk_idx, const void* src_rows,
                       const void* src_scales, int32_t* counts, int32_t* offsets,
                       int32_t* row_token, int32_t* token_row, void* dst_rows, void* dst_scales,
@@ -1137,19 +1165,52 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   void* shared_out = c.I_shared > 0 ? b + F.shared_out : nullptr;
   MOE_TRY(zero_mlp_scratch(c, workspace, s));
   MOE_TRY(do_route(c, xd, w_router, bias, nullptr, logits, topk_idx, topk_w, workspace, s));
-  const void* xq = xd;
-  MlpQuant q{nullptr, nullptr, nullptr, nullptr};
-  if (!is_bf16(c)) {
-    float* xg = reinterpret_cast<float*>(b + F.x_g);
-    MOE_TRY(moe_quantize(c.dtype, xd, c.T, c.H, b + F.x_q, b + F.x_sf, xg, s));
-    xq = b + F.x_q;
-    q = MlpQuant{b + F.rows_sf, b + F.x_sf, xg, nullptr};
-  }
   // an expert-major copy of the rows: fc1 reads it with 32-row TMA boxes, which
   // streams faster than per-row gathers from x (moe_grouped_mlp with rows == NULL)
   void* rows = b + F.rows;
-  MOE_TRY(do_permute(c, topk_idx, xq, q.x_scales, counts, offsets, row_token, token_row, rows,
-                     b + F.rows_sf, workspace, s));
+  const void* xq = xd;
+  MlpQuant q{nullptr, nullptr, nullptr, nullptr};
+  if (is_bf16(c)) {
+    MOE_TRY(do_permute(c, topk_idx, xd, nullptr, counts, offsets, row_token, token_row, rows,
+                       nullptr, workspace, s));
+  } else {
+    // MXFP8 / NVFP4: each token is quantized once and its codes and scales go
+    // straight to its expert-major rows (and to token order for the shared
+    // expert); NVFP4 first takes x's global scale from its amax
+    float* xg = reinterpret_cast<float*>(b + F.x_g);
+    if (is_nv(c)) {
+      const int64_t n = static_cast<int64_t>(c.T) * c.H;
+      MOE_CUDA(cudaMemsetAsync(xg, 0, 4, s));
+      const unsigned nb = static_cast<unsigned>((n / 8 + 255) / 256 < 2048 ? (n / 8 + 255) / 256 : 2048);
+      MOE_TRY(launch_pdl(amax_groups_kernel, dim3(nb, 1), dim3(256), 0, s,
+                         static_cast<const __nv_bfloat16*>(xd), n, xg));
+      MOE_TRY(launch_check());
+      MOE_TRY(launch_pdl(amax_to_global_kernel, dim3(1), dim3(32), 0, s, xg, 1));
+      MOE_TRY(launch_check());
+    }
+    MOE_TRY(do_permute_maps(c, topk_idx, counts, offsets, row_token, token_row, workspace, s));
+    const bool sh = c.I_shared > 0;
+    QScatterArgs qa;
+    qa.x = static_cast<const __nv_bfloat16*>(xd);
+    qa.token_row = token_row;
+    qa.row_token = row_token;
+    qa.offsets = offsets;
+    qa.rows = static_cast<uint8_t*>(rows);
+    qa.rows_sf = b + F.rows_sf;
+    qa.xq = sh ? b + F.x_q : nullptr;
+    qa.xq_sf = sh ? b + F.x_sf : nullptr;
+    qa.g = xg;
+    qa.T = c.T;
+    qa.H = c.H;
+    qa.k = c.top_k;
+    qa.E = c.E;
+    const dim3 grid(sm_count() * 8), block(256);
+    if (is_nv(c)) MOE_TRY(launch_pdl(quantize_scatter_kernel<true>, grid, block, 0, s, qa));
+    else MOE_TRY(launch_pdl(quantize_scatter_kernel<false>, grid, block, 0, s, qa));
+    MOE_TRY(launch_check());
+    xq = b + F.x_q;
+    q = MlpQuant{b + F.rows_sf, b + F.x_sf, xg, nullptr};
+  }
   MOE_TRY(do_grouped_mlp(c, *w, rows, xq, q, counts, offsets, out_rows, shared_out, workspace,
                          s, /*scratch_zeroed=*/true));
   MOE_TRY(do_combine(c, out_rows, token_row, topk_w, shared_out, yd, s));
