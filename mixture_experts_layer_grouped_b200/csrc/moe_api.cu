@@ -1173,12 +1173,22 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   if (is_bf16(c)) {
     MOE_TRY(do_permute(c, topk_idx, xd, nullptr, counts, offsets, row_token, token_row, rows,
                        nullptr, workspace, s));
-  } else {
-    // MXFP8 / NVFP4: each token is quantized once and its codes and scales go
-    // straight to its expert-major rows (and to token order for the shared
-    // expert); NVFP4 first takes x's global scale from its amax
+  } else if (is_mx(c)) {
+    // MXFP8: quantize in token order, then gather codes and scales (its top_k
+    // row copies make the one-pass form below write-bound and slower on B200:
+    // DeepSeek-V3 dims 103 us against 15 + 73 us)
     float* xg = reinterpret_cast<float*>(b + F.x_g);
-    if (is_nv(c)) {
+    MOE_TRY(moe_quantize(c.dtype, xd, c.T, c.H, b + F.x_q, b + F.x_sf, xg, s));
+    xq = b + F.x_q;
+    q = MlpQuant{b + F.rows_sf, b + F.x_sf, xg, nullptr};
+    MOE_TRY(do_permute(c, topk_idx, xq, q.x_scales, counts, offsets, row_token, token_row, rows,
+                       b + F.rows_sf, workspace, s));
+  } else {
+    // NVFP4: each token is quantized once and its codes and scales go straight
+    // to its expert-major rows (and to token order for the shared expert),
+    // after x's global scale is taken from its amax
+    float* xg = reinterpret_cast<float*>(b + F.x_g);
+    {
       const int64_t n = static_cast<int64_t>(c.T) * c.H;
       MOE_CUDA(cudaMemsetAsync(xg, 0, 4, s));
       const unsigned nb = static_cast<unsigned>((n / 8 + 255) / 256 < 2048 ? (n / 8 + 255) / 256 : 2048);
@@ -1205,8 +1215,7 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
     qa.k = c.top_k;
     qa.E = c.E;
     const dim3 grid(sm_count() * 8), block(256);
-    if (is_nv(c)) MOE_TRY(launch_pdl(quantize_scatter_kernel<true>, grid, block, 0, s, qa));
-    else MOE_TRY(launch_pdl(quantize_scatter_kernel<false>, grid, block, 0, s, qa));
+    MOE_TRY(launch_pdl(quantize_scatter_kernel<true>, grid, block, 0, s, qa));
     MOE_TRY(launch_check());
     xq = b + F.x_q;
     q = MlpQuant{b + F.rows_sf, b + F.x_sf, xg, nullptr};

@@ -399,10 +399,10 @@ __device__ __forceinline__ uint32_t gather_scale_word(uint32_t byte, int lane) {
   return (lane & 3) == 0 ? w : 0u;
 }
 
-// A warp per token (then per pad row).  NV = true: NVFP4 (16-element blocks,
-// 8 code bytes each); false: MXFP8 (32-element blocks, 32 code bytes).  H is
-// a multiple of 256 (NVFP4) or 128 (MXFP8), so a round of 32 lanes covers
-// whole 4-block scale words.
+// Work items of one token and 32 consecutive blocks of its row (a block per
+// lane), so that short batches still spread over every SM; then a warp per
+// expert-major row, zeroing the pads.  NV = true: NVFP4 (16-element blocks, 8
+// code bytes each); false: MXFP8 (32-element blocks, 32 code bytes).
 template <bool NV>
 __global__ void __launch_bounds__(256) quantize_scatter_kernel(QScatterArgs a) {
   pdl_wait();
@@ -410,92 +410,85 @@ __global__ void __launch_bounds__(256) quantize_scatter_kernel(QScatterArgs a) {
   constexpr int BE = NV ? 16 : 32;   // elements per block
   constexpr int CB = NV ? 8 : 32;    // code bytes per block
   const int lane = threadIdx.x & 31;
-  const int KB = a.H / BE, row_bytes = KB * CB;
+  const int KB = a.H / BE, row_bytes = KB * CB, nch = (KB + 31) / 32;
   const int64_t warp0 = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const float g = NV ? __ldg(a.g) : 1.0f;
-  for (int64_t t = warp0; t < a.T; t += warps) {
+  const int64_t items = static_cast<int64_t>(a.T) * nch;
+  for (int64_t it = warp0; it < items; it += warps) {
+    const int64_t t = it / nch;
+    // KB is a multiple of 4 (H % 128 == 0), so the four lanes of a scale word
+    // are all in range or all past it; every lane takes part in the shuffles
+    const int kb = static_cast<int>(it - t * nch) * 32 + lane;
+    const bool valid = kb < KB;
     int dst = -1;  // lane j < k: row of (t, j)
     if (lane < a.k) dst = __ldg(a.token_row + t * a.k + lane);
-    for (int kb0 = 0; kb0 < KB; kb0 += 32) {
-      // KB is a multiple of 4 (H % 128 == 0), so the four lanes of a scale word
-      // are all in range or all past it; every lane takes part in the shuffles
-      const int kb = kb0 + lane;
-      const bool valid = kb < KB;
-      const __nv_bfloat16* src = a.x + t * a.H + static_cast<int64_t>(valid ? kb : 0) * BE;
-      uint4 code[2];
-      uint2 code8 = make_uint2(0, 0);
-      uint32_t sc = 0;
-      if (!valid) {
-      } else if constexpr (NV) {
-        float v[16];
-        load_bf16x16(src, v);
-        uint32_t packed[2];
-        sc = nv_quantize_block16(v, g, packed);
-        code8 = make_uint2(packed[0], packed[1]);
+    const __nv_bfloat16* src = a.x + t * a.H + static_cast<int64_t>(valid ? kb : 0) * BE;
+    uint4 code[2];
+    uint2 code8 = make_uint2(0, 0);
+    uint32_t sc = 0;
+    if (!valid) {
+    } else if constexpr (NV) {
+      float v[16];
+      load_bf16x16(src, v);
+      uint32_t packed[2];
+      sc = nv_quantize_block16(v, g, packed);
+      code8 = make_uint2(packed[0], packed[1]);
+    } else {
+      float v[32];
+      load_bf16x16(src, *reinterpret_cast<float(*)[16]>(v));
+      load_bf16x16(src + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      sc = mx_scale_code(amax);
+      const float inv = mx_inv_scale(sc);
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        w[i] = static_cast<uint32_t>(to_e4m3(v[4 * i] * inv)) |
+               (static_cast<uint32_t>(to_e4m3(v[4 * i + 1] * inv)) << 8) |
+               (static_cast<uint32_t>(to_e4m3(v[4 * i + 2] * inv)) << 16) |
+               (static_cast<uint32_t>(to_e4m3(v[4 * i + 3] * inv)) << 24);
+      code[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      code[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+    const uint32_t word = gather_scale_word(sc, lane);
+    for (int j = 0; j <= a.k; ++j) {
+      int64_t r;
+      uint8_t *codes, *scales;
+      if (j < a.k) {
+        r = __shfl_sync(0xffffffffu, dst, j);
+        if (r < 0) continue;          // an entry the permute dropped (bad expert index)
+        codes = a.rows;
+        scales = a.rows_sf;
       } else {
-        float v[32];
-        load_bf16x16(src, *reinterpret_cast<float(*)[16]>(v));
-        load_bf16x16(src + 16, *reinterpret_cast<float(*)[16]>(v + 16));
-        float amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-        sc = mx_scale_code(amax);
-        const float inv = mx_inv_scale(sc);
-        uint32_t w[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          w[i] = static_cast<uint32_t>(to_e4m3(v[4 * i] * inv)) |
-                 (static_cast<uint32_t>(to_e4m3(v[4 * i + 1] * inv)) << 8) |
-                 (static_cast<uint32_t>(to_e4m3(v[4 * i + 2] * inv)) << 16) |
-                 (static_cast<uint32_t>(to_e4m3(v[4 * i + 3] * inv)) << 24);
-        code[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        code[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        if (a.xq == nullptr) break;   // token order only for the shared expert
+        r = t;
+        codes = a.xq;
+        scales = a.xq_sf;
       }
-      const uint32_t word = gather_scale_word(sc, lane);
-      for (int j = 0; j <= a.k; ++j) {
-        int64_t r;
-        uint8_t *codes, *scales;
-        if (j < a.k) {
-          r = __shfl_sync(0xffffffffu, dst, j);
-          if (r < 0) continue;          // an entry the permute dropped (bad expert index)
-          codes = a.rows;
-          scales = a.rows_sf;
-        } else {
-          if (a.xq == nullptr) break;   // token order only for the shared expert
-          r = t;
-          codes = a.xq;
-          scales = a.xq_sf;
-        }
-        if (!valid) continue;
-        uint8_t* cd = codes + r * row_bytes + static_cast<int64_t>(kb) * CB;
-        if constexpr (NV) {
-          *reinterpret_cast<uint2*>(cd) = code8;
-        } else {
-          reinterpret_cast<uint4*>(cd)[0] = code[0];
-          reinterpret_cast<uint4*>(cd)[1] = code[1];
-        }
-        if ((lane & 3) == 0)
-          *reinterpret_cast<uint32_t*>(scales + sf_offset(r, kb, KB)) = word;
+      if (!valid) continue;
+      uint8_t* cd = codes + r * row_bytes + static_cast<int64_t>(kb) * CB;
+      if constexpr (NV) {
+        *reinterpret_cast<uint2*>(cd) = code8;
+      } else {
+        reinterpret_cast<uint4*>(cd)[0] = code[0];
+        reinterpret_cast<uint4*>(cd)[1] = code[1];
       }
+      if ((lane & 3) == 0)
+        *reinterpret_cast<uint32_t*>(scales + sf_offset(r, kb, KB)) = word;
     }
   }
   // pad rows of the expert-major layout: zero codes and scale words
   const int rows_used = __ldg(a.offsets + a.E);
   const int W = KB / 4;
-  for (int64_t r0 = warp0 * 32; r0 < rows_used; r0 += warps * 32) {
-    const int64_t r = r0 + lane;
-    const bool pad = r < rows_used && __ldg(a.row_token + r) < 0;
-    uint32_t m = __ballot_sync(0xffffffffu, pad);
-    while (m) {
-      const int i = __ffs(m) - 1;
-      m &= m - 1;
-      const int64_t rr = r0 + i;
-      uint4* cd = reinterpret_cast<uint4*>(a.rows + rr * row_bytes);
-      for (int v = lane; v < row_bytes / 16; v += 32) cd[v] = make_uint4(0, 0, 0, 0);
-      for (int w = lane; w < W; w += 32)
-        *reinterpret_cast<uint32_t*>(a.rows_sf + sf_offset(rr, 4 * w, KB)) = 0u;
-    }
+  for (int64_t r = warp0; r < rows_used; r += warps) {
+    if (__ldg(a.row_token + r) >= 0) continue;
+    uint4* cd = reinterpret_cast<uint4*>(a.rows + r * row_bytes);
+    for (int v = lane; v < row_bytes / 16; v += 32) cd[v] = make_uint4(0, 0, 0, 0);
+    for (int w = lane; w < W; w += 32)
+      *reinterpret_cast<uint32_t*>(a.rows_sf + sf_offset(r, 4 * w, KB)) = 0u;
   }
 }
 
