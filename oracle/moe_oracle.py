@@ -426,19 +426,25 @@ def swiglu(a, u):
     return silu(a) * np.asarray(u, np.float64)
 
 
-def expert_fc1(X, W1, W3):
+def _store(v, rounding):
+    """The value a bf16 tensor stores (rounding=False: the exact value, for the
+    smooth function the backward differentiates)."""
+    return round_bf16(v) if rounding else np.asarray(v, np.float64)
+
+
+def expert_fc1(X, W1, W3, rounding=True):
     """h = bf16(silu(X W1^T) * (X W3^T)) for one expert's rows X [m, H]."""
     a = X @ W1.T
     u = X @ W3.T
-    return round_bf16(swiglu(a, u))
+    return _store(swiglu(a, u), rounding)
 
 
-def expert_fc2(h, W2):
+def expert_fc2(h, W2, rounding=True):
     """o = bf16(h W2^T) for one expert's (possibly dequantized) h [m, I]."""
-    return round_bf16(h @ W2.T)
+    return _store(h @ W2.T, rounding)
 
 
-def combine(out_rows, token_row, w, shared_out=None):
+def combine(out_rows, token_row, w, shared_out=None, rounding=True):
     """y[t] = bf16(sum_j w[t, j] * out_rows[token_row[t*k + j]] (+ shared[t])).
 
     The gate-weighted scatter-add of the pages, written as a per-token sum in
@@ -452,7 +458,7 @@ def combine(out_rows, token_row, w, shared_out=None):
         acc += w[:, j:j + 1] * out_rows[tr[:, j]]
     if shared_out is not None:
         acc += shared_out
-    return round_bf16(acc)
+    return _store(acc, rounding)
 
 
 # ---------------------------------------------------------------------------
@@ -472,7 +478,7 @@ def prepare_expert_weights(W1, W3, W2, dtype):
     return w13[:I], w13[I:], quantize_dequantize(W2, dtype)
 
 
-def expert_forward(X_deq, W1, W3, W2, dtype, h_global=None, prepared=False):
+def expert_forward(X_deq, W1, W3, W2, dtype, h_global=None, prepared=False, rounding=True):
     """One expert on its rows: dequantized x rows in, bf16 fc2 rows out.
 
     W1/W3/W2 are the bf16 weight values, or (``prepared=True``) the output of
@@ -482,24 +488,26 @@ def expert_forward(X_deq, W1, W3, W2, dtype, h_global=None, prepared=False):
     unless ``h_global`` is given.
     """
     w1, w3, w2 = (W1, W3, W2) if prepared else prepare_expert_weights(W1, W3, W2, dtype)
-    h = expert_fc1(X_deq, w1, w3)
+    h = expert_fc1(X_deq, w1, w3, rounding)
     if dtype == "nvfp4":
         g = nvfp4_global_scale(np.abs(h).max()) if h_global is None else h_global
         hq = quantize_dequantize(h, dtype, g)
     else:
         hq = quantize_dequantize(h, dtype)
-    return h, expert_fc2(hq, w2)
+    return h, expert_fc2(hq, w2, rounding)
 
 
 def forward(cfg, x, w_router, bias, w1, w3, w2, shared=None, logits=None,
-            experts=None):
+            experts=None, rounding=True):
     """Full layer forward on the host.
 
     ``x``, ``w_router`` and the weights are float64 arrays of the bf16 inputs;
     ``w1``/``w3``/``w2`` may be callables ``e -> array`` so that large
     workloads can hand over one expert at a time.  ``experts`` limits the
     expert math to a subset (rows of other experts stay zero); the routing,
-    the maps and the quantized x cover all tokens.
+    the maps and the quantized x cover all tokens.  ``rounding=False`` skips
+    the bf16 storage of h, the fc2 rows and y (the smooth function the
+    backward differentiates).
     """
     T, H = x.shape
     E = cfg.E
@@ -520,12 +528,104 @@ def forward(cfg, x, w_router, bias, w1, w3, w2, shared=None, logits=None,
         lo, cnt = int(m["offsets"][e]), int(m["counts"][e])
         if cnt == 0:
             continue
-        h, o = expert_forward(rows[lo:lo + cnt], get(w1, e), get(w3, e), get(w2, e), cfg.dtype)
+        h, o = expert_forward(rows[lo:lo + cnt], get(w1, e), get(w3, e), get(w2, e), cfg.dtype,
+                              rounding=rounding)
         h_rows[lo:lo + cnt] = h
         out_rows[lo:lo + cnt] = o
     shared_out = None
     if shared is not None:
-        _, shared_out = expert_forward(xq, shared[0], shared[1], shared[2], cfg.dtype)
-    y = combine(out_rows, m["token_row"], r["w"], shared_out)
+        _, shared_out = expert_forward(xq, shared[0], shared[1], shared[2], cfg.dtype,
+                                       rounding=rounding)
+    y = combine(out_rows, m["token_row"], r["w"], shared_out, rounding)
     return dict(logits=logits, route=r, maps=m, xq=xq, rows=rows, h_rows=h_rows,
                 out_rows=out_rows, shared_out=shared_out, y=y)
+
+
+# ---------------------------------------------------------------------------
+# Backward (input gradients) of the bf16 layer
+# (TransformerEngine PR "DeepSeekV3Layer", Performance, "fused grouped MLP"
+#  row: dGLU backward and the grouped GEMMs of the backward pass)
+# ---------------------------------------------------------------------------
+
+def expert_backward(X, W1, W3, W2, dO):
+    """Input gradient of one expert on its rows.
+
+    Forward: a = X W1^T, u = X W3^T, h = silu(a) u, O = h W2^T.  Given dO =
+    dL/dO [m, H]:
+      dh = dO W2;  da = dh * u * silu'(a);  du = dh * silu(a);
+      dX = da W1 + du W3,
+    with silu'(a) = sigma(a) (1 + a (1 - sigma(a))).  The bf16 storage of h
+    and O has no derivative; it is read as the identity (the gradient of the
+    smooth function, forward with rounding=False).  Returns dX and the
+    intermediates.
+    """
+    X, W1, W3, W2, dO = (np.asarray(t, np.float64) for t in (X, W1, W3, W2, dO))
+    a = X @ W1.T
+    u = X @ W3.T
+    sg = sigmoid(a)
+    dh = dO @ W2
+    da = dh * u * (sg * (1.0 + a * (1.0 - sg)))
+    du = dh * (a * sg)
+    return da @ W1 + du @ W3, dict(a=a, u=u, dh=dh, da=da, du=du)
+
+
+def gate_backward(logits, idx, rsf, dgate):
+    """d logits from d gates.  Gates: w_j = rsf * s_j / S over the selected
+    experts (s = sigmoid(logit), S = sum of the selected s); the selection and
+    the bias are piecewise constant, so only selected experts get a gradient:
+      ds_j = rsf * (g_j / S - sum_i g_i s_i / S^2),  dlogit_j = ds_j s_j (1 - s_j)
+    with g = dL/dw.  Returns [T, E]."""
+    logits = np.asarray(logits, np.float64)
+    s = sigmoid(logits)
+    s_sel = np.take_along_axis(s, idx, axis=1)
+    S = s_sel.sum(axis=1, keepdims=True)
+    g = np.asarray(dgate, np.float64)
+    ds = rsf * (g / S - (g * s_sel).sum(axis=1, keepdims=True) / S ** 2)
+    dl = np.zeros_like(logits)
+    np.put_along_axis(dl, idx, ds * s_sel * (1.0 - s_sel), axis=1)
+    return dl
+
+
+def backward(cfg, x, w_router, bias, w1, w3, w2, dy, shared=None, logits=None, rounding=True):
+    """dL/dx of the bf16 layer for dL/dy = dy, with its intermediates.
+
+    y[t] = sum_j w[t, j] O[row(t, j)] + shared(x[t]); the combine's backward
+    gives dO[row(t, j)] = w[t, j] dy[t] and dgate[t, j] = <dy[t], O[row(t, j)]>
+    (O as the forward stores it, bf16); each expert's rows give dX rows
+    (expert_backward); dx[t] = sum_j dX[row(t, j)] + shared's dx[t] +
+    (d logits W_r)[t] (gate_backward through the router GEMM).  Weight
+    gradients are not computed.  ``w1``/``w3``/``w2`` may be callables
+    e -> array, as in forward.  ``rounding=False``: the O in dgate is the
+    exact fc2 output (the gradient of forward with rounding=False).
+    """
+    if cfg.dtype != "bf16":
+        raise ValueError("the backward is written for the bf16 layer")
+    get = (lambda W, e: W(e) if callable(W) else W[e])
+    f = forward(cfg, x, w_router, bias, w1, w3, w2, shared=shared, logits=logits,
+                rounding=rounding)
+    r, m = f["route"], f["maps"]
+    dy = np.asarray(dy, np.float64)
+    T, k = r["idx"].shape
+    tr = np.asarray(m["token_row"]).reshape(T, k)
+    dgate = np.einsum("th,tjh->tj", dy, f["out_rows"][tr])
+    dO = np.zeros_like(f["out_rows"])
+    for j in range(k):
+        dO[tr[:, j]] = r["w"][:, j:j + 1] * dy
+    dX_rows = np.zeros_like(f["rows"])
+    for e in range(cfg.E):
+        lo, cnt = int(m["offsets"][e]), int(m["counts"][e])
+        if cnt == 0:
+            continue
+        dX_rows[lo:lo + cnt] = expert_backward(f["rows"][lo:lo + cnt], get(w1, e), get(w3, e),
+                                               get(w2, e), dO[lo:lo + cnt])[0]
+    dx = np.zeros_like(np.asarray(x, np.float64))
+    for j in range(k):
+        dx += dX_rows[tr[:, j]]
+    dx_shared = None
+    if shared is not None:
+        dx_shared = expert_backward(x, shared[0], shared[1], shared[2], dy)[0]
+        dx += dx_shared
+    dl = gate_backward(f["logits"], r["idx"], cfg.rsf, dgate)
+    dx += dl @ np.asarray(w_router, np.float64)
+    return dict(dx=dx, dlogits=dl, dgate=dgate, dO=dO, dX_rows=dX_rows, dx_shared=dx_shared,
+                fwd=f)
