@@ -586,17 +586,32 @@ def gate_backward(logits, idx, rsf, dgate):
     return dl
 
 
-def backward(cfg, x, w_router, bias, w1, w3, w2, dy, shared=None, logits=None, rounding=True):
-    """dL/dx of the bf16 layer for dL/dy = dy, with its intermediates.
+def expert_weight_grads(X, dO, mid, rounding=True):
+    """Weight gradients of one expert from its rows X, dO and the
+    intermediates of expert_backward: with h = silu(a) u as the forward
+    stores it (bf16 when ``rounding``),
+      dW1 = da^T X,  dW3 = du^T X,  dW2 = dO^T h."""
+    X, dO = np.asarray(X, np.float64), np.asarray(dO, np.float64)
+    h = _store(swiglu(mid["a"], mid["u"]), rounding)
+    return mid["da"].T @ X, mid["du"].T @ X, dO.T @ h
+
+
+def backward(cfg, x, w_router, bias, w1, w3, w2, dy, shared=None, logits=None, rounding=True,
+             weight_grads=None):
+    """Gradients of the bf16 layer for dL/dy = dy, with its intermediates.
 
     y[t] = sum_j w[t, j] O[row(t, j)] + shared(x[t]); the combine's backward
     gives dO[row(t, j)] = w[t, j] dy[t] and dgate[t, j] = <dy[t], O[row(t, j)]>
     (O as the forward stores it, bf16); each expert's rows give dX rows
     (expert_backward); dx[t] = sum_j dX[row(t, j)] + shared's dx[t] +
-    (d logits W_r)[t] (gate_backward through the router GEMM).  Weight
-    gradients are not computed.  ``w1``/``w3``/``w2`` may be callables
-    e -> array, as in forward.  ``rounding=False``: the O in dgate is the
-    exact fc2 output (the gradient of forward with rounding=False).
+    (d logits W_r)[t] (gate_backward through the router GEMM).
+    ``weight_grads``: None for none, True for every expert, or an iterable
+    of expert ids; then dw1/dw3/dw2 map those experts to dW1_e, dW3_e, dW2_e
+    (expert_weight_grads on the expert's rows), and dws1/dws3/dws2 (shared
+    expert on x with dO = dy) and dw_router = dlogits^T x are added.
+    ``w1``/``w3``/``w2`` may be callables e -> array, as in forward.
+    ``rounding=False``: the O in dgate and the h in dW2 are the exact values
+    (the gradient of forward with rounding=False).
     """
     if cfg.dtype != "bf16":
         raise ValueError("the backward is written for the bf16 layer")
@@ -611,21 +626,41 @@ def backward(cfg, x, w_router, bias, w1, w3, w2, dy, shared=None, logits=None, r
     dO = np.zeros_like(f["out_rows"])
     for j in range(k):
         dO[tr[:, j]] = r["w"][:, j:j + 1] * dy
+    if weight_grads is None:
+        wg = set()
+    elif weight_grads is True:
+        wg = set(range(cfg.E))
+    else:
+        wg = set(int(e) for e in weight_grads)
+    dw1, dw3, dw2 = {}, {}, {}
     dX_rows = np.zeros_like(f["rows"])
     for e in range(cfg.E):
         lo, cnt = int(m["offsets"][e]), int(m["counts"][e])
         if cnt == 0:
+            if e in wg:
+                dw1[e] = np.zeros((cfg.I, cfg.H))
+                dw3[e] = np.zeros((cfg.I, cfg.H))
+                dw2[e] = np.zeros((cfg.H, cfg.I))
             continue
-        dX_rows[lo:lo + cnt] = expert_backward(f["rows"][lo:lo + cnt], get(w1, e), get(w3, e),
-                                               get(w2, e), dO[lo:lo + cnt])[0]
+        Xe, dOe = f["rows"][lo:lo + cnt], dO[lo:lo + cnt]
+        dX_rows[lo:lo + cnt], mid = expert_backward(Xe, get(w1, e), get(w3, e), get(w2, e), dOe)
+        if e in wg:
+            dw1[e], dw3[e], dw2[e] = expert_weight_grads(Xe, dOe, mid, rounding)
     dx = np.zeros_like(np.asarray(x, np.float64))
     for j in range(k):
         dx += dX_rows[tr[:, j]]
     dx_shared = None
+    out = {}
     if shared is not None:
-        dx_shared = expert_backward(x, shared[0], shared[1], shared[2], dy)[0]
+        dx_shared, mid_s = expert_backward(x, shared[0], shared[1], shared[2], dy)
         dx += dx_shared
+        if weight_grads is not None:
+            out["dws1"], out["dws3"], out["dws2"] = expert_weight_grads(x, dy, mid_s, rounding)
     dl = gate_backward(f["logits"], r["idx"], cfg.rsf, dgate)
     dx += dl @ np.asarray(w_router, np.float64)
-    return dict(dx=dx, dlogits=dl, dgate=dgate, dO=dO, dX_rows=dX_rows, dx_shared=dx_shared,
-                fwd=f)
+    if weight_grads is not None:
+        out.update(dw1=dw1, dw3=dw3, dw2=dw2,
+                   dw_router=dl.T @ np.asarray(x, np.float64))
+    out.update(dx=dx, dlogits=dl, dgate=dgate, dO=dO, dX_rows=dX_rows, dx_shared=dx_shared,
+               fwd=f)
+    return out

@@ -96,3 +96,58 @@ def test_layer_backward_matches_finite_differences():
     assert np.max(np.abs(b["dx"] - fd)) < 1e-6 * max(1.0, np.abs(fd).max())
     # without the router term the gradient is wrong: the pin sees every part
     assert np.max(np.abs((b["dx"] - b["dlogits"] @ wr) - fd)) > 1e-3
+
+
+def test_layer_weight_grads_match_finite_differences():
+    """dW1, dW3, dW2 per expert, the shared expert's and the router's weight
+    gradients, each entry against a central difference of the loss."""
+    cfg = synth.MoEShape(name="bwd_tiny_w", T=5, H=16, I=8, E=4, n_group=2, topk_group=1,
+                         top_k=2, rsf=2.5, I_shared=8, dtype="bf16", pad_multiple=1,
+                         router_std=0.5)
+    rng = np.random.default_rng(7)
+    x = rng.normal(size=(cfg.T, cfg.H))
+    wr = rng.normal(size=(cfg.E, cfg.H)) * 0.5
+    bias = rng.uniform(-0.1, 0.1, size=cfg.E)
+    W = {"w1": rng.normal(size=(cfg.E, cfg.I, cfg.H)) * 0.3,
+         "w3": rng.normal(size=(cfg.E, cfg.I, cfg.H)) * 0.3,
+         "w2": rng.normal(size=(cfg.E, cfg.H, cfg.I)) * 0.3,
+         "ws1": rng.normal(size=(8, 16)) * 0.3, "ws3": rng.normal(size=(8, 16)) * 0.3,
+         "ws2": rng.normal(size=(16, 8)) * 0.3, "wr": wr}
+    dy = rng.normal(size=(cfg.T, cfg.H))
+
+    def run(V, **kw):
+        return O.backward(cfg, x, V["wr"], bias, V["w1"], V["w3"], V["w2"], dy,
+                          shared=(V["ws1"], V["ws3"], V["ws2"]), rounding=False, **kw)
+
+    b = run(W, weight_grads=True)
+    r = b["fwd"]["route"]
+    assert r["expert_margin"].min() > 1e-4 and r["group_margin"].min() > 1e-4
+    counts = b["fwd"]["maps"]["counts"]
+    assert (counts > 0).any()
+
+    def loss(V):
+        f = O.forward(cfg, x, V["wr"], bias, V["w1"], V["w3"], V["w2"],
+                      shared=(V["ws1"], V["ws3"], V["ws2"]), rounding=False)
+        assert np.array_equal(f["route"]["idx"], r["idx"])
+        return float(np.sum(dy * f["y"]))
+
+    analytic = {
+        "w1": np.stack([b["dw1"][e] for e in range(cfg.E)]),
+        "w3": np.stack([b["dw3"][e] for e in range(cfg.E)]),
+        "w2": np.stack([b["dw2"][e] for e in range(cfg.E)]),
+        "ws1": b["dws1"], "ws3": b["dws3"], "ws2": b["dws2"], "wr": b["dw_router"]}
+    eps = 1e-6
+    for name, g in analytic.items():
+        # 24 entries per weight, drawn over every expert and position
+        for flat in rng.choice(g.size, size=min(24, g.size), replace=False):
+            i = np.unravel_index(flat, g.shape)
+            Vp = dict(W); Vm = dict(W)
+            Vp[name] = W[name].copy(); Vm[name] = W[name].copy()
+            Vp[name][i] += eps
+            Vm[name][i] -= eps
+            fd = (loss(Vp) - loss(Vm)) / (2 * eps)
+            assert abs(g[i] - fd) < 1e-6 * max(1.0, abs(fd)), (name, i, g[i], fd)
+    # experts no token picked have zero gradients
+    for e in range(cfg.E):
+        if counts[e] == 0:
+            assert not analytic["w1"][e].any() and not analytic["w2"][e].any()
