@@ -1215,7 +1215,7 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
     qa.k = c.top_k;
     qa.E = c.E;
     const dim3 grid(sm_count() * 8), block(256);
-    MOE_TRY(launch_pdl(quantize_scatter_kernel<true>, grid, block, 0, s, qa));
+    MOE_TRY(launch_pdl(quantize_scatter_nvfp4_kernel, grid, block, 0, s, qa));
     MOE_TRY(launch_check());
     xq = b + F.x_q;
     q = MlpQuant{b + F.rows_sf, b + F.x_sf, xg, nullptr};

@@ -369,91 +369,61 @@ __global__ void __launch_bounds__(256) permute_gather_nv_kernel(GatherMxArgs a) 
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// Quantize and permute in one pass (the forward's path for MXFP8 / NVFP4):
-// each token's row of x is read once, quantized once (the same per-block
-// arithmetic as quantize_mxfp8_rows_kernel / quantize_nvfp4_kernel), and its
-// codes and scales are written to every expert-major row the token feeds
-// (token_row), and to token order when the shared expert needs them.  Expert-
-// major rows without a token (segment pads) get zero codes and scales, as the
-// separate permute gives them.
+// NVFP4 quantize and permute in one pass (the one-call forward's path): each
+// token's row of x is read once, quantized once (the per-block arithmetic of
+// quantize_nvfp4_kernel), and its codes and scales are written to every
+// expert-major row the token feeds (token_row), and to token order when the
+// shared expert needs them.  Expert-major rows without a token (segment pads)
+// get zero codes and scales, as the separate permute gives them.
 // ---------------------------------------------------------------------------
 struct QScatterArgs {
   const __nv_bfloat16* x;     // [T, H]
   const int32_t* token_row;   // [T * k]
   const int32_t* row_token;   // [r_cap]
   const int32_t* offsets;     // [E + 1]: offsets[E] = expert-major rows in use
-  uint8_t* rows;              // [r_cap, row_bytes] codes
+  uint8_t* rows;              // [r_cap, H / 2] packed e2m1 codes
   uint8_t* rows_sf;           // MMA scale layout over r_cap rows
-  uint8_t* xq;                // [T, row_bytes] codes in token order, or null
+  uint8_t* xq;                // [T, H / 2] codes in token order, or null
   uint8_t* xq_sf;             // their scales, or null
-  const float* g;             // NVFP4: global encode scale of x
+  const float* g;             // global encode scale of x
   int T, H, k, E;
 };
 
-// 4 consecutive scale bytes (lanes 4q .. 4q+3) as one word in lane 4q
-__device__ __forceinline__ uint32_t gather_scale_word(uint32_t byte, int lane) {
-  uint32_t w = byte & 0xFFu;
-  w |= (__shfl_down_sync(0xffffffffu, byte, 1) & 0xFFu) << 8;
-  w |= (__shfl_down_sync(0xffffffffu, byte, 2) & 0xFFu) << 16;
-  w |= (__shfl_down_sync(0xffffffffu, byte, 3) & 0xFFu) << 24;
-  return (lane & 3) == 0 ? w : 0u;
-}
-
-// Work items of one token and 32 consecutive blocks of its row (a block per
-// lane), so that short batches still spread over every SM; then a warp per
-// expert-major row, zeroing the pads.  NV = true: NVFP4 (16-element blocks, 8
-// code bytes each); false: MXFP8 (32-element blocks, 32 code bytes).
-template <bool NV>
-__global__ void __launch_bounds__(256) quantize_scatter_kernel(QScatterArgs a) {
+// Work items of one token and 64 consecutive 16-element blocks of its row, two
+// blocks per lane (16 code bytes, one vector store per destination row), so
+// that short batches still spread over every SM; then a warp per expert-major
+// row zeroes the pads.  H % 256 == 0, so the block count KB is a multiple of
+// 16 and the two lanes of a 4-block scale word are both in range or both past it.
+__global__ void __launch_bounds__(256) quantize_scatter_nvfp4_kernel(QScatterArgs a) {
   pdl_wait();
   pdl_trigger();
-  constexpr int BE = NV ? 16 : 32;   // elements per block
-  constexpr int CB = NV ? 8 : 32;    // code bytes per block
   const int lane = threadIdx.x & 31;
-  const int KB = a.H / BE, row_bytes = KB * CB, nch = (KB + 31) / 32;
+  const int KB = a.H / 16, row_bytes = a.H / 2, nch = (KB + 63) / 64;
   const int64_t warp0 = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  const float g = NV ? __ldg(a.g) : 1.0f;
+  const float g = __ldg(a.g);
   const int64_t items = static_cast<int64_t>(a.T) * nch;
   for (int64_t it = warp0; it < items; it += warps) {
     const int64_t t = it / nch;
-    // KB is a multiple of 4 (H % 128 == 0), so the four lanes of a scale word
-    // are all in range or all past it; every lane takes part in the shuffles
-    const int kb = static_cast<int>(it - t * nch) * 32 + lane;
+    const int kb = static_cast<int>(it - t * nch) * 64 + 2 * lane;  // this lane's first block
     const bool valid = kb < KB;
     int dst = -1;  // lane j < k: row of (t, j)
     if (lane < a.k) dst = __ldg(a.token_row + t * a.k + lane);
-    const __nv_bfloat16* src = a.x + t * a.H + static_cast<int64_t>(valid ? kb : 0) * BE;
-    uint4 code[2];
-    uint2 code8 = make_uint2(0, 0);
-    uint32_t sc = 0;
-    if (!valid) {
-    } else if constexpr (NV) {
-      float v[16];
-      load_bf16x16(src, v);
-      uint32_t packed[2];
-      sc = nv_quantize_block16(v, g, packed);
-      code8 = make_uint2(packed[0], packed[1]);
-    } else {
-      float v[32];
-      load_bf16x16(src, *reinterpret_cast<float(*)[16]>(v));
-      load_bf16x16(src + 16, *reinterpret_cast<float(*)[16]>(v + 16));
-      float amax = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-      sc = mx_scale_code(amax);
-      const float inv = mx_inv_scale(sc);
-      uint32_t w[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        w[i] = static_cast<uint32_t>(to_e4m3(v[4 * i] * inv)) |
-               (static_cast<uint32_t>(to_e4m3(v[4 * i + 1] * inv)) << 8) |
-               (static_cast<uint32_t>(to_e4m3(v[4 * i + 2] * inv)) << 16) |
-               (static_cast<uint32_t>(to_e4m3(v[4 * i + 3] * inv)) << 24);
-      code[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      code[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    uint4 code = make_uint4(0, 0, 0, 0);
+    uint32_t sc2 = 0;  // the two blocks' scale bytes
+    if (valid) {
+      const __nv_bfloat16* src = a.x + t * a.H + static_cast<int64_t>(kb) * 16;
+      float v0[16], v1[16];
+      load_bf16x16(src, v0);
+      load_bf16x16(src + 16, v1);
+      uint32_t p0[2], p1[2];
+      const uint32_t s0 = nv_quantize_block16(v0, g, p0);
+      const uint32_t s1 = nv_quantize_block16(v1, g, p1);
+      code = make_uint4(p0[0], p0[1], p1[0], p1[1]);
+      sc2 = (s0 & 0xFFu) | ((s1 & 0xFFu) << 8);
     }
-    const uint32_t word = gather_scale_word(sc, lane);
+    // even lanes hold blocks kb .. kb + 3 of a scale word (kb % 4 == 0)
+    const uint32_t word = sc2 | (__shfl_down_sync(0xffffffffu, sc2, 1) << 16);
     for (int j = 0; j <= a.k; ++j) {
       int64_t r;
       uint8_t *codes, *scales;
@@ -469,14 +439,8 @@ __global__ void __launch_bounds__(256) quantize_scatter_kernel(QScatterArgs a) {
         scales = a.xq_sf;
       }
       if (!valid) continue;
-      uint8_t* cd = codes + r * row_bytes + static_cast<int64_t>(kb) * CB;
-      if constexpr (NV) {
-        *reinterpret_cast<uint2*>(cd) = code8;
-      } else {
-        reinterpret_cast<uint4*>(cd)[0] = code[0];
-        reinterpret_cast<uint4*>(cd)[1] = code[1];
-      }
-      if ((lane & 3) == 0)
+      *reinterpret_cast<uint4*>(codes + r * row_bytes + static_cast<int64_t>(kb) * 8) = code;
+      if ((lane & 1) == 0)
         *reinterpret_cast<uint32_t*>(scales + sf_offset(r, kb, KB)) = word;
     }
   }
