@@ -8,6 +8,7 @@ at prefill size (T=8192, H=7168, I=3072, E=384, groups 8/4, top-6); --config
 picks another.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --backward --config mid_bf16_shared_T2048   (the bf16 backward)
 
 With N > 1 (torchrun) every rank runs an independent replica on its own batch
 (tokens are independent, so the layer shards by batch with no exchange): weak
@@ -331,6 +332,153 @@ def prepare_streaming(M, cfg, c, dev):
     return p
 
 
+def backward_algorithmic(cfg, touched):
+    """Bytes and FLOPs the backward cannot avoid: the touched experts', the
+    shared expert's and the router's bf16 weights read once; their fp32
+    gradients written once; x, dy and the saved rows and fc2 outputs read,
+    dx written.  FLOPs: dh, dX and the three weight gradients, 12*H*I per
+    routed row (the recomputation of a and u, 4*H*I more, is not counted)."""
+    R = cfg.T * cfg.top_k
+    w_el = 3 * cfg.H * (touched * cfg.I + cfg.I_shared) + cfg.E * cfg.H
+    b = 2 * w_el + 4 * w_el + 2 * (3 * cfg.T * cfg.H + 2 * R * cfg.H)
+    f = 12 * cfg.H * (R * cfg.I + cfg.T * cfg.I_shared) + 4 * cfg.T * cfg.H * cfg.E
+    return b, f
+
+
+def run_backward(args, cfg):
+    """The backward of the bf16 layer (moe_backward: dx, router and weight
+    gradients), one call per step, captured in a CUDA graph."""
+    import mixture_experts_layer_grouped_b200 as M
+    if cfg.dtype != "bf16":
+        raise SystemExit("--backward: the backward is built for the bf16 layer")
+    if cfg.pad_multiple % 64:
+        cfg = cfg.scaled(pad_multiple=64)  # routed weight gradients read 64-row steps
+    ws_n, rank, local = _dist()
+    if ws_n > 1:
+        raise SystemExit("--backward runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    c = M.config_from_shape(cfg)
+    x, w_r, bias = replica_inputs(cfg, rank, dev)
+    prepared = prepare_streaming(M, cfg, c, dev)
+    sz = M.moe_backward_weights_size(c)
+    bw = {k: (torch.empty(v, dtype=torch.uint8, device=dev) if v else None)
+          for k, v in sz.items()}
+    for e in range(cfg.E):
+        M.moe_prepare_backward_weights(c, 0, e, 1, *synth.gen_expert_weights(cfg, e, dev), None,
+                                       bw)
+    sh = synth.gen_shared_weights(cfg, dev) or (None, None, None)
+    M.moe_prepare_backward_weights(c, 1, 0, 1, *sh, w_r, bw)
+    # the forward's saved state, through the step calls
+    nbytes, r_cap = M.moe_workspace_size(c)
+    wsf = M.binding.new_workspace(nbytes, dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    T, H, E, I, Is, k = cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k
+    sv = {"x": x, "logits": torch.empty(T, E, dtype=torch.float32, device=dev),
+          "topk_idx": torch.empty(T, k, **i32),
+          "topk_w": torch.empty(T, k, dtype=torch.float32, device=dev),
+          "counts": torch.empty(E, **i32), "offsets": torch.empty(E + 1, **i32),
+          "row_token": torch.empty(r_cap, **i32), "token_row": torch.empty(T * k, **i32),
+          "rows": torch.empty(r_cap, H, dtype=torch.bfloat16, device=dev),
+          "out_rows": torch.empty(r_cap, H, dtype=torch.bfloat16, device=dev)}
+    M.moe_route(c, x, w_r, bias, sv["topk_idx"], sv["topk_w"], wsf, logits_out=sv["logits"])
+    M.moe_permute(c, sv["topk_idx"], x, sv["counts"], sv["offsets"], sv["row_token"],
+                  sv["token_row"], sv["rows"], wsf)
+    shared_out = torch.empty(T, H, dtype=torch.bfloat16, device=dev) if Is else None
+    M.moe_grouped_mlp(c, prepared, sv["rows"], sv["counts"], sv["offsets"], sv["out_rows"], wsf,
+                      x=x, shared_out=shared_out)
+    dy = synth.gen_dy(cfg, dev)
+    dx = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    dlogits = torch.empty(T, E, dtype=torch.float32, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = {"dw1": torch.empty(E, I, H, **f32), "dw3": torch.empty(E, I, H, **f32),
+             "dw2": torch.empty(E, H, I, **f32), "dw_router": torch.empty(E, H, **f32)}
+    if Is:
+        grads.update(dws1=torch.empty(Is, H, **f32), dws3=torch.empty(Is, H, **f32),
+                     dws2=torch.empty(H, Is, **f32))
+    wsb = M.binding.new_workspace(M.moe_backward_workspace_size(c), dev)
+    stream = torch.cuda.current_stream()
+
+    def call(with_grads):
+        M.moe_backward(c, prepared, bw, sv, dy, dx, wsb, dlogits=dlogits,
+                       grads=grads if with_grads else None)
+
+    def timed(with_grads):
+        for _ in range(args.warmup):
+            torch.cuda.nvtx.range_push("moe_backward")
+            call(with_grads)
+            torch.cuda.nvtx.range_pop()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(graph):
+            call(with_grads)
+        graph.instantiate()
+        names = graph_kernel_names(graph)
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        if M.moe_get_device_status(wsb) != 0:
+            raise RuntimeError("device status set in the backward")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps, names
+
+    clk = ClockSampler(local).__enter__()
+    t_soak = time.time()
+    ms_dgrad, _ = timed(False)
+    ms, names = timed(True)
+    t_end = time.time()
+    clk.__exit__(None, None, None)
+    touched = int((sv["counts"] > 0).sum().item())
+    hbm, tf_burst, tf_sus, peak_kind = _peaks()
+    b, f = backward_algorithmic(cfg, touched)
+    gbs = b / (ms * 1e-3) / 1e9
+    tfs = f / (ms * 1e-3) / 1e12
+    roof_ms = max(b / (hbm * 1e9), f / (tf_burst * 1e12)) * 1e3
+    # the weight-gradient kernel alone, by difference: the fp32 gradients
+    # written and its operands read once per expert
+    w_el = 3 * H * (touched * I + Is) + E * H
+    # operands per routed row: [da | du] (2I) and X (H), dO (H) and h (I); per
+    # token: the shared expert's (3 I_s + 2H when present) and the router's
+    # bf16 dlogits (E) and x (H)
+    wg_bytes = 4 * w_el + 2 * (T * k * (3 * I + 2 * H) + T * ((3 * Is + 2 * H if Is else 0) + E + H))
+    wg_ms = ms - ms_dgrad
+    clocks = clk.summary(t_soak, t_end)
+    line = {
+        "metric": "MoE layer bwd (dgrad + wgrad) tokens/s at 1 B200",
+        "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 (fp32 accumulation, fp32 weight gradients)",
+        "data": "synthetic (seeded normal inputs, dy and random-init weights of the workload)",
+        "config": dict(_workload(cfg, "inputs larger than L2: %.0f MB of bf16 weights read and "
+                                 "%.0f MB of fp32 gradients written per step"
+                                 % (2 * w_el / 1e6, 4 * w_el / 1e6)),
+                       workload=f"routed MoE layer backward, {cfg.name}",
+                       launch="CUDA graph of one moe_backward call", parallelism="replicas1"),
+        "roofline": {"bound": "hbm" if b / (hbm * 1e9) >= f / (tf_burst * 1e12) else "tensor",
+                     "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": roof_ms / ms,
+                     "kernel": "the whole moe_backward call (its roofline time = max of "
+                               "algorithmic bytes / HBM and FLOPs / bf16 peak)",
+                     "algorithmic_bytes": b, "flops": f, "tensor_tflops": tfs,
+                     "roofline_ms": roof_ms, "traffic": None,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, bf16_tflops)"},
+        "wgrad": {"ms": wg_ms, "bytes": wg_bytes, "gbs": wg_bytes / (wg_ms * 1e-3) / 1e9,
+                  "frac": wg_bytes / (wg_ms * 1e-3) / 1e9 / hbm,
+                  "how": "moe_backward with weight gradients minus without"},
+        "dgrad_ms": ms_dgrad,
+        "cpu_baseline": None,
+        "gpu_launches": len(names) * args.steps if names is not None else None,
+        "gpu_launches_per_step": names,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"], "samples": clocks["samples"]},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_ours(args, cfg):
     import mixture_experts_layer_grouped_b200 as M
     ws_n, rank, local = _dist()
@@ -563,6 +711,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="profiling only: run this many tokens (with --experts, keeps the "
                          "token-side kernels at full size while the weights stay small)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward of the bf16 layer (moe_backward) instead")
     ap.add_argument("--soak-s", type=float, default=1.5,
                     help="untimed graph replays before the timed region (clock sampling)")
     args = ap.parse_args()
@@ -572,7 +722,9 @@ def main():
         cfg = cfg.scaled(E=args.experts, T=t, name=f"{cfg.name}_E{args.experts}_T{t}")
     elif args.tokens:
         cfg = cfg.scaled(T=args.tokens, name=f"{cfg.name}_T{args.tokens}")
-    if args.impl == "reference":
+    if args.backward:
+        run_backward(args, cfg)
+    elif args.impl == "reference":
         run_reference(args, cfg)
     else:
         run_ours(args, cfg)

@@ -1,6 +1,7 @@
 /*
- * moe_b200.h -- C ABI of the routed Mixture-of-Experts layer forward on one
- * NVIDIA B200 (sm_100a).
+ * moe_b200.h -- C ABI of the routed Mixture-of-Experts layer on one NVIDIA
+ * B200 (sm_100a): the forward, and the backward of the bf16 layer
+ * (moe_backward, at the end).
  *
  * The layer (TransformerEngine PR "DeepSeekV3Layer: full MoE transformer
  * layer", Description, DeepSeekV3MoE bullet): a sigmoid router with an
@@ -294,6 +295,109 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w,
                        const void* w_router, const float* bias,
                        const void* x, void* y, int32_t xy_on_host,
                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward of the bf16 layer: the gradients of a loss L with respect to the
+ * layer's input, router and weights, given dy = dL/dy (TransformerEngine PR
+ * "DeepSeekV3Layer", Performance, "fused grouped MLP" row: the dGLU backward,
+ * the dgrad and wgrad grouped GEMMs, and the router's gradient).  With
+ * y[t] = sum_j w[t,j] O[row(t,j)] + shared(x[t]), w the gates of moe_route
+ * and O = h W2_e^T, h = silu(a) u, a = X W1_e^T, u = X W3_e^T:
+ *   dO[row(t,j)] = w[t,j] dy[t];   dgate[t,j] = <dy[t], O[row(t,j)]>;
+ *   dh = dO W2_e;  da = dh u silu'(a);  du = dh silu(a),
+ *     silu'(a) = s (1 + a (1 - s)), s = sigmoid(a);
+ *   dX = da W1_e + du W3_e (per expert-major row), and the same for the shared
+ *     expert on x with dO = dy;
+ *   gates w_j = rsf s_j / S (s = sigmoid(logit), S = sum over the selected
+ *     experts): dlogit_j = rsf (g_j / S - sum_i g_i s_i / S^2) s_j (1 - s_j)
+ *     for selected experts, 0 elsewhere (the selection and the bias are
+ *     piecewise constant and get no gradient), g = dgate;
+ *   dx[t] = sum_j dX[row(t,j)] + dx_shared[t] + (dlogits W_r)[t];
+ *   dW1_e = da^T X, dW3_e = du^T X, dW2_e = dO^T h over the expert's rows;
+ *   dWs1 = da_s^T x, dWs3 = du_s^T x, dWs2 = dy^T h_s;  dW_r = dlogits^T x.
+ * The bf16 roundings of the forward (h, O) are read as the identity.  a, u
+ * and h are recomputed from the saved rows (bf16), the intermediate gradients
+ * are stored as bf16 (dO, dh, da, du, dX, and the bf16 copy of dlogits the
+ * dx and dW_r contractions read), every contraction accumulates in fp32.
+ * Only dtype MOE_BF16 (MOE_ERR_UNSUPPORTED otherwise).
+ *
+ * Transposed weight copies the dgrad contractions read, tile-major as in
+ * moe_weights (element (r, k) of an R x K matrix at bf16 offset
+ * ((r/128)*(K/64) + k/64)*8192 + (r%128)*64 + k%64):
+ *   w2t  [E*I rows, H]: rows e*I + i hold W2_e[:, i];
+ *   w13t [E*H rows, 2I]: row e*H + h holds [W1_e[:, h] | W3_e[:, h]];
+ *   ws2t [I_shared rows, H]: Ws2^T (unused when I_shared == 0);
+ *   wdt  [H rows, Kd]: row h holds [Ws1[:, h] | Ws3[:, h] | W_r[:, h] | 0],
+ *        Kd = 2 I_shared + E rounded up to a multiple of 64.
+ * Sizes in bytes from moe_backward_weights_size; written by
+ * moe_prepare_backward_weights from row-major bf16 sources:
+ *   which == 0: routed experts e_begin .. e_begin+e_count-1, w1 and w3
+ *               [e_count, I, H], w2 [e_count, H, I] (w_router unused);
+ *   which == 1: the shared expert and the router (e_begin 0, e_count 1):
+ *               w1, w3 [I_shared, H], w2 [H, I_shared] (NULL when
+ *               I_shared == 0), w_router [E, H].
+ */
+typedef struct moe_bwd_weights {
+  void* w2t; void* w13t; void* ws2t; void* wdt;
+} moe_bwd_weights;
+
+typedef struct moe_bwd_weight_sizes {
+  size_t w2t, w13t, ws2t, wdt;
+} moe_bwd_weight_sizes;
+
+moe_status moe_backward_weights_size(const moe_config* cfg, moe_bwd_weight_sizes* sizes);
+moe_status moe_prepare_backward_weights(const moe_config* cfg, int32_t which, int32_t e_begin,
+                                        int32_t e_count, const void* w1, const void* w3,
+                                        const void* w2, const void* w_router,
+                                        const moe_bwd_weights* dst, void* stream);
+
+/*
+ * What the forward saved, as the step calls wrote it: x [T, H] bf16; rows
+ * [r_cap, H] bf16 (moe_permute's dst_rows, pad rows zero); logits [T, E]
+ * (moe_route's logits_out); topk_idx, topk_w (moe_route); counts, offsets,
+ * row_token, token_row (moe_permute); out_rows [r_cap, H] bf16
+ * (moe_grouped_mlp).
+ */
+typedef struct moe_fwd_saved {
+  const void* x;
+  const void* rows;
+  const float* logits;
+  const int32_t* topk_idx;
+  const float* topk_w;
+  const int32_t* counts;
+  const int32_t* offsets;
+  const int32_t* row_token;
+  const int32_t* token_row;
+  const void* out_rows;
+} moe_fwd_saved;
+
+/*
+ * Weight gradients, fp32 row-major, written (not accumulated) by moe_backward:
+ * dw1, dw3 [E, I, H]; dw2 [E, H, I]; dws1, dws3 [I_shared, H]; dws2
+ * [H, I_shared]; dw_router [E, H].  Any field may be NULL: that gradient is
+ * not computed.  The routed ones need pad_multiple % 64 == 0
+ * (MOE_ERR_UNSUPPORTED otherwise): each expert's rows are read in 64-row
+ * steps and the segment pads supply the zeros past its last row.
+ */
+typedef struct moe_weight_grads {
+  float* dw1; float* dw3; float* dw2;
+  float* dws1; float* dws3; float* dws2;
+  float* dw_router;
+} moe_weight_grads;
+
+/*
+ * dy [T, H] bf16 -> dx [T, H] bf16; dlogits [T, E] fp32 and dgate [T, top_k]
+ * fp32 (either may be NULL); dw (NULL: no weight gradient).  w: the forward's
+ * prepared weights (their W1, W3 and, for the shared expert, Ws1 and Ws3 are
+ * read for the recomputation of a and u); wb: moe_prepare_backward_weights's
+ * copies.  workspace: moe_backward_workspace_size bytes, its first 4 bytes
+ * (the status word) zero before the first call, as for moe_workspace_size.
+ */
+moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes);
+moe_status moe_backward(const moe_config* cfg, const moe_weights* w, const moe_bwd_weights* wb,
+                        const moe_fwd_saved* saved, const void* dy, void* dx, float* dlogits,
+                        float* dgate, const moe_weight_grads* dw, void* workspace,
+                        size_t workspace_bytes, void* stream);
 
 /*
  * Reads (and clears) the device status word at the start of `workspace`.

@@ -1,4 +1,5 @@
-"""Routed Mixture-of-Experts layer forward on one B200 (sm_100a).
+"""Routed Mixture-of-Experts layer on one B200 (sm_100a): the forward, and the
+backward of the bf16 layer.
 
 A thin ctypes binding over ``libmoe_b200.so``: the functions below marshal
 torch tensors into device pointers and call the C ABI of include/moe_b200.h
@@ -29,4 +30,12 @@ from .binding import (  # noqa: F401
     prepare_weights,
     allocate_prepared_weights,
     MoELayer,
+    MoEBwdWeights,
+    MoEFwdSaved,
+    MoEWeightGrads,
+    moe_backward_weights_size,
+    moe_prepare_backward_weights,
+    prepare_backward_weights,
+    moe_backward_workspace_size,
+    moe_backward,
 )

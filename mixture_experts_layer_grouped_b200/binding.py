@@ -54,6 +54,29 @@ class MoEWeightSizes(ctypes.Structure):
                  "ws2_scales", "w_globals", "ws_globals")]
 
 
+class MoEBwdWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w2t", "w13t", "ws2t", "wdt")]
+
+
+class MoEBwdWeightSizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("w2t", "w13t", "ws2t", "wdt")]
+
+
+_SAVED_FIELDS = ("x", "rows", "logits", "topk_idx", "topk_w", "counts", "offsets",
+                 "row_token", "token_row", "out_rows")
+
+
+class MoEFwdSaved(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _SAVED_FIELDS]
+
+
+_GRAD_FIELDS = ("dw1", "dw3", "dw2", "dws1", "dws3", "dws2", "dw_router")
+
+
+class MoEWeightGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _GRAD_FIELDS]
+
+
 def config_from_shape(s, T=None) -> MoEConfig:
     """MoEConfig from any object with the layer's shape attributes."""
     return MoEConfig(
@@ -99,6 +122,17 @@ def lib() -> ctypes.CDLL:
                               _VP], ctypes.c_int),
             "moe_prepare_weights": ([_CFG, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _VP,
                                      _VP, _VP, ctypes.POINTER(MoEWeights), _VP], ctypes.c_int),
+            "moe_backward_weights_size": ([_CFG, ctypes.POINTER(MoEBwdWeightSizes)],
+                                          ctypes.c_int),
+            "moe_prepare_backward_weights": ([_CFG, ctypes.c_int32, ctypes.c_int32,
+                                              ctypes.c_int32, _VP, _VP, _VP, _VP,
+                                              ctypes.POINTER(MoEBwdWeights), _VP], ctypes.c_int),
+            "moe_backward_workspace_size": ([_CFG, ctypes.POINTER(ctypes.c_size_t)],
+                                            ctypes.c_int),
+            "moe_backward": ([_CFG, ctypes.POINTER(MoEWeights), ctypes.POINTER(MoEBwdWeights),
+                              ctypes.POINTER(MoEFwdSaved), _VP, _VP, _VP, _VP,
+                              ctypes.POINTER(MoEWeightGrads), _VP, ctypes.c_size_t, _VP],
+                             ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -296,6 +330,78 @@ def moe_get_device_status(workspace, stream=None) -> int:
     _check("moe_get_device_status",
            lib().moe_get_device_status(_p(workspace), ctypes.byref(v), _stream(stream)))
     return v.value
+
+
+def moe_backward_weights_size(cfg: MoEConfig) -> dict:
+    v = MoEBwdWeightSizes()
+    _check("moe_backward_weights_size",
+           lib().moe_backward_weights_size(ctypes.byref(cfg), ctypes.byref(v)))
+    return {n: getattr(v, n) for n, _ in MoEBwdWeightSizes._fields_}
+
+
+def moe_prepare_backward_weights(cfg, which, e_begin, e_count, w1, w3, w2, w_router, dst,
+                                 stream=None):
+    """Transposed tile-major weight copies for the backward (dst: a dict of
+    uint8 buffers keyed w2t, w13t, ws2t, wdt, or an MoEBwdWeights)."""
+    st = dst if isinstance(dst, MoEBwdWeights) else MoEBwdWeights(
+        **{k: (dst[k].data_ptr() if dst.get(k) is not None else None)
+           for k, _ in MoEBwdWeights._fields_})
+    bf = torch.bfloat16
+    _check("moe_prepare_backward_weights", lib().moe_prepare_backward_weights(
+        ctypes.byref(cfg), which, e_begin, e_count, _p(_cuda(w1, bf, "w1")),
+        _p(_cuda(w3, bf, "w3")), _p(_cuda(w2, bf, "w2")),
+        _p(_cuda(w_router, bf, "w_router")), ctypes.byref(st), _stream(stream)))
+
+
+def prepare_backward_weights(cfg, raw: dict, w_router, stream=None) -> dict:
+    """Allocate and fill the backward's weight copies from the row-major bf16
+    tensors in ``raw`` (keys w1, w3, w2 and, with a shared expert, ws1, ws3,
+    ws2) and the router weight [E, H]."""
+    sz = moe_backward_weights_size(cfg)
+    dev = raw["w1"].device
+    out = {k: (torch.empty(v, dtype=torch.uint8, device=dev) if v else None)
+           for k, v in sz.items()}
+    moe_prepare_backward_weights(cfg, 0, 0, cfg.E, raw["w1"], raw["w3"], raw["w2"], None, out,
+                                 stream)
+    moe_prepare_backward_weights(cfg, 1, 0, 1, raw.get("ws1"), raw.get("ws3"), raw.get("ws2"),
+                                 w_router, out, stream)
+    return out
+
+
+def moe_backward_workspace_size(cfg: MoEConfig) -> int:
+    n = ctypes.c_size_t()
+    _check("moe_backward_workspace_size",
+           lib().moe_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def moe_backward(cfg, weights, bwd_weights, saved: dict, dy, dx, workspace, dlogits=None,
+                 dgate=None, grads=None, stream=None):
+    """Gradients of the bf16 layer.  ``saved`` maps the moe_fwd_saved field
+    names (x, rows, logits, topk_idx, topk_w, counts, offsets, row_token,
+    token_row, out_rows) to the forward's tensors; ``grads`` (optional) maps
+    dw1, dw3, dw2, dws1, dws3, dws2, dw_router to fp32 output tensors."""
+    ws = weights if isinstance(weights, MoEWeights) else weights_struct(weights)
+    bw = bwd_weights if isinstance(bwd_weights, MoEBwdWeights) else MoEBwdWeights(
+        **{k: (bwd_weights[k].data_ptr() if bwd_weights.get(k) is not None else None)
+           for k, _ in MoEBwdWeights._fields_})
+    types = {"x": torch.bfloat16, "rows": torch.bfloat16, "logits": torch.float32,
+             "topk_idx": torch.int32, "topk_w": torch.float32, "counts": torch.int32,
+             "offsets": torch.int32, "row_token": torch.int32, "token_row": torch.int32,
+             "out_rows": torch.bfloat16}
+    sv = MoEFwdSaved(**{k: _cuda(saved[k], types[k], k).data_ptr() for k in _SAVED_FIELDS})
+    gr = None
+    if grads is not None:
+        gr = MoEWeightGrads(**{k: (_cuda(grads[k], torch.float32, k).data_ptr()
+                                   if grads.get(k) is not None else None)
+                               for k in _GRAD_FIELDS})
+    bf = torch.bfloat16
+    _check("moe_backward", lib().moe_backward(
+        ctypes.byref(cfg), ctypes.byref(ws), ctypes.byref(bw), ctypes.byref(sv),
+        _p(_cuda(dy, bf, "dy")), _p(_cuda(dx, bf, "dx")),
+        _p(_cuda(dlogits, torch.float32, "dlogits")), _p(_cuda(dgate, torch.float32, "dgate")),
+        ctypes.byref(gr) if gr is not None else None, _p(workspace), workspace.numel(),
+        _stream(stream)))
 
 
 class MoELayer:

@@ -1,0 +1,231 @@
+// Backward of the bf16 layer (input gradients): the memory-bound steps.  The
+// contractions run on the grouped GEMM (grouped_gemm.cuh, fc2 mode) with
+// transposed weight copies; see moe_backward in moe_api.cu.
+//
+//   combine backward:  dO[row(t, j)] = bf16(w[t, j] * dy[t]),
+//                      g[t, j] = <dy[t], O[row(t, j)]>  (fp32),
+//   gate backward:     w_j = rsf * s_j / S over the selected experts, so
+//                      ds_j = rsf * (g_j / S - sum_i g_i s_i / S^2),
+//                      dlogit_j = ds_j * s_j * (1 - s_j), zero elsewhere;
+//   SwiGLU backward:   h = silu(a) * u:  da = dh * u * silu'(a),
+//                      du = dh * silu(a), silu'(a) = s (1 + a (1 - s)), s = sigmoid(a).
+// (TransformerEngine PR "DeepSeekV3Layer", Performance, "fused grouped MLP"
+//  row: dGLU backward and the grouped GEMMs of the backward pass.)
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+struct CombineBwdArgs {
+  const __nv_bfloat16* dy;        // [T, H]
+  const __nv_bfloat16* out_rows;  // [r_cap, H]: the forward's fc2 rows (O)
+  const int32_t* token_row;       // [T * k]
+  const int32_t* topk_idx;        // [T * k]
+  const float* topk_w;            // [T * k]
+  const float* logits;            // [T, E]: the forward's router logits
+  __nv_bfloat16* dO;              // [r_cap, H]
+  float* dgate;                   // [T * k]
+  float* dlogits;                 // [T, E] or null
+  __nv_bfloat16* dense_b;         // [T, ld_b]: dlogits as bf16 at column col_b, zeros to ld_b
+  int T, H, k, E, col_b, ld_b;
+  float rsf;
+};
+
+// A block per token (256 threads, 8 bf16 columns per thread and vector).
+template <int K>
+__global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float red[8][32];
+  __shared__ float g_s[32];
+  const int t = blockIdx.x;
+  const int kk = K > 0 ? K : a.k;
+  int rows[K > 0 ? K : 32];
+  float ws[K > 0 ? K : 32], part[K > 0 ? K : 32];
+#pragma unroll
+  for (int j = 0; j < (K > 0 ? K : 32); ++j) {
+    if (j < kk) {
+      rows[j] = __ldg(a.token_row + static_cast<int64_t>(t) * kk + j);
+      ws[j] = __ldg(a.topk_w + static_cast<int64_t>(t) * kk + j);
+    }
+    part[j] = 0.f;
+  }
+  const int vecs = a.H >> 3;
+  const uint4* dy4 = reinterpret_cast<const uint4*>(a.dy + static_cast<int64_t>(t) * a.H);
+  for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
+    const uint4 draw = __ldg(dy4 + v);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&draw);
+    float d[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(d2[q]);
+      d[2 * q] = f.x;
+      d[2 * q + 1] = f.y;
+    }
+#pragma unroll
+    for (int j = 0; j < (K > 0 ? K : 32); ++j) {
+      if (j >= kk || rows[j] < 0) continue;
+      const uint4 oraw = __ldg(reinterpret_cast<const uint4*>(
+                                   a.out_rows + static_cast<int64_t>(rows[j]) * a.H) + v);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&oraw);
+      float s = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(o2[q]);
+        s = fmaf(d[2 * q], f.x, s);
+        s = fmaf(d[2 * q + 1], f.y, s);
+      }
+      part[j] += s;
+      uint4 o;
+      __nv_bfloat162* w2 = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        w2[q] = __floats2bfloat162_rn(ws[j] * d[2 * q], ws[j] * d[2 * q + 1]);
+      reinterpret_cast<uint4*>(a.dO + static_cast<int64_t>(rows[j]) * a.H)[v] = o;
+    }
+  }
+  // g[t, j]: block sum of the per-thread partial dot products
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int j = 0; j < (K > 0 ? K : 32); ++j) {
+    if (j >= kk) break;
+    float v = part[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp][j] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < kk) {
+    float v = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) v += red[w][threadIdx.x];
+    g_s[threadIdx.x] = v;
+    a.dgate[static_cast<int64_t>(t) * kk + threadIdx.x] = v;
+  }
+  __syncthreads();
+  // gate backward: the token's dlogits (fp32, optional) and their bf16 copy in
+  // the dense GEMM's operand row, zeros elsewhere
+  const float* lg = a.logits + static_cast<int64_t>(t) * a.E;
+  float S = 0.f, gs = 0.f;
+  for (int j = 0; j < kk; ++j) {
+    const int e = __ldg(a.topk_idx + static_cast<int64_t>(t) * kk + j);
+    if (e < 0 || e >= a.E) continue;
+    const float s = 1.0f / (1.0f + expf(-__ldg(lg + e)));
+    S += s;
+    gs += g_s[j] * s;
+  }
+  __nv_bfloat16* brow = a.dense_b + static_cast<int64_t>(t) * a.ld_b;
+  for (int e = threadIdx.x; e < a.ld_b - a.col_b; e += blockDim.x) {
+    float dl = 0.f;
+    if (e < a.E) {
+      for (int j = 0; j < kk; ++j) {
+        if (__ldg(a.topk_idx + static_cast<int64_t>(t) * kk + j) != e) continue;
+        const float s = 1.0f / (1.0f + expf(-__ldg(lg + e)));
+        const float ds = a.rsf * (g_s[j] / S - gs / (S * S));
+        dl = ds * s * (1.0f - s);
+      }
+      if (a.dlogits) a.dlogits[static_cast<int64_t>(t) * a.E + e] = dl;
+    }
+    brow[a.col_b + e] = __float2bfloat16_rn(dl);
+  }
+}
+
+// SwiGLU backward for rows of [rows, n] (a, u: the recomputed fc1 outputs, dh:
+// the gradient of h), written as [da | du] at the start of rows of out_ld
+// elements, and h = bf16(silu(a) u) itself into h_out [rows, n] when h_out is
+// given (the fc2 weight gradient's operand).  Rows with row_token < 0 (segment
+// pads) are zeroed; a null row_token means every row holds a token, and
+// rows_used (when given) bounds the rows.  Eight columns per thread and vector.
+__global__ void __launch_bounds__(256) swiglu_backward_kernel(
+    const __nv_bfloat16* __restrict__ a_in, const __nv_bfloat16* __restrict__ u_in,
+    const __nv_bfloat16* __restrict__ dh, __nv_bfloat16* __restrict__ dz, int64_t out_ld,
+    __nv_bfloat16* __restrict__ h_out, const int32_t* __restrict__ row_token,
+    const int32_t* __restrict__ rows_used, int64_t rows, int n) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t nrows = rows_used ? __ldg(rows_used) : rows;
+  const int vpr = n >> 3;
+  const int64_t total = nrows * vpr;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / vpr;
+    const int v = static_cast<int>(i - r * vpr);
+    uint4 da4 = make_uint4(0, 0, 0, 0), du4 = make_uint4(0, 0, 0, 0), h4 = make_uint4(0, 0, 0, 0);
+    if (!row_token || __ldg(row_token + r) >= 0) {
+      const int64_t off = r * n + v * 8;
+      const uint4 ar = __ldg(reinterpret_cast<const uint4*>(a_in + off));
+      const uint4 ur = __ldg(reinterpret_cast<const uint4*>(u_in + off));
+      const uint4 hr = __ldg(reinterpret_cast<const uint4*>(dh + off));
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ar);
+      const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&ur);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hr);
+      __nv_bfloat162* da2 = reinterpret_cast<__nv_bfloat162*>(&da4);
+      __nv_bfloat162* du2 = reinterpret_cast<__nv_bfloat162*>(&du4);
+      __nv_bfloat162* hh2 = reinterpret_cast<__nv_bfloat162*>(&h4);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 av = __bfloat1622float2(a2[q]), uv = __bfloat1622float2(u2[q]),
+                     hv = __bfloat1622float2(h2[q]);
+        const float s0 = 1.0f / (1.0f + expf(-av.x)), s1 = 1.0f / (1.0f + expf(-av.y));
+        const float g0 = s0 * (1.0f + av.x * (1.0f - s0)), g1 = s1 * (1.0f + av.y * (1.0f - s1));
+        da2[q] = __floats2bfloat162_rn(hv.x * uv.x * g0, hv.y * uv.y * g1);
+        du2[q] = __floats2bfloat162_rn(hv.x * av.x * s0, hv.y * av.y * s1);
+        hh2[q] = __floats2bfloat162_rn(av.x * s0 * uv.x, av.y * s1 * uv.y);
+      }
+    }
+    if (h_out) reinterpret_cast<uint4*>(h_out + r * n)[v] = h4;
+    __nv_bfloat16* out = dz + r * out_ld;
+    reinterpret_cast<uint4*>(out)[v] = da4;
+    reinterpret_cast<uint4*>(out + n)[v] = du4;
+  }
+}
+
+// Weight preparation for the backward: a tile-major matrix (tiles of 128 rows
+// x 64 columns, as the forward's prepared weights) whose element (r, c) is
+// taken, transposed, from up to three row-major bf16 sources laid side by side
+// along c: for the segment s holding column c, source row c - start_s and
+// source column r % rows_per_group of group r / rows_per_group (each group a
+// block of group_stride elements).  Columns past the last segment are zero.
+// A block moves one 64 x 64 square through shared memory, so that both the
+// reads (along a source row) and the writes (along a tile row) are coalesced.
+struct TransposeSeg {
+  const __nv_bfloat16* src;
+  int64_t group_stride;  // elements between consecutive groups (experts)
+  int ld;                // source row length (elements)
+  int start, width;      // destination columns [start, start + width)
+};
+struct TransposeArgs {
+  TransposeSeg seg[3];
+  int nseg;
+  __nv_bfloat16* dst;
+  int64_t rows;          // destination rows (a multiple of 128)
+  int cols;              // destination columns (a multiple of 64)
+  int rows_per_group;    // a multiple of 64
+};
+
+__global__ void __launch_bounds__(256) transpose_tiles_kernel(TransposeArgs a) {
+  __shared__ __nv_bfloat16 sq[64][66];
+  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 64;
+  const int c0 = blockIdx.y * 64;
+  const int64_t grp = r0 / a.rows_per_group, rl0 = r0 - grp * a.rows_per_group;
+  for (int cc = ty; cc < 64; cc += 4) {
+    const int c = c0 + cc;
+    __nv_bfloat16 v = __float2bfloat16_rn(0.f);
+    for (int s = 0; s < a.nseg; ++s) {
+      const TransposeSeg& g = a.seg[s];
+      if (c >= g.start && c < g.start + g.width)
+        v = g.src[grp * g.group_stride + static_cast<int64_t>(c - g.start) * g.ld + rl0 + tx];
+    }
+    sq[cc][tx] = v;
+  }
+  __syncthreads();
+  for (int rr = ty; rr < 64; rr += 4) {
+    const int64_t r = r0 + rr;
+    const int c = c0 + tx;
+    const int64_t tile = (r >> 7) * (a.cols >> 6) + (c >> 6);
+    a.dst[tile * 8192 + (r & 127) * 64 + (c & 63)] = sq[tx][rr];
+  }
+}
+
+}  // namespace moe

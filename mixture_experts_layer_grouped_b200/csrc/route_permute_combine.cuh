@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(256) permute_gather_row_kernel(GatherArgs a) {
 struct CombineArgs {
   const __nv_bfloat16* out_rows;  // [r_cap, H]
   const int32_t* token_row;       // [T*k]
-  const float* topk_w;            // [T*k]
+  const float* topk_w;            // [T*k], or null: every weight 1 (the backward's dx sum)
   const __nv_bfloat16* shared;    // [T, H] or null
   __nv_bfloat16* y;               // [T, H]
   int T, H, k;
@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   for (int j = 0; j < (K > 0 ? K : 32); ++j) {
     if (j < kk) {
       rows[j] = __ldg(a.token_row + static_cast<int64_t>(t) * kk + j);
-      ws[j] = __ldg(a.topk_w + static_cast<int64_t>(t) * kk + j);
+      ws[j] = a.topk_w ? __ldg(a.topk_w + static_cast<int64_t>(t) * kk + j) : 1.0f;
     }
   }
   const int vecs = a.H >> 3;

@@ -8,6 +8,7 @@ can consume the same bytes without sharing any code of the method.
 from .configs import CONFIGS, MoEShape, get_config  # noqa: F401
 from .inputs import (  # noqa: F401
     gen_x,
+    gen_dy,
     gen_router,
     gen_expert_weights,
     gen_shared_weights,

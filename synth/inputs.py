@@ -15,7 +15,9 @@ Distributions (std, not variance):
   ``skew_factor``;
 * bias ~ U(-bias_range, bias_range), fp32;
 * W1, W3 [I, H] ~ N(0, 1/sqrt(H)); W2 [H, I] ~ N(0, 1/sqrt(I)); the shared
-  expert uses the same rule with I_shared.
+  expert uses the same rule with I_shared;
+* dy (the gradient of a loss with respect to the layer's output, the
+  backward's input) ~ N(0, 1).
 
 All matrices are returned in bf16 (bias in fp32), row-major.
 """
@@ -48,6 +50,10 @@ def _normal(shape, std, g, device) -> torch.Tensor:
 def gen_x(cfg: MoEShape, device="cpu", T: int = None) -> torch.Tensor:
     T = cfg.T if T is None else T
     return _normal((T, cfg.H), 1.0, _gen(cfg, "x", 0, device), device)
+
+
+def gen_dy(cfg: MoEShape, device="cpu") -> torch.Tensor:
+    return _normal((cfg.T, cfg.H), 1.0, _gen(cfg, "dy", 0, device), device)
 
 
 def gen_router(cfg: MoEShape, device="cpu"):

@@ -126,3 +126,49 @@ def test_block_scaled_needs_64_row_padding(M):
     s = s.scaled(pad_multiple=64)
     assert M.lib().moe_prepared_weights_size(ctypes.byref(M.config_from_shape(s)),
                                              ctypes.byref(sizes)) == 0
+
+
+def test_backward_rejects_bad_arguments(M):
+    """moe_backward validates on the host: bf16 only, the saved forward state
+    and weight copies required, routed weight gradients only with 64-row
+    segment pads, and a workspace of moe_backward_workspace_size bytes."""
+    lib = M.lib()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    s = synth.get_config("tiny_bf16_T64").scaled(pad_multiple=64)
+    c = M.config_from_shape(s)
+    nb = M.moe_backward_workspace_size(c)
+    w = M.MoEWeights(w1=fake, w3=fake, w2=fake)
+    bw = M.MoEBwdWeights(w2t=fake, w13t=fake, wdt=fake)
+    sv = M.MoEFwdSaved(**{k: fake for k, _ in M.MoEFwdSaved._fields_})
+    gr = M.MoEWeightGrads(dw1=fake)
+
+    def call(cfg=c, bw=bw, sv=sv, gr=gr, ws=nb, dy=fake):
+        return lib.moe_backward(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(bw),
+                                ctypes.byref(sv), dy, fake, None, None,
+                                ctypes.byref(gr) if gr is not None else None, fake, ws, None)
+
+    assert call(ws=16) == 3
+    assert call(dy=None) == 1
+    assert call(bw=M.MoEBwdWeights(w2t=fake, w13t=fake)) == 1
+    sv_missing = M.MoEFwdSaved(**{k: fake for k, _ in M.MoEFwdSaved._fields_ if k != "logits"})
+    assert call(sv=sv_missing) == 1
+    # shared-expert gradients of a layer without one
+    assert call(gr=M.MoEWeightGrads(dws1=fake)) == 1
+    # routed weight gradients need segment pads of a multiple of 64 rows
+    c8 = M.config_from_shape(s.scaled(pad_multiple=8))
+    nb8 = M.moe_backward_workspace_size(c8)
+    assert call(cfg=c8, ws=nb8) == 2
+    # block-scaled layers have no backward
+    cq = M.config_from_shape(synth.get_config("dsv3_mxfp8_shared_T4096"))
+    assert call(cfg=cq) == 2
+    n = ctypes.c_size_t()
+    assert lib.moe_backward_workspace_size(ctypes.byref(cq), ctypes.byref(n)) == 2
+
+
+def test_backward_weight_sizes(M):
+    s = synth.get_config("mid_bf16_shared_T2048")
+    sz = M.moe_backward_weights_size(M.config_from_shape(s))
+    assert sz["w2t"] == s.E * s.I * s.H * 2
+    assert sz["w13t"] == s.E * s.H * 2 * s.I * 2
+    assert sz["ws2t"] == s.I_shared * s.H * 2
+    assert sz["wdt"] == s.H * (2 * s.I_shared + 64) * 2  # E = 64 columns of W_r^T

@@ -1,0 +1,157 @@
+"""Parity of the backward of the bf16 layer (moe_backward) with the oracle's
+backward: dx, dgate, dlogits and every weight gradient, on the same seeded
+inputs and the same routing (TransformerEngine PR "DeepSeekV3Layer",
+Performance, "fused grouped MLP" row: the dGLU backward, the dgrad and wgrad
+grouped GEMMs, and the router's gradient).
+
+Tolerance: relative Frobenius error <= 1e-2 for every result, the bar the
+forward's bf16 output meets.  The GPU stores six intermediates as bf16 on the
+way to dx (dO, a, u, dh, da/du, dX) and accumulates each contraction in fp32;
+each bf16 store adds a relative error of at most 2^-9 per element, about
+1.1e-3 rms, so the expected error of dx is near sqrt(6) * 1.1e-3 = 2.7e-3.
+The weight gradients take two bf16 operands each (about 1.6e-3 rms).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from moe_testlib import f64, near_ties, rel_frob, run_steps, weights_dict
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+SHAPES = {
+    # several 128 x 256 wgrad tiles per expert, shared expert, top_k 4
+    "small_shared": synth.MoEShape(
+        name="bwd_small_shared", T=256, H=512, I=256, E=16, n_group=4, topk_group=2, top_k=4,
+        rsf=2.5, I_shared=256, dtype="bf16", pad_multiple=64, router_std=0.02),
+    # ragged T, H not a multiple of the 256-column wgrad tile, E = 32 (a
+    # partly empty router tile), top_k 6, skewed load
+    "ragged_k6": synth.MoEShape(
+        name="bwd_ragged_k6", T=333, H=384, I=128, E=32, n_group=8, topk_group=4, top_k=6,
+        rsf=2.5, I_shared=0, dtype="bf16", pad_multiple=64, router_std=0.02, skew_experts=4,
+        skew_factor=3.0),
+    # decode-sized: most experts get no token (zero gradients), 64-token tiles
+    "decode_shared": synth.MoEShape(
+        name="bwd_decode_shared", T=8, H=256, I=128, E=16, n_group=4, topk_group=2, top_k=4,
+        rsf=2.5, I_shared=128, dtype="bf16", pad_multiple=128, router_std=0.02),
+}
+
+
+def _run(cfg, grads=True):
+    import mixture_experts_layer_grouped_b200 as M
+    d = synth.gen_all(cfg, "cuda")
+    s = run_steps(cfg, d)
+    assert s["status"] == 0
+    c = M.config_from_shape(cfg)
+    prepared = M.prepare_weights(c, weights_dict(d))
+    bwd_w = M.prepare_backward_weights(c, weights_dict(d), d["w_router"])
+    dy = synth.gen_dy(cfg, "cuda")
+    saved = {k: s[k] for k in ("rows", "logits", "topk_idx", "topk_w", "counts", "offsets",
+                               "row_token", "token_row", "out_rows")}
+    saved["x"] = d["x"]
+    T, H, E, I, Is, k = cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k
+    dx = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    dlogits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    dgate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    g = None
+    if grads:
+        f32 = dict(dtype=torch.float32, device="cuda")
+        g = {"dw1": torch.full((E, I, H), float("nan"), **f32),
+             "dw3": torch.full((E, I, H), float("nan"), **f32),
+             "dw2": torch.full((E, H, I), float("nan"), **f32),
+             "dw_router": torch.full((E, H), float("nan"), **f32)}
+        if Is:
+            g["dws1"] = torch.full((Is, H), float("nan"), **f32)
+            g["dws3"] = torch.full((Is, H), float("nan"), **f32)
+            g["dws2"] = torch.full((H, Is), float("nan"), **f32)
+    ws = M.binding.new_workspace(M.moe_backward_workspace_size(c), "cuda")
+    M.moe_backward(c, prepared, bwd_w, saved, dy, dx, ws, dlogits=dlogits, dgate=dgate,
+                   grads=g)
+    torch.cuda.synchronize()
+    assert M.moe_get_device_status(ws) == 0
+    return d, s, dy, dx, dlogits, dgate, g
+
+
+def _oracle(cfg, d, s, dy, weight_grads=True):
+    h = {k: f64(v) for k, v in d.items()}
+    shared = (h["ws1"], h["ws3"], h["ws2"]) if cfg.I_shared else None
+    b = O.backward(cfg, h["x"], h["w_router"], h["bias"], h["w1"], h["w3"], h["w2"], f64(dy),
+                   shared=shared, logits=f64(s["logits"]), weight_grads=weight_grads)
+    # the oracle routes on the GPU's fp32 logits; a near-tie could still
+    # choose differently in fp64, which would make the gradients incomparable:
+    # the selections must agree on every token (near-ties included)
+    # the selections must agree on every token, near-ties included; a near-tie
+    # may order two selected experts differently, and then the oracle's dgate
+    # row is put in the GPU's order
+    r = b["fwd"]["route"]
+    gi = s["topk_idx"].cpu().numpy()
+    same = np.all(np.sort(r["idx"], axis=1) == np.sort(gi, axis=1), axis=1)
+    assert same.all(), ("routing differs", np.nonzero(~same)[0], near_ties(r).sum())
+    for t in np.nonzero(np.any(r["idx"] != gi, axis=1))[0]:
+        pos = {int(e): j for j, e in enumerate(r["idx"][t])}
+        b["dgate"][t] = b["dgate"][t][[pos[int(e)] for e in gi[t]]]
+    return b
+
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_backward_matches_oracle(name):
+    cfg = SHAPES[name]
+    d, s, dy, dx, dlogits, dgate, g = _run(cfg)
+    b = _oracle(cfg, d, s, dy)
+    errs = {"dx": rel_frob(f64(dx), b["dx"]),
+            "dgate": rel_frob(f64(dgate), b["dgate"]),
+            "dlogits": rel_frob(f64(dlogits), b["dlogits"])}
+    counts = s["counts"].cpu().numpy()
+    for key in ("dw1", "dw3", "dw2"):
+        got = f64(g[key])
+        assert np.isfinite(got).all(), key
+        ref = np.stack([b[key][e] for e in range(cfg.E)])
+        errs[key] = rel_frob(got, ref)
+        # experts no token picked: exactly zero
+        assert not got[counts == 0].any(), key
+    errs["dw_router"] = rel_frob(f64(g["dw_router"]), b["dw_router"])
+    if cfg.I_shared:
+        for key in ("dws1", "dws3", "dws2"):
+            errs[key] = rel_frob(f64(g[key]), b[key])
+    print(name, {k: f"{v:.2e}" for k, v in errs.items()})
+    for key, v in errs.items():
+        assert v <= TOL, (key, v)
+
+
+def test_backward_without_weight_grads_matches():
+    """dw = NULL: only dx, dlogits and dgate; the same values as with it."""
+    cfg = SHAPES["small_shared"]
+    _, _, _, dx0, dl0, dg0, _ = _run(cfg, grads=True)
+    _, _, _, dx1, dl1, dg1, _ = _run(cfg, grads=False)
+    assert torch.equal(dx0, dx1) and torch.equal(dl0, dl1) and torch.equal(dg0, dg1)
+
+
+def test_backward_mid_size():
+    """The mid bf16 layer with a shared expert (T=2048, H=2048, I=1024,
+    E=64, top_k=6, skewed router), with 64-row segment pads: dx, dgate and
+    dlogits over every token, the weight gradients of the most and least
+    loaded experts and of the shared expert and the router."""
+    cfg = synth.get_config("mid_bf16_shared_T2048").scaled(pad_multiple=64)
+    d, s, dy, dx, dlogits, dgate, g = _run(cfg)
+    counts = s["counts"].cpu().numpy()
+    pick = [int(np.argmax(counts)), int(np.argmin(np.where(counts > 0, counts, 1 << 30)))]
+    b = _oracle(cfg, d, s, dy, weight_grads=pick)
+    errs = {"dx": rel_frob(f64(dx), b["dx"]),
+            "dgate": rel_frob(f64(dgate), b["dgate"]),
+            "dlogits": rel_frob(f64(dlogits), b["dlogits"]),
+            "dw_router": rel_frob(f64(g["dw_router"]), b["dw_router"])}
+    for key in ("dws1", "dws3", "dws2"):
+        errs[key] = rel_frob(f64(g[key]), b[key])
+    for e in pick:
+        for key in ("dw1", "dw3", "dw2"):
+            errs[f"{key}[{e}]"] = rel_frob(f64(g[key][e]), b[key][e])
+    for key in ("dw1", "dw3", "dw2"):
+        assert torch.isfinite(g[key]).all(), key
+    print("mid", {k: f"{v:.2e}" for k, v in errs.items()})
+    for key, v in errs.items():
+        assert v <= TOL, (key, v)
