@@ -219,6 +219,21 @@ def time_oracle(cfg, n_tokens, steps, warmup, device):
     return n_tokens / dt, dt, len(W)
 
 
+def time_oracle_backward(cfg, n_tokens, device):
+    """The oracle's backward with every weight gradient (fp64, as it stands)
+    on an n_tokens sample; returns (tokens/s, seconds per pass, experts
+    touched)."""
+    from oracle import moe_oracle as O
+    xh, wrh, bh, W, sh = oracle_sample(cfg, n_tokens, device)
+    dyh = O.from_bf16(synth.gen_dy(cfg, device)[:n_tokens])
+    scfg = cfg.scaled(T=n_tokens)
+    w = [(lambda e, k=k: O.from_bf16(W[e][k])) for k in range(3)]
+    t0 = time.perf_counter()
+    O.backward(scfg, xh, wrh, bh, w[0], w[1], w[2], dyh, shared=sh, weight_grads=sorted(W))
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt, len(W)
+
+
 def _oracle_note(cfg, n_tokens, n_experts):
     return (f"oracle forward (fp64; weights of the {n_experts} experts the sample touches "
             f"quantized inside each pass, as the oracle stands) on the first {n_tokens} tokens of "
@@ -448,6 +463,17 @@ def run_backward(args, cfg):
     wg_bytes = 4 * w_el + 2 * (T * k * (3 * I + 2 * H) + T * ((3 * Is + 2 * H if Is else 0) + E + H))
     wg_ms = ms - ms_dgrad
     clocks = clk.summary(t_soak, t_end)
+    cpu = None
+    if not args.no_cpu_baseline:
+        n = args.ref_tokens
+        if not n:  # about 15 s of host work: a one-token pass sizes the sample
+            _, t1, _ = time_oracle_backward(cfg, 1, dev)
+            n = max(1, min(32, int(15.0 / max(t1, 1e-6))))
+        tps, dt, ne = time_oracle_backward(cfg, n, dev)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": _host_cores(), "kind": "oracle",
+               "sample": f"oracle backward (fp64, every weight gradient of the {ne} experts "
+                         f"the sample touches) on the first {n} tokens of the {cfg.name} "
+                         f"batch, one pass of {dt:.1f} s"}
     line = {
         "metric": "MoE layer bwd (dgrad + wgrad) tokens/s at 1 B200",
         "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
@@ -470,7 +496,7 @@ def run_backward(args, cfg):
                   "frac": wg_bytes / (wg_ms * 1e-3) / 1e9 / hbm,
                   "how": "moe_backward with weight gradients minus without"},
         "dgrad_ms": ms_dgrad,
-        "cpu_baseline": None,
+        "cpu_baseline": cpu,
         "gpu_launches": len(names) * args.steps if names is not None else None,
         "gpu_launches_per_step": names,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
@@ -666,10 +692,11 @@ def run_ours(args, cfg):
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
                      "frac": achieved_gbs / hbm,
                      "traffic": traffic,
-                     "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
-                                        "fc1 and fc2 launches, per algorithmic weight byte, "
-                                        f"captured on kernel source {src_hash}, x this call's "
-                                        "algorithmic bytes" if traffic is not None else
+                     "traffic_source": ("estimate, not counted in this run: the ratio of "
+                                        "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
+                                        "the fc1 and fc2 launches to their algorithmic weight "
+                                        f"bytes, captured on kernel source {src_hash}, x this "
+                                        "call's algorithmic bytes" if traffic is not None else
                                         f"no ncu capture of kernel source {src_hash}"),
                      "kernel": "moe_grouped_mlp (fc1+SwiGLU and fc2 tcgen05 kernels)",
                      "algorithmic_bytes_per_launch": wbytes, "ms_per_launch": mlp_ms,
