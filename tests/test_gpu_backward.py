@@ -155,3 +155,101 @@ def test_backward_mid_size():
     print("mid", {k: f"{v:.2e}" for k, v in errs.items()})
     for key, v in errs.items():
         assert v <= TOL, (key, v)
+
+
+@pytest.mark.slow
+def test_backward_full_size_dsv4_bf16():
+    """The DeepSeek-V4 routed-expert geometry in bf16 (T=4096, H=4096, I=2048,
+    E=256, top-6) with 64-row pads, every token on the GPU.  The oracle routes
+    from its own fp64 logits and checks, away from near-ties: the weight
+    gradients of the most loaded expert and two seeded others (each from that
+    expert's own rows and dO = w * dy), and dx, dgate and dlogits of eight
+    tokens (their backward on their own: a token's gradients depend on no other
+    token)."""
+    import mixture_experts_layer_grouped_b200 as M
+    from moe_testlib import check_routing, pick_tokens, prepare_streaming
+    cfg = synth.get_config("dsv4_bf16_T4096").scaled(pad_multiple=64)
+    c = M.config_from_shape(cfg)
+    T, H, E, I, k = cfg.T, cfg.H, cfg.E, cfg.I, cfg.top_k
+    x = synth.gen_x(cfg, "cuda")
+    w_r, bias = synth.gen_router(cfg, "cuda")
+    prepared = prepare_streaming(M, cfg)
+    bw = {n: (torch.empty(v, dtype=torch.uint8, device="cuda") if v else None)
+          for n, v in M.moe_backward_weights_size(c).items()}
+    for e in range(E):
+        M.moe_prepare_backward_weights(c, 0, e, 1, *synth.gen_expert_weights(cfg, e, "cuda"),
+                                       None, bw)
+    M.moe_prepare_backward_weights(c, 1, 0, 1, None, None, None, w_r, bw)
+    nbytes, r_cap = M.moe_workspace_size(c)
+    ws = M.binding.new_workspace(nbytes, "cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    sv = {"x": x, "logits": torch.empty(T, E, dtype=torch.float32, device="cuda"),
+          "topk_idx": torch.empty(T, k, **i32),
+          "topk_w": torch.empty(T, k, dtype=torch.float32, device="cuda"),
+          "counts": torch.empty(E, **i32), "offsets": torch.empty(E + 1, **i32),
+          "row_token": torch.empty(r_cap, **i32), "token_row": torch.empty(T * k, **i32),
+          "rows": torch.empty(r_cap, H, dtype=torch.bfloat16, device="cuda"),
+          "out_rows": torch.empty(r_cap, H, dtype=torch.bfloat16, device="cuda")}
+    M.moe_route(c, x, w_r, bias, sv["topk_idx"], sv["topk_w"], ws, logits_out=sv["logits"])
+    M.moe_permute(c, sv["topk_idx"], x, sv["counts"], sv["offsets"], sv["row_token"],
+                  sv["token_row"], sv["rows"], ws)
+    M.moe_grouped_mlp(c, prepared, sv["rows"], sv["counts"], sv["offsets"], sv["out_rows"], ws)
+    dy = synth.gen_dy(cfg, "cuda")
+    dx = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    dlogits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    dgate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    g = {"dw1": torch.empty(E, I, H, **f32), "dw3": torch.empty(E, I, H, **f32),
+         "dw2": torch.empty(E, H, I, **f32), "dw_router": torch.empty(E, H, **f32)}
+    wsb = M.binding.new_workspace(M.moe_backward_workspace_size(c), "cuda")
+    M.moe_backward(c, prepared, bw, sv, dy, dx, wsb, dlogits=dlogits, dgate=dgate, grads=g)
+    torch.cuda.synchronize()
+    assert M.moe_get_device_status(ws) == 0 and M.moe_get_device_status(wsb) == 0
+
+    # the oracle's own routing
+    xh, dyh = f64(x), f64(dy)
+    wrh, bh = f64(w_r), f64(bias)
+    logits = O.router_logits(xh, wrh)
+    r = O.route(logits, bh, cfg.n_group, cfg.topk_group, cfg.top_k, cfg.rsf)
+    idx_gpu = sv["topk_idx"].cpu().numpy()
+    keep, bad = check_routing(r, idx_gpu, sv["topk_w"].cpu().numpy(), cfg.rsf)
+    assert not bad, f"{len(bad)} tokens routed differently"
+    bad_e = set(r["idx"][~keep].ravel().tolist()) | set(idx_gpu[~keep].ravel().tolist())
+    weights = {}
+
+    def expert(e):
+        if e not in weights:
+            weights[e] = tuple(f64(t) for t in synth.gen_expert_weights(cfg, e, "cuda"))
+        return weights[e]
+
+    # whole experts: weight gradients from the expert's own rows
+    counts = np.bincount(r["idx"].ravel(), minlength=E)
+    touched = [e for e in np.nonzero(counts)[0].tolist() if e not in bad_e]
+    hot = max(touched, key=lambda e: (counts[e], -e))
+    rng = np.random.default_rng(0)
+    rest = [e for e in touched if e != hot]
+    errs = {}
+    for e in [hot] + sorted(rng.choice(rest, 2, replace=False).tolist()):
+        tok, j = np.nonzero(r["idx"] == e)          # ascending tokens
+        Xe = xh[tok]
+        dOe = r["w"][tok, j][:, None] * dyh[tok]
+        W1, W3, W2 = expert(e)
+        _, mid = O.expert_backward(Xe, W1, W3, W2, dOe)
+        d1, d3, d2 = O.expert_weight_grads(Xe, dOe, mid)
+        errs[f"dw1[{e}]"] = rel_frob(f64(g["dw1"][e]), d1)
+        errs[f"dw3[{e}]"] = rel_frob(f64(g["dw3"][e]), d3)
+        errs[f"dw2[{e}]"] = rel_frob(f64(g["dw2"][e]), d2)
+    # eight tokens end to end, sharing experts where they can
+    cand = [t for t in np.nonzero(keep)[0].tolist() if not (set(r["idx"][t]) & bad_e)]
+    toks, _ = pick_tokens(r["idx"], cand, [hot], 8, E, seed=1)
+    toks = np.sort(toks)
+    scfg = cfg.scaled(T=len(toks))
+    w = [(lambda e, q=q: expert(e)[q]) for q in range(3)]
+    b = O.backward(scfg, xh[toks], wrh, bh, w[0], w[1], w[2], dyh[toks], logits=logits[toks])
+    assert np.array_equal(b["fwd"]["route"]["idx"], r["idx"][toks])
+    errs["dx"] = rel_frob(f64(dx)[toks], b["dx"])
+    errs["dgate"] = rel_frob(f64(dgate)[toks], b["dgate"])
+    errs["dlogits"] = rel_frob(f64(dlogits)[toks], b["dlogits"])
+    print("dsv4 bf16 backward", {kk: f"{v:.2e}" for kk, v in errs.items()})
+    for kk, v in errs.items():
+        assert v <= TOL, (kk, v)
