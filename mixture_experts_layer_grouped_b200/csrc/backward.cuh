@@ -1,6 +1,9 @@
-// Backward of the bf16 layer (input gradients): the memory-bound steps.  The
-// contractions run on the grouped GEMM (grouped_gemm.cuh, fc2 mode) with
-// transposed weight copies; see moe_backward in moe_api.cu.
+// Backward of the bf16 layer: the combine and gate backward, the SwiGLU
+// backward, and the weight copies the dgrad contractions read.  The
+// contractions run on the grouped GEMM (grouped_gemm.cuh: fc2 mode with
+// transposed weight copies, and fc1's backward form, which recomputes a and u
+// and stores both); the weight gradients in wgrad.cuh; see moe_backward in
+// moe_api.cu.
 //
 //   combine backward:  dO[row(t, j)] = bf16(w[t, j] * dy[t]),
 //                      g[t, j] = <dy[t], O[row(t, j)]>  (fp32),
@@ -32,29 +35,30 @@ struct CombineBwdArgs {
   float rsf;
 };
 
-// A block per token (256 threads, 8 bf16 columns per thread and vector).
+// A warp per token, eight tokens per 256-thread block: each lane takes every
+// 32nd 16-byte vector of the row (8 bf16 columns), two vectors per round with
+// all their loads issued first, and the k dot products are reduced across the
+// warp with shuffles (every lane ends with all of them).
 template <int K>
 __global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float red[8][32];
-  __shared__ float g_s[32];
-  const int t = blockIdx.x;
+  constexpr int KM = K > 0 ? K : 32;
+  const int lane = threadIdx.x & 31;
+  const int t = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  if (t >= a.T) return;
   const int kk = K > 0 ? K : a.k;
-  int rows[K > 0 ? K : 32];
-  float ws[K > 0 ? K : 32], part[K > 0 ? K : 32];
+  int rows[KM];
+  float ws[KM], part[KM];
 #pragma unroll
-  for (int j = 0; j < (K > 0 ? K : 32); ++j) {
-    if (j < kk) {
-      rows[j] = __ldg(a.token_row + static_cast<int64_t>(t) * kk + j);
-      ws[j] = __ldg(a.topk_w + static_cast<int64_t>(t) * kk + j);
-    }
+  for (int j = 0; j < KM; ++j) {
+    rows[j] = j < kk ? __ldg(a.token_row + static_cast<int64_t>(t) * kk + j) : -1;
+    ws[j] = j < kk ? __ldg(a.topk_w + static_cast<int64_t>(t) * kk + j) : 0.f;
     part[j] = 0.f;
   }
   const int vecs = a.H >> 3;
   const uint4* dy4 = reinterpret_cast<const uint4*>(a.dy + static_cast<int64_t>(t) * a.H);
-  for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
-    const uint4 draw = __ldg(dy4 + v);
+  auto body = [&](int v, const uint4& draw, const uint4 (&o)[KM]) {
     const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&draw);
     float d[8];
 #pragma unroll
@@ -64,65 +68,69 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a)
       d[2 * q + 1] = f.y;
     }
 #pragma unroll
-    for (int j = 0; j < (K > 0 ? K : 32); ++j) {
+    for (int j = 0; j < KM; ++j) {
       if (j >= kk || rows[j] < 0) continue;
-      const uint4 oraw = __ldg(reinterpret_cast<const uint4*>(
-                                   a.out_rows + static_cast<int64_t>(rows[j]) * a.H) + v);
-      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&oraw);
-      float s = 0.f;
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o[j]);
+      float sdot = 0.f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 f = __bfloat1622float2(o2[q]);
-        s = fmaf(d[2 * q], f.x, s);
-        s = fmaf(d[2 * q + 1], f.y, s);
+        sdot = fmaf(d[2 * q], f.x, sdot);
+        sdot = fmaf(d[2 * q + 1], f.y, sdot);
       }
-      part[j] += s;
-      uint4 o;
-      __nv_bfloat162* w2 = reinterpret_cast<__nv_bfloat162*>(&o);
+      part[j] += sdot;
+      uint4 w;
+      __nv_bfloat162* w2 = reinterpret_cast<__nv_bfloat162*>(&w);
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         w2[q] = __floats2bfloat162_rn(ws[j] * d[2 * q], ws[j] * d[2 * q + 1]);
-      reinterpret_cast<uint4*>(a.dO + static_cast<int64_t>(rows[j]) * a.H)[v] = o;
+      reinterpret_cast<uint4*>(a.dO + static_cast<int64_t>(rows[j]) * a.H)[v] = w;
     }
-  }
-  // g[t, j]: block sum of the per-thread partial dot products
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  };
+  for (int v = lane; v < vecs; v += 32) {
+    const uint4 draw = __ldg(dy4 + v);
+    uint4 o[KM];
 #pragma unroll
-  for (int j = 0; j < (K > 0 ? K : 32); ++j) {
+    for (int j = 0; j < KM; ++j)
+      if (j < kk && rows[j] >= 0)
+        o[j] = __ldg(reinterpret_cast<const uint4*>(a.out_rows + static_cast<int64_t>(rows[j]) * a.H) + v);
+    body(v, draw, o);
+  }
+  // g[t, j]: every lane ends with the warp's sums
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
     if (j >= kk) break;
-    float v = part[j];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[warp][j] = v;
+    for (int off = 16; off > 0; off >>= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], off);
   }
-  __syncthreads();
-  if (threadIdx.x < kk) {
-    float v = 0.f;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) v += red[w][threadIdx.x];
-    g_s[threadIdx.x] = v;
-    a.dgate[static_cast<int64_t>(t) * kk + threadIdx.x] = v;
-  }
-  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < KM; ++j)
+    if (j < kk && lane == j) a.dgate[static_cast<int64_t>(t) * kk + j] = part[j];
   // gate backward: the token's dlogits (fp32, optional) and their bf16 copy in
   // the dense GEMM's operand row, zeros elsewhere
   const float* lg = a.logits + static_cast<int64_t>(t) * a.E;
+  const int32_t* ti = a.topk_idx + static_cast<int64_t>(t) * kk;
   float S = 0.f, gs = 0.f;
-  for (int j = 0; j < kk; ++j) {
-    const int e = __ldg(a.topk_idx + static_cast<int64_t>(t) * kk + j);
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    if (j >= kk) break;
+    const int e = __ldg(ti + j);
     if (e < 0 || e >= a.E) continue;
-    const float s = 1.0f / (1.0f + expf(-__ldg(lg + e)));
-    S += s;
-    gs += g_s[j] * s;
+    const float sg = 1.0f / (1.0f + expf(-__ldg(lg + e)));
+    S += sg;
+    gs += part[j] * sg;
   }
   __nv_bfloat16* brow = a.dense_b + static_cast<int64_t>(t) * a.ld_b;
-  for (int e = threadIdx.x; e < a.ld_b - a.col_b; e += blockDim.x) {
+  for (int e = lane; e < a.ld_b - a.col_b; e += 32) {
     float dl = 0.f;
     if (e < a.E) {
-      for (int j = 0; j < kk; ++j) {
-        if (__ldg(a.topk_idx + static_cast<int64_t>(t) * kk + j) != e) continue;
-        const float s = 1.0f / (1.0f + expf(-__ldg(lg + e)));
-        const float ds = a.rsf * (g_s[j] / S - gs / (S * S));
-        dl = ds * s * (1.0f - s);
+#pragma unroll
+      for (int j = 0; j < KM; ++j) {
+        if (j >= kk) break;
+        if (__ldg(ti + j) != e) continue;
+        const float sg = 1.0f / (1.0f + expf(-__ldg(lg + e)));
+        const float ds = a.rsf * (part[j] / S - gs / (S * S));
+        dl = ds * sg * (1.0f - sg);
       }
       if (a.dlogits) a.dlogits[static_cast<int64_t>(t) * a.E + e] = dl;
     }
@@ -130,15 +138,16 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a)
   }
 }
 
-// SwiGLU backward for rows of [rows, n] (a, u: the recomputed fc1 outputs, dh:
-// the gradient of h), written as [da | du] at the start of rows of out_ld
-// elements, and h = bf16(silu(a) u) itself into h_out [rows, n] when h_out is
-// given (the fc2 weight gradient's operand).  Rows with row_token < 0 (segment
-// pads) are zeroed; a null row_token means every row holds a token, and
-// rows_used (when given) bounds the rows.  Eight columns per thread and vector.
+// SwiGLU backward in place: row r of z holds [a | u] (n columns each, row
+// length ld), the fc1 outputs recomputed by the backward form of the fc1
+// kernel; with dh [rows, n] it becomes [da | du], and h = bf16(silu(a) u) goes
+// to h_out [rows, n] when h_out is given (the fc2 weight gradient's operand).
+// Rows with row_token < 0 (segment pads) are zeroed in z and h_out; a null
+// row_token means every row holds a token, and rows_used (when given) bounds the
+// rows.  Eight columns per thread and vector; each thread reads its a, u, dh
+// before writing the same places.
 __global__ void __launch_bounds__(256) swiglu_backward_kernel(
-    const __nv_bfloat16* __restrict__ a_in, const __nv_bfloat16* __restrict__ u_in,
-    const __nv_bfloat16* __restrict__ dh, __nv_bfloat16* __restrict__ dz, int64_t out_ld,
+    __nv_bfloat16* __restrict__ z, int64_t ld, const __nv_bfloat16* __restrict__ dh,
     __nv_bfloat16* __restrict__ h_out, const int32_t* __restrict__ row_token,
     const int32_t* __restrict__ rows_used, int64_t rows, int n) {
   pdl_wait();
@@ -151,32 +160,31 @@ __global__ void __launch_bounds__(256) swiglu_backward_kernel(
     const int64_t r = i / vpr;
     const int v = static_cast<int>(i - r * vpr);
     uint4 da4 = make_uint4(0, 0, 0, 0), du4 = make_uint4(0, 0, 0, 0), h4 = make_uint4(0, 0, 0, 0);
+    uint4* za = reinterpret_cast<uint4*>(z + r * ld) + v;
+    uint4* zu = reinterpret_cast<uint4*>(z + r * ld + n) + v;
     if (!row_token || __ldg(row_token + r) >= 0) {
-      const int64_t off = r * n + v * 8;
-      const uint4 ar = __ldg(reinterpret_cast<const uint4*>(a_in + off));
-      const uint4 ur = __ldg(reinterpret_cast<const uint4*>(u_in + off));
-      const uint4 hr = __ldg(reinterpret_cast<const uint4*>(dh + off));
+      const uint4 ar = *za, ur = *zu;
+      const uint4 hr = __ldg(reinterpret_cast<const uint4*>(dh + r * n) + v);
       const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ar);
       const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&ur);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hr);
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&hr);
       __nv_bfloat162* da2 = reinterpret_cast<__nv_bfloat162*>(&da4);
       __nv_bfloat162* du2 = reinterpret_cast<__nv_bfloat162*>(&du4);
       __nv_bfloat162* hh2 = reinterpret_cast<__nv_bfloat162*>(&h4);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 av = __bfloat1622float2(a2[q]), uv = __bfloat1622float2(u2[q]),
-                     hv = __bfloat1622float2(h2[q]);
+                     gv = __bfloat1622float2(g2[q]);
         const float s0 = 1.0f / (1.0f + expf(-av.x)), s1 = 1.0f / (1.0f + expf(-av.y));
-        const float g0 = s0 * (1.0f + av.x * (1.0f - s0)), g1 = s1 * (1.0f + av.y * (1.0f - s1));
-        da2[q] = __floats2bfloat162_rn(hv.x * uv.x * g0, hv.y * uv.y * g1);
-        du2[q] = __floats2bfloat162_rn(hv.x * av.x * s0, hv.y * av.y * s1);
+        const float d0 = s0 * (1.0f + av.x * (1.0f - s0)), d1 = s1 * (1.0f + av.y * (1.0f - s1));
+        da2[q] = __floats2bfloat162_rn(gv.x * uv.x * d0, gv.y * uv.y * d1);
+        du2[q] = __floats2bfloat162_rn(gv.x * av.x * s0, gv.y * av.y * s1);
         hh2[q] = __floats2bfloat162_rn(av.x * s0 * uv.x, av.y * s1 * uv.y);
       }
     }
+    *za = da4;
+    *zu = du4;
     if (h_out) reinterpret_cast<uint4*>(h_out + r * n)[v] = h4;
-    __nv_bfloat16* out = dz + r * out_ld;
-    reinterpret_cast<uint4*>(out)[v] = da4;
-    reinterpret_cast<uint4*>(out + n)[v] = du4;
   }
 }
 

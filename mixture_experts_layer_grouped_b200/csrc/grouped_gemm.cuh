@@ -112,6 +112,9 @@ struct GemmParams {
   // dynamic tile order (null: CTA i takes tiles i, i + grid, ...): the next
   // tile index is claimed from this zeroed counter
   int32_t* unit_counter;
+  // backward form of fc1 (the BWD kernel): per group, the column of `out` where
+  // u's features start (a at the feature's own column)
+  int32_t bwd_u_col[2];
 };
 
 constexpr int pow2_at_least(int v) {
@@ -449,10 +452,13 @@ __device__ __forceinline__ void sf_copies_mxf8(uint32_t sf_a0, uint32_t sf_a1, u
 // over both CTAs' shared memory (cta_group::2), each CTA loads its own 128
 // weight rows and half of the tile's token rows, and the loads of both count
 // on rank 0's full barrier.
-template <int MODE, int TILE_N, int DT, bool PAIR = false>
+// BWD (fc1, bf16 only): the backward's recomputation of a = X W1^T and
+// u = X W3^T, both stored (see the fc2-shaped epilogue branch).
+template <int MODE, int TILE_N, int DT, bool PAIR = false, bool BWD = false>
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
     const __grid_constant__ GemmParams p) {
   using C = GemmCfg<MODE, TILE_N, DT, PAIR>;
+  static_assert(!BWD || (MODE == kFc1 && DT == kBF16), "the backward form is bf16 fc1");
   static_assert(!PAIR || MODE != kRouter, "CTA pairs serve fc1 and fc2");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -887,7 +893,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
       if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
       float hmax = 0.f;  // fc1 NVFP4: amax of this warp's bf16 h values
-      if constexpr (MODE == kFc1 && DT != kMXF8) {
+      if constexpr (MODE == kFc1 && DT != kMXF8 && !BWD) {
         // h of this warp's chunks (32 tokens each) goes from TMEM straight into
         // registers as bf16 pairs, the accumulator is released, and only then
         // are the rows staged and stored: the next tile's MMAs wait for the
@@ -960,19 +966,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
         }
         signal_chunk(p, t, lane);
         if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
-      } else if constexpr (MODE == kFc2 || (MODE == kFc1 && DT == kMXF8)) {
+      } else if constexpr (MODE == kFc2 || (MODE == kFc1 && DT == kMXF8) || BWD) {
         // As above: TMEM -> registers (packed bf16), release the accumulator,
         // then stage and store.  fc2 keeps both 128-feature halves of its chunks
         // (128 registers for 256-token tiles, which therefore read 16 columns
         // at a time: 16 raw registers live instead of 64, within the 168 a
-        // thread gets); MXFP8 fc1 keeps h, quantized after the release.
+        // thread gets); MXFP8 fc1 keeps h, quantized after the release.  The
+        // backward form of fc1 stores its two accumulators, a and u, as the two
+        // halves: a at the feature's column of `out`, u bwd_u_col further.
+        constexpr bool TWO = (MODE == kFc2) || BWD;
         constexpr int NCH = (TILE_N + 63) / 64;
-        constexpr int NH = (MODE == kFc2) ? 2 : 1;
+        constexpr int NH = TWO ? 2 : 1;
         uint32_t hp[NCH][NH][16];
 #pragma unroll
         for (int i = 0; i < NCH; ++i) {
           const int c0 = member * 32 + 64 * i;
-          if (MODE == kFc2 && TILE_N > 192 && c0 < t.n_tok) {
+          if (TWO && TILE_N > 192 && c0 < t.n_tok) {
 #pragma unroll
             for (int q = 0; q < 2 * NH; ++q) {  // (half, 16-column part)
               uint32_t r[16];
@@ -990,7 +999,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              if (MODE == kFc2) {
+              if (TWO) {
                 hp[i][0][j >> 1] = bf16x2_bits(__uint_as_float(r0[j]) * alpha,
                                                __uint_as_float(r0[j + 1]) * alpha);
                 hp[i][NH - 1][j >> 1] = bf16x2_bits(__uint_as_float(r1[j]) * alpha,
@@ -1013,13 +1022,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
           const int c0 = member * 32 + 64 * i;
           if (c0 >= t.n_tok) continue;
           const int rows_here = min(32, t.n_tok - c0);
-          if constexpr (MODE == kFc2) {
+          if constexpr (TWO) {
             __nv_bfloat16* out = static_cast<__nv_bfloat16*>(G.out);
             const uint4* s4 = reinterpret_cast<const uint4*>(my_stg);
             uint16_t* s16 = reinterpret_cast<uint16_t*>(my_stg);
 #pragma unroll
             for (int half = 0; half < NH; ++half) {
-              const int f0 = f_base + half * kBM;
+              const int f0 = f_base + half * (BWD ? p.bwd_u_col[t.grp] : kBM);
+              const bool fvalid = (BWD ? f_base : f0) < G.a_valid_rows;
 #pragma unroll
               for (int j = 0; j < 32; j += 2) {
                 s16[j * 32 + lane] = static_cast<uint16_t>(hp[i][half][j >> 1] & 0xFFFFu);
@@ -1030,7 +1040,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(
               for (int it = 0; it < 4; ++it) {
                 const int c = it * 32 + lane;
                 const int j = c >> 2, part = c & 3;
-                if (j < rows_here && f0 < G.a_valid_rows)
+                if (j < rows_here && fvalid)
                   *reinterpret_cast<uint4*>(out + static_cast<int64_t>(t.row0 + c0 + j) *
                                                       G.out_ld + f0 + part * 8) = s4[j * 4 + part];
               }

@@ -338,10 +338,10 @@ int sm_count() {
 
 // One persistent CTA per SM, or (PAIR) one two-CTA cluster per SM pair, as
 // many as can be resident at once, capped by the number of tiles.
-template <int MODE, int TILE_N, int DT, bool PAIR = false>
+template <int MODE, int TILE_N, int DT, bool PAIR = false, bool BWD = false>
 moe_status launch_gemm(const GemmParams& p, int max_units, cudaStream_t s) {
   using C = GemmCfg<MODE, TILE_N, DT, PAIR>;
-  auto kern = grouped_gemm_kernel<MODE, TILE_N, DT, PAIR>;
+  auto kern = grouped_gemm_kernel<MODE, TILE_N, DT, PAIR, BWD>;
   MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
   if (!PAIR) {
     int grid = sm_count();
@@ -872,7 +872,7 @@ int64_t dense_bwd_cols(const moe_config& c) {
 }
 
 struct BwdLayout {
-  size_t status, dO, a, u, dh, dz, h, dX, a_s, u_s, dh_s, h_s, dense_b, dx_dense, dgate, total;
+  size_t status, dO, dh, dz, h, dX, dh_s, h_s, dense_b, dx_dense, dgate, total;
   int32_t r_cap;
 };
 
@@ -883,14 +883,10 @@ BwdLayout bwd_layout(const moe_config& c) {
   size_t o = 0;
   L.status = o; o = align_up(o + 4);
   L.dO = o; o = align_up(o + R * H * 2);
-  L.a = o; o = align_up(o + R * I * 2);
-  L.u = o; o = align_up(o + R * I * 2);
   L.dh = o; o = align_up(o + R * I * 2);
   L.dz = o; o = align_up(o + R * 2 * I * 2);
   L.h = o; o = align_up(o + R * I * 2);
   L.dX = o; o = align_up(o + R * H * 2);
-  L.a_s = o; o = align_up(o + T * Is * 2);
-  L.u_s = o; o = align_up(o + T * Is * 2);
   L.dh_s = o; o = align_up(o + T * Is * 2);
   L.h_s = o; o = align_up(o + T * Is * 2);
   L.dense_b = o; o = align_up(o + T * static_cast<size_t>(dense_bwd_cols(c)) * 2);
@@ -942,6 +938,49 @@ moe_status rows_gemm(const moe_config& c, const void* a_r, int M_r, int K_r, con
   const int dense_chunks = (c.T + TILE_N - 1) / TILE_N;
   const int units = max_chunks * p.g[0].n_slabs + (dense ? dense_chunks * p.g[1].n_slabs : 0);
   return launch_gemm<kFc2, TILE_N, kBF16, PAIR>(p, units, s);
+}
+
+// a = X W1^T and u = X W3^T recomputed in one pass of the fc1 kernel's
+// backward form (W1 and W3 slabs per stage, as in the forward), stored as
+// [a | u] rows of dz (row length 2I); the shared expert's on x into the first
+// 2 I_shared columns of the dense operand (row length Kd).
+template <int TILE_N, bool PAIR>
+moe_status fc1_recompute(const moe_config& c, const moe_weights& w, const void* rows,
+                         const void* x, void* dz, void* dense_b, int Kd, const int32_t* counts,
+                         const int32_t* offsets, int32_t* status, cudaStream_t s) {
+  constexpr int span = GemmCfg<kFc1, TILE_N, kBF16, PAIR>::SLAB_SPAN;
+  const int32_t r_cap = r_cap_of(c);
+  const bool sh = c.I_shared > 0;
+  const uint64_t H = c.H, I = c.I, Is = sh ? c.I_shared : 0, E = c.E;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  MOE_TRY(make_tiled_map(&p.a0[0], w.w1, E * I, H * 2));
+  MOE_TRY(make_tiled_map(&p.a1[0], w.w3, E * I, H * 2));
+  MOE_TRY(make_map(&p.b[0], rows, bf, 2, H, r_cap, H * 2, kBoxRows));
+  if (sh) {
+    MOE_TRY(make_tiled_map(&p.a0[1], w.ws1, Is, H * 2));
+    MOE_TRY(make_tiled_map(&p.a1[1], w.ws3, Is, H * 2));
+    MOE_TRY(make_map(&p.b[1], x, bf, 2, H, c.T, H * 2, kBoxRows));
+  } else {
+    p.a0[1] = p.a0[0];
+    p.a1[1] = p.a1[0];
+    p.b[1] = p.b[0];
+  }
+  p.g[0] = GemmGroup{c.I, c.I, (c.I + span - 1) / span, c.H / kBK, 1, dz, 2 * c.I, 0};
+  p.g[1] = GemmGroup{0, static_cast<int32_t>(Is), static_cast<int32_t>((Is + span - 1) / span),
+                     c.H / kBK, 1, dense_b, Kd, 0};
+  p.bwd_u_col[0] = c.I;
+  p.bwd_u_col[1] = static_cast<int32_t>(Is);
+  p.counts = counts;
+  p.offsets = offsets;
+  p.E = c.E;
+  p.dense_rows = sh ? c.T : 0;
+  p.status = status;
+  const int max_chunks = c.E + (c.T * c.top_k) / TILE_N + 1;
+  const int dense_chunks = (c.T + TILE_N - 1) / TILE_N;
+  const int units = max_chunks * p.g[0].n_slabs + (sh ? dense_chunks * p.g[1].n_slabs : 0);
+  return launch_gemm<kFc1, TILE_N, kBF16, PAIR, true>(p, units, s);
 }
 
 // One wgrad contraction as the host describes it.
@@ -1028,11 +1067,17 @@ moe_status backward_steps(const moe_config& c, const moe_weights& w, const moe_b
   cb.col_b = 2 * (sh ? Is : 0);
   cb.ld_b = Kd;
   cb.rsf = c.routed_scaling_factor;
+  const dim3 cgrid((c.T + 7) / 8);  // a warp per token
   switch (c.top_k) {
-    case 4: MOE_TRY(launch_pdl(combine_backward_kernel<4>, dim3(c.T), dim3(256), 0, s, cb)); break;
-    case 6: MOE_TRY(launch_pdl(combine_backward_kernel<6>, dim3(c.T), dim3(256), 0, s, cb)); break;
-    case 8: MOE_TRY(launch_pdl(combine_backward_kernel<8>, dim3(c.T), dim3(256), 0, s, cb)); break;
-    default: MOE_TRY(launch_pdl(combine_backward_kernel<0>, dim3(c.T), dim3(256), 0, s, cb)); break;
+    case 1: MOE_TRY(launch_pdl(combine_backward_kernel<1>, cgrid, dim3(256), 0, s, cb)); break;
+    case 2: MOE_TRY(launch_pdl(combine_backward_kernel<2>, cgrid, dim3(256), 0, s, cb)); break;
+    case 3: MOE_TRY(launch_pdl(combine_backward_kernel<3>, cgrid, dim3(256), 0, s, cb)); break;
+    case 4: MOE_TRY(launch_pdl(combine_backward_kernel<4>, cgrid, dim3(256), 0, s, cb)); break;
+    case 5: MOE_TRY(launch_pdl(combine_backward_kernel<5>, cgrid, dim3(256), 0, s, cb)); break;
+    case 7: MOE_TRY(launch_pdl(combine_backward_kernel<7>, cgrid, dim3(256), 0, s, cb)); break;
+    case 6: MOE_TRY(launch_pdl(combine_backward_kernel<6>, cgrid, dim3(256), 0, s, cb)); break;
+    case 8: MOE_TRY(launch_pdl(combine_backward_kernel<8>, cgrid, dim3(256), 0, s, cb)); break;
+    default: MOE_TRY(launch_pdl(combine_backward_kernel<0>, cgrid, dim3(256), 0, s, cb)); break;
   }
   MOE_TRY(launch_check());
   const unsigned g = static_cast<unsigned>(sm_count() * 8);
@@ -1042,33 +1087,26 @@ moe_status backward_steps(const moe_config& c, const moe_weights& w, const moe_b
                        f.row_token, f.offsets + c.E));
     MOE_TRY(launch_check());
   }
-  // a = X W1^T, u = X W3^T (recomputed from the saved rows), dh = dO W2; the
-  // shared expert's on x and dy
-  MOE_TRY((rows_gemm<TILE_N, PAIR>(c, w.w1, I, H, f.rows, b + L.a, sh ? w.ws1 : nullptr, Is, H,
-                                   f.x, b + L.a_s, f.counts, f.offsets, status, s)));
-  MOE_TRY((rows_gemm<TILE_N, PAIR>(c, w.w3, I, H, f.rows, b + L.u, sh ? w.ws3 : nullptr, Is, H,
-                                   f.x, b + L.u_s, f.counts, f.offsets, status, s)));
+  // dh = dO W2 (the shared expert's: dy Ws2)
   MOE_TRY((rows_gemm<TILE_N, PAIR>(c, wb.w2t, I, H, b + L.dO, b + L.dh, sh ? wb.ws2t : nullptr,
                                    Is, H, dy, b + L.dh_s, f.counts, f.offsets, status, s)));
-  // SwiGLU backward: [da | du] per expert-major row (and h for dW2); the shared
-  // expert's into the first 2 * I_shared columns of the dense operand
+  // [a | u] recomputed from the saved rows in one fc1 pass (the shared
+  // expert's into the dense operand), then the SwiGLU backward in place:
+  // [da | du] per expert-major row (pads zeroed) and h for dW2
+  MOE_TRY((fc1_recompute<TILE_N, PAIR>(c, w, f.rows, f.x, b + L.dz, b + L.dense_b, Kd, f.counts,
+                                       f.offsets, status, s)));
   const bool want_h = dw && dw->dw2;
-  MOE_TRY(launch_pdl(swiglu_backward_kernel, dim3(g), dim3(256), 0, s,
-                     static_cast<const __nv_bfloat16*>(bfp(L.a)),
-                     static_cast<const __nv_bfloat16*>(bfp(L.u)),
-                     static_cast<const __nv_bfloat16*>(bfp(L.dh)), bfp(L.dz),
-                     static_cast<int64_t>(2 * I), want_h ? bfp(L.h) : nullptr, f.row_token,
-                     f.offsets + c.E, static_cast<int64_t>(L.r_cap), I));
+  MOE_TRY(launch_pdl(swiglu_backward_kernel, dim3(g), dim3(256), 0, s, bfp(L.dz),
+                     static_cast<int64_t>(2 * I), static_cast<const __nv_bfloat16*>(bfp(L.dh)),
+                     want_h ? bfp(L.h) : nullptr, f.row_token, f.offsets + c.E,
+                     static_cast<int64_t>(L.r_cap), I));
   MOE_TRY(launch_check());
   if (sh) {
     const bool want_hs = dw && dw->dws2;
-    MOE_TRY(launch_pdl(swiglu_backward_kernel, dim3(g), dim3(256), 0, s,
-                       static_cast<const __nv_bfloat16*>(bfp(L.a_s)),
-                       static_cast<const __nv_bfloat16*>(bfp(L.u_s)),
-                       static_cast<const __nv_bfloat16*>(bfp(L.dh_s)), bfp(L.dense_b),
-                       static_cast<int64_t>(Kd), want_hs ? bfp(L.h_s) : nullptr,
-                       static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr),
-                       static_cast<int64_t>(c.T), Is));
+    MOE_TRY(launch_pdl(swiglu_backward_kernel, dim3(g), dim3(256), 0, s, bfp(L.dense_b),
+                       static_cast<int64_t>(Kd), static_cast<const __nv_bfloat16*>(bfp(L.dh_s)),
+                       want_hs ? bfp(L.h_s) : nullptr, static_cast<const int32_t*>(nullptr),
+                       static_cast<const int32_t*>(nullptr), static_cast<int64_t>(c.T), Is));
     MOE_TRY(launch_check());
   }
   // dX rows = [da | du] [W1; W3] (K = 2I); dense dx = [da_s | du_s | dlogits]
