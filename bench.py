@@ -276,8 +276,8 @@ TENSOR_RATIO = {"bf16": 1.0, "mxfp8": 2.0, "nvfp4": 4.0}  # nominal dense peak v
 # captured on fewer experts with the same tokens per expert; the ratio carries
 # over per touched expert.
 TRAFFIC_RATIO = {
-    "dsv4_nvfp4_prefill_T8192": (1.066, "dcc545b0947a04af"),
-    "mid_bf16_shared_T2048": (1.190, "dcc545b0947a04af"),
+    "dsv4_nvfp4_prefill_T8192": (1.066, "32a54879bb76cd88"),
+    "mid_bf16_shared_T2048": (1.191, "32a54879bb76cd88"),
     "dsv4_bf16_T4096": (1.032, "dcc545b0947a04af"),
     "dsv3_mxfp8_shared_T4096": (1.080, "dcc545b0947a04af"),
     "dsv4_mxfp8_T4096": (1.018, "dcc545b0947a04af"),
