@@ -39,6 +39,14 @@ SHAPES = {
     "decode_shared": synth.MoEShape(
         name="bwd_decode_shared", T=8, H=256, I=128, E=16, n_group=4, topk_group=2, top_k=4,
         rsf=2.5, I_shared=128, dtype="bf16", pad_multiple=128, router_std=0.02),
+    # top-8 (the DeepSeek-V3 fan-out) with a shared expert
+    "top8_shared": synth.MoEShape(
+        name="bwd_top8_shared", T=200, H=256, I=256, E=32, n_group=4, topk_group=4, top_k=8,
+        rsf=2.5, I_shared=128, dtype="bf16", pad_multiple=64, router_std=0.02),
+    # top-10: the combine kernels' generic (any top_k) form
+    "top10": synth.MoEShape(
+        name="bwd_top10", T=96, H=256, I=128, E=64, n_group=8, topk_group=4, top_k=10,
+        rsf=1.0, I_shared=0, dtype="bf16", pad_multiple=64, router_std=0.02),
 }
 
 
