@@ -36,9 +36,9 @@ struct CombineBwdArgs {
 };
 
 // A warp per token, eight tokens per 256-thread block: each lane takes every
-// 32nd 16-byte vector of the row (8 bf16 columns), two vectors per round with
-// all their loads issued first, and the k dot products are reduced across the
-// warp with shuffles (every lane ends with all of them).
+// 32nd 16-byte vector of the row (8 bf16 columns), issuing the vector's k + 1
+// loads (dy and the k fc2 rows) before its arithmetic, and the k dot products
+// are reduced across the warp with shuffles (every lane ends with all of them).
 template <int K>
 __global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a) {
   pdl_wait();
