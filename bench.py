@@ -267,7 +267,10 @@ def run_reference(args, cfg):
 # ---------------------------------------------------------------------------
 
 WEIGHT_BYTES = {"bf16": 2.0, "mxfp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}  # per element
-TENSOR_RATIO = {"bf16": 1.0, "mxfp8": 2.0, "nvfp4": 4.0}  # nominal dense peak vs bf16
+# Dense tensor peaks of the block-scaled types, TFLOP/s: library GEMMs at 8192^3
+# timed on one B200 by `bench.py --tensor-peaks` (burst); bf16 comes from the
+# driver's measurement (MEASURED_PEAKS.json).
+TENSOR_PEAK = {"mxfp8": 2834.6, "nvfp4": 6217.2}
 # DRAM bytes (read + written) of one grouped-MLP call's fc1 and fc2 launches per
 # algorithmic weight byte, from ncu dram__bytes_read.sum + dram__bytes_write.sum
 # captures, keyed by workload, each with the hash of the kernel source it was
@@ -345,6 +348,48 @@ def prepare_streaming(M, cfg, c, dev):
         M.moe_prepare_weights(c, 1, 0, 1, *synth.gen_shared_weights(cfg, dev), dst)
     torch.cuda.synchronize()
     return p
+
+
+def tensor_peaks(device="cuda"):
+    """Dense library GEMM throughput on this GPU, 8192^3, burst (50 timed calls after
+    5 untimed): bf16 (torch matmul), MXFP8 and NVFP4 (torch._scaled_mm with block
+    scales; the scale values do not change the work).  The denominators of the
+    block-scaled tensor fractions."""
+    M = N = K = 8192
+    res = {}
+
+    def timeit(fn, iters=50):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return 2 * M * N * K / (e0.elapsed_time(e1) / iters * 1e-3) / 1e12
+
+    def pad(v, m):
+        return (v + m - 1) // m * m
+
+    u8 = dict(dtype=torch.uint8, device=device)
+    x = torch.randn(M, K, device=device, dtype=torch.bfloat16)
+    y = torch.randn(K, N, device=device, dtype=torch.bfloat16)
+    res["bf16_tflops"] = timeit(lambda: x @ y)
+    a8 = torch.randn(M, K, device=device).to(torch.float8_e4m3fn)
+    b8 = torch.randn(N, K, device=device).to(torch.float8_e4m3fn).t()
+    s8a = torch.full((pad(M, 128) * pad(K // 32, 4),), 127, **u8).view(torch.float8_e8m0fnu)
+    s8b = torch.full((pad(N, 128) * pad(K // 32, 4),), 127, **u8).view(torch.float8_e8m0fnu)
+    res["mxfp8_tflops"] = timeit(lambda: torch._scaled_mm(a8, b8, s8a, s8b,
+                                                          out_dtype=torch.bfloat16))
+    a4 = torch.randint(0, 255, (M, K // 2), **u8).view(torch.float4_e2m1fn_x2)
+    b4 = torch.randint(0, 255, (N, K // 2), **u8).view(torch.float4_e2m1fn_x2).t()
+    s4a = torch.full((pad(M, 128) * pad(K // 16, 4),), 56, **u8).view(torch.float8_e4m3fn)
+    s4b = torch.full((pad(N, 128) * pad(K // 16, 4),), 56, **u8).view(torch.float8_e4m3fn)
+    res["nvfp4_tflops"] = timeit(lambda: torch._scaled_mm(a4, b4, s4a, s4b,
+                                                          out_dtype=torch.bfloat16))
+    return res
 
 
 def backward_algorithmic(cfg, touched):
@@ -656,8 +701,8 @@ def run_ours(args, cfg):
     mlp_ms = statistics.mean(steps_ms["grouped_mlp"])
     wbytes, flops = grouped_mlp_algorithmic(cfg, touched)
     hbm, tf_burst, tf_sus, peak_kind = _peaks()
-    # a contraction takes the peak of its own dtype: bf16 peak x the nominal ratio
-    tf_dtype = tf_burst * TENSOR_RATIO[cfg.dtype]
+    # a contraction takes the peak of its own dtype
+    tf_dtype = TENSOR_PEAK.get(cfg.dtype, tf_burst)
     achieved_gbs = wbytes / (mlp_ms * 1e-3) / 1e9
     lb, lf = layer_algorithmic(cfg, touched)
     roof_ms = max(lb / (hbm * 1e9), lf / (tf_dtype * 1e12)) * 1e3
@@ -702,8 +747,11 @@ def run_ours(args, cfg):
                      "algorithmic_bytes_per_launch": wbytes, "ms_per_launch": mlp_ms,
                      "tensor_tflops": flops / (mlp_ms * 1e-3) / 1e12,
                      "tensor_frac": flops / (mlp_ms * 1e-3) / 1e12 / tf_dtype,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs; bf16_tflops x "
-                                    f"{TENSOR_RATIO[cfg.dtype]:g} for {cfg.dtype})"},
+                     "tensor_peak_tflops": tf_dtype,
+                     "peak_source": (f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs; tensor: " +
+                                     ("bf16_tflops" if cfg.dtype == "bf16" else
+                                      f"{cfg.dtype} library GEMM measured by bench.py "
+                                      "--tensor-peaks") + ")")},
         "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_max,
                            "bytes": lb, "flops": lf, "experts_touched": touched},
         "step_ms": {k: statistics.mean(v) for k, v in steps_ms.items()},
@@ -738,6 +786,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="profiling only: run this many tokens (with --experts, keeps the "
                          "token-side kernels at full size while the weights stay small)")
+    ap.add_argument("--tensor-peaks", action="store_true",
+                    help="measure the dense bf16 / MXFP8 / NVFP4 library GEMM throughput")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward of the bf16 layer (moe_backward) instead")
     ap.add_argument("--soak-s", type=float, default=1.5,
@@ -749,7 +799,9 @@ def main():
         cfg = cfg.scaled(E=args.experts, T=t, name=f"{cfg.name}_E{args.experts}_T{t}")
     elif args.tokens:
         cfg = cfg.scaled(T=args.tokens, name=f"{cfg.name}_T{args.tokens}")
-    if args.backward:
+    if args.tensor_peaks:
+        print(json.dumps(tensor_peaks()), flush=True)
+    elif args.backward:
         run_backward(args, cfg)
     elif args.impl == "reference":
         run_reference(args, cfg)
