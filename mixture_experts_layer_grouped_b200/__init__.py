@@ -30,6 +30,7 @@ from .binding import (  # noqa: F401
     prepare_weights,
     allocate_prepared_weights,
     MoELayer,
+    MoETrainLayer,
     MoEBwdWeights,
     MoEFwdSaved,
     MoEWeightGrads,

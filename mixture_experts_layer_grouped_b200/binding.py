@@ -432,3 +432,76 @@ class MoELayer:
 
     def device_status(self) -> int:
         return moe_get_device_status(self.workspace)
+
+
+class MoETrainLayer(MoELayer):
+    """A bf16 layer that can also run its backward.
+
+    ``forward(x)`` runs the step calls (route, permute, grouped MLP, combine)
+    and keeps what the backward reads; ``backward(dy)`` then returns dx and,
+    by default, every weight gradient (fp32, dict keyed like moe_weight_grads)
+    plus dlogits and dgate.  ``weights`` are the row-major bf16 tensors (w1, w3,
+    w2 and, with a shared expert, ws1, ws3, ws2): they are prepared for the
+    forward and transposed for the backward once, here.  Routed weight
+    gradients need cfg.pad_multiple % 64 == 0.
+    """
+
+    def __init__(self, cfg: MoEConfig, weights: dict, w_router, bias, device="cuda"):
+        super().__init__(cfg, weights, w_router, bias, device)
+        self.bwd_weights = prepare_backward_weights(cfg, weights, w_router)
+        nbytes, r_cap = moe_workspace_size(cfg)
+        self.step_ws = new_workspace(nbytes, device)
+        self.bwd_ws = new_workspace(moe_backward_workspace_size(cfg), device)
+        T, H, E, k = cfg.T, cfg.H, cfg.E, cfg.top_k
+        i32 = dict(dtype=torch.int32, device=device)
+        self.saved = {"logits": torch.empty(T, E, dtype=torch.float32, device=device),
+                      "topk_idx": torch.empty(T, k, **i32),
+                      "topk_w": torch.empty(T, k, dtype=torch.float32, device=device),
+                      "counts": torch.empty(E, **i32), "offsets": torch.empty(E + 1, **i32),
+                      "row_token": torch.empty(r_cap, **i32),
+                      "token_row": torch.empty(T * k, **i32),
+                      "rows": torch.empty(r_cap, H, dtype=torch.bfloat16, device=device),
+                      "out_rows": torch.empty(r_cap, H, dtype=torch.bfloat16, device=device)}
+        self.shared_out = (torch.empty(T, H, dtype=torch.bfloat16, device=device)
+                           if cfg.I_shared > 0 else None)
+
+    def forward(self, x, out=None, stream=None):
+        c, sv = self.cfg, self.saved
+        if out is None:
+            out = torch.empty(c.T, c.H, dtype=torch.bfloat16, device=x.device)
+        moe_route(c, x, self.w_router, self.bias, sv["topk_idx"], sv["topk_w"], self.step_ws,
+                  logits_out=sv["logits"], stream=stream)
+        moe_permute(c, sv["topk_idx"], x, sv["counts"], sv["offsets"], sv["row_token"],
+                    sv["token_row"], sv["rows"], self.step_ws, stream=stream)
+        moe_grouped_mlp(c, self._ws_struct, sv["rows"], sv["counts"], sv["offsets"],
+                        sv["out_rows"], self.step_ws, x=x, shared_out=self.shared_out,
+                        stream=stream)
+        moe_combine(c, sv["out_rows"], sv["token_row"], sv["topk_w"], out,
+                    shared_out=self.shared_out, stream=stream)
+        sv["x"] = x
+        return out
+
+    def backward(self, dy, weight_grads=True, stream=None):
+        c = self.cfg
+        dev = dy.device
+        f32 = dict(dtype=torch.float32, device=dev)
+        dx = torch.empty(c.T, c.H, dtype=torch.bfloat16, device=dev)
+        res = {"dx": dx, "dlogits": torch.empty(c.T, c.E, **f32),
+               "dgate": torch.empty(c.T, c.top_k, **f32)}
+        grads = None
+        if weight_grads:
+            grads = {"dw1": torch.empty(c.E, c.I, c.H, **f32),
+                     "dw3": torch.empty(c.E, c.I, c.H, **f32),
+                     "dw2": torch.empty(c.E, c.H, c.I, **f32),
+                     "dw_router": torch.empty(c.E, c.H, **f32)}
+            if c.I_shared > 0:
+                grads.update(dws1=torch.empty(c.I_shared, c.H, **f32),
+                             dws3=torch.empty(c.I_shared, c.H, **f32),
+                             dws2=torch.empty(c.H, c.I_shared, **f32))
+            res.update(grads)
+        moe_backward(c, self._ws_struct, self.bwd_weights, self.saved, dy, dx, self.bwd_ws,
+                     dlogits=res["dlogits"], dgate=res["dgate"], grads=grads, stream=stream)
+        return res
+
+    def device_status(self) -> int:
+        return max(moe_get_device_status(self.step_ws), moe_get_device_status(self.bwd_ws))

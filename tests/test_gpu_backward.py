@@ -261,3 +261,22 @@ def test_backward_full_size_dsv4_bf16():
     print("dsv4 bf16 backward", {kk: f"{v:.2e}" for kk, v in errs.items()})
     for kk, v in errs.items():
         assert v <= TOL, (kk, v)
+
+
+def test_train_layer_gives_the_same_bits():
+    """MoETrainLayer (forward through the step calls, then backward) gives the
+    bits of the explicit calls above."""
+    import mixture_experts_layer_grouped_b200 as M
+    cfg = SHAPES["small_shared"]
+    d, s, dy, dx, dlogits, dgate, g = _run(cfg)
+    c = M.config_from_shape(cfg)
+    layer = M.MoETrainLayer(c, weights_dict(d), d["w_router"], d["bias"])
+    y = layer.forward(d["x"])
+    res = layer.backward(dy)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.equal(y, s["y"])
+    assert torch.equal(res["dx"], dx) and torch.equal(res["dlogits"], dlogits)
+    assert torch.equal(res["dgate"], dgate)
+    for key in g:
+        assert torch.equal(res[key], g[key]), key
