@@ -1,4 +1,5 @@
-"""CPU oracle of the routed MoE layer forward -- TEST INFRASTRUCTURE ONLY.
+"""CPU oracle of the routed MoE layer (forward, and the bf16 backward) -- TEST
+INFRASTRUCTURE ONLY.
 
 Only the tests, the smoke check and the benchmark's CPU-baseline leg may import
 this module.  The library never calls it, and it shares no code with the CUDA
@@ -18,6 +19,10 @@ Sources (page title, then the passage):
 * sglang PR "Mistral Large 3 NVFP4 TRTLLM MoE support", Modifications: W4A4
   NVFP4 (e2m1 elements, e4m3 scale per 16 along K, fp32 per-tensor global
   scale from amax).
+* TransformerEngine PR "DeepSeekV3Layer", Performance section, "fused grouped
+  MLP" row: the backward of the expert MLP (dGLU and the wgrad GEMMs); the
+  backward here is the gradient of the same layer (dx, the router's dlogits,
+  every weight gradient), written out by the chain rule.
 
 quant_rows.c restates the two row quantizers in plain C (loaded through
 native.py when gcc is available; the CPU tests check it against the numpy
@@ -30,8 +35,9 @@ output rows and of y; the quantized codes of x, of the weights and of h.
 Where the pages leave a step open, the reading taken is stated at the function.
 
 Parity status: every function here is pinned by the CPU tests (brute force on
-tiny inputs, closed forms, library cross-checks, invariants, and a hand-worked
-NVFP4 and MXFP8 expert that pins the quantized composition stage by stage).
+tiny inputs, closed forms, library cross-checks, invariants, a hand-worked
+NVFP4 and MXFP8 expert that pins the quantized composition stage by stage, and
+central finite differences of the forward for every backward function).
 Quantization noise itself has no external truth to pin against; only the
 code-level rules (round-to-nearest-even, saturation, scale selection and the
 scope of each global scale) are pinned.
