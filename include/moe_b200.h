@@ -372,17 +372,21 @@ typedef struct moe_fwd_saved {
 } moe_fwd_saved;
 
 /*
- * Weight gradients, fp32 row-major, written (not accumulated) by moe_backward:
- * dw1, dw3 [E, I, H]; dw2 [E, H, I]; dws1, dws3 [I_shared, H]; dws2
- * [H, I_shared]; dw_router [E, H].  Any field may be NULL: that gradient is
- * not computed.  The routed ones need pad_multiple % 64 == 0
- * (MOE_ERR_UNSUPPORTED otherwise): each expert's rows are read in 64-row
- * steps and the segment pads supply the zeros past its last row.
+ * Weight gradients, fp32 row-major: dw1, dw3 [E, I, H]; dw2 [E, H, I]; dws1,
+ * dws3 [I_shared, H]; dws2 [H, I_shared]; dw_router [E, H].  Any field may be
+ * NULL: that gradient is not computed.  accumulate == 0: the gradients are
+ * written; accumulate != 0: they are added to the values already there (each
+ * element read, summed in fp32 and written by one thread, so repeated calls
+ * give the same bits), e.g. to sum micro-batches.  The routed ones need
+ * pad_multiple % 64 == 0 (MOE_ERR_UNSUPPORTED otherwise): each expert's rows
+ * are read in 64-row steps and the segment pads supply the zeros past its
+ * last row.
  */
 typedef struct moe_weight_grads {
   float* dw1; float* dw3; float* dw2;
   float* dws1; float* dws3; float* dws2;
   float* dw_router;
+  int32_t accumulate;
 } moe_weight_grads;
 
 /*

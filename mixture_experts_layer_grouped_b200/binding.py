@@ -74,7 +74,7 @@ _GRAD_FIELDS = ("dw1", "dw3", "dw2", "dws1", "dws3", "dws2", "dw_router")
 
 
 class MoEWeightGrads(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in _GRAD_FIELDS]
+    _fields_ = [(n, ctypes.c_void_p) for n in _GRAD_FIELDS] + [("accumulate", ctypes.c_int32)]
 
 
 def config_from_shape(s, T=None) -> MoEConfig:
@@ -376,11 +376,12 @@ def moe_backward_workspace_size(cfg: MoEConfig) -> int:
 
 
 def moe_backward(cfg, weights, bwd_weights, saved: dict, dy, dx, workspace, dlogits=None,
-                 dgate=None, grads=None, stream=None):
+                 dgate=None, grads=None, accumulate=False, stream=None):
     """Gradients of the bf16 layer.  ``saved`` maps the moe_fwd_saved field
     names (x, rows, logits, topk_idx, topk_w, counts, offsets, row_token,
     token_row, out_rows) to the forward's tensors; ``grads`` (optional) maps
-    dw1, dw3, dw2, dws1, dws3, dws2, dw_router to fp32 output tensors."""
+    dw1, dw3, dw2, dws1, dws3, dws2, dw_router to fp32 output tensors, which
+    are overwritten, or added to with ``accumulate=True``."""
     ws = weights if isinstance(weights, MoEWeights) else weights_struct(weights)
     bw = bwd_weights if isinstance(bwd_weights, MoEBwdWeights) else MoEBwdWeights(
         **{k: (bwd_weights[k].data_ptr() if bwd_weights.get(k) is not None else None)
@@ -394,7 +395,7 @@ def moe_backward(cfg, weights, bwd_weights, saved: dict, dy, dx, workspace, dlog
     if grads is not None:
         gr = MoEWeightGrads(**{k: (_cuda(grads[k], torch.float32, k).data_ptr()
                                    if grads.get(k) is not None else None)
-                               for k in _GRAD_FIELDS})
+                               for k in _GRAD_FIELDS}, accumulate=1 if accumulate else 0)
     bf = torch.bfloat16
     _check("moe_backward", lib().moe_backward(
         ctypes.byref(cfg), ctypes.byref(ws), ctypes.byref(bw), ctypes.byref(sv),
@@ -481,15 +482,19 @@ class MoETrainLayer(MoELayer):
         sv["x"] = x
         return out
 
-    def backward(self, dy, weight_grads=True, stream=None):
+    def backward(self, dy, weight_grads=True, grads=None, accumulate=False, stream=None):
+        """``grads``: fp32 tensors to write (or, with ``accumulate``, add) the
+        weight gradients into, keyed like moe_weight_grads; allocated when
+        not given."""
         c = self.cfg
         dev = dy.device
         f32 = dict(dtype=torch.float32, device=dev)
         dx = torch.empty(c.T, c.H, dtype=torch.bfloat16, device=dev)
         res = {"dx": dx, "dlogits": torch.empty(c.T, c.E, **f32),
                "dgate": torch.empty(c.T, c.top_k, **f32)}
-        grads = None
-        if weight_grads:
+        if grads is not None:
+            res.update(grads)
+        elif weight_grads:
             grads = {"dw1": torch.empty(c.E, c.I, c.H, **f32),
                      "dw3": torch.empty(c.E, c.I, c.H, **f32),
                      "dw2": torch.empty(c.E, c.H, c.I, **f32),
@@ -500,7 +505,8 @@ class MoETrainLayer(MoELayer):
                              dws2=torch.empty(c.H, c.I_shared, **f32))
             res.update(grads)
         moe_backward(c, self._ws_struct, self.bwd_weights, self.saved, dy, dx, self.bwd_ws,
-                     dlogits=res["dlogits"], dgate=res["dgate"], grads=grads, stream=stream)
+                     dlogits=res["dlogits"], dgate=res["dgate"], grads=grads,
+                     accumulate=accumulate, stream=stream)
         return res
 
     def device_status(self) -> int:

@@ -995,8 +995,9 @@ struct WgDesc {
   bool routed;
 };
 
-moe_status launch_wgrad(const moe_config& c, const WgDesc* d, int n, const int32_t* counts,
-                        const int32_t* offsets, int32_t* status, cudaStream_t s) {
+moe_status launch_wgrad(const moe_config& c, const WgDesc* d, int n, bool accumulate,
+                        const int32_t* counts, const int32_t* offsets, int32_t* status,
+                        cudaStream_t s) {
   if (n < 1) return MOE_OK;
   if (n > kWgMaxProblems) return MOE_ERR_INVALID_ARG;
   WgradParams P;
@@ -1024,6 +1025,7 @@ moe_status launch_wgrad(const moe_config& c, const WgDesc* d, int n, const int32
   P.offsets = offsets;
   P.E = c.E;
   P.dense_rows = c.T;
+  P.accumulate = accumulate ? 1 : 0;
   P.status = status;
   MOE_CUDA(cudaFuncSetAttribute(wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kWgSmemBytes));
@@ -1130,7 +1132,7 @@ moe_status backward_steps(const moe_config& c, const moe_weights& w, const moe_b
   if (dw->dw1) d[n++] = WgDesc{bfp(L.dz), 2 * I, I, f.rows, H, I, H, dw->dw1, true};
   if (dw->dw3) d[n++] = WgDesc{bfp(L.dz) + I, 2 * I, I, f.rows, H, I, H, dw->dw3, true};
   if (dw->dw2) d[n++] = WgDesc{bfp(L.dO), H, H, bfp(L.h), I, H, I, dw->dw2, true};
-  return launch_wgrad(c, d, n, f.counts, f.offsets, status, s);
+  return launch_wgrad(c, d, n, dw->accumulate != 0, f.counts, f.offsets, status, s);
 }
 
 moe_status check_bwd(const moe_config& c, const moe_weights* w, const moe_bwd_weights* wb,

@@ -59,6 +59,7 @@ struct WgradParams {
   const int32_t* counts;   // [E]
   const int32_t* offsets;  // [E + 1]
   int32_t E, dense_rows;
+  int32_t accumulate;  // add to the output's values instead of writing them
   int32_t* status;
 };
 
@@ -240,8 +241,8 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgrad_kernel(const __grid_const
       const int m = t.m0 + quarter * 32 + lane;
       const int nb = t.n0 + half * 128;
       if (t.nrows == 0) {
-        // an expert no token picked: its gradient is zero
-        if (m < q.M) {
+        // an expert no token picked: its gradient is zero (nothing to add)
+        if (m < q.M && !P.accumulate) {
           for (int c = 0; c < 128; c += 4)
             if (nb + c < q.N)
               *reinterpret_cast<float4*>(out + static_cast<int64_t>(m) * q.N + nb + c) =
@@ -273,10 +274,19 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgrad_kernel(const __grid_const
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int row = 4 * i + (lane >> 3), col = 4 * (lane & 7);
-            if (m_base + row < q.M)
-              *reinterpret_cast<float4*>(out + static_cast<int64_t>(m_base + row) * q.N + n +
-                                         col) =
-                  *reinterpret_cast<const float4*>(my + row * kWgStgLd + col);
+            if (m_base + row < q.M) {
+              float4* dst = reinterpret_cast<float4*>(out + static_cast<int64_t>(m_base + row) * q.N +
+                                                      n + col);
+              float4 v = *reinterpret_cast<const float4*>(my + row * kWgStgLd + col);
+              if (P.accumulate) {
+                const float4 o = *dst;
+                v.x += o.x;
+                v.y += o.y;
+                v.z += o.z;
+                v.w += o.w;
+              }
+              *dst = v;
+            }
           }
         }
         __syncwarp();

@@ -280,3 +280,32 @@ def test_train_layer_gives_the_same_bits():
     assert torch.equal(res["dgate"], dgate)
     for key in g:
         assert torch.equal(res[key], g[key]), key
+
+
+def test_weight_grads_accumulate():
+    """accumulate: a second backward adds its weight gradients to the first
+    one's (x + x = 2x exactly in fp32), and experts no token picked keep the
+    values that were there."""
+    import mixture_experts_layer_grouped_b200 as M
+    cfg = SHAPES["decode_shared"]  # most experts empty
+    d = synth.gen_all(cfg, "cuda")
+    c = M.config_from_shape(cfg)
+    layer = M.MoETrainLayer(c, weights_dict(d), d["w_router"], d["bias"])
+    layer.forward(d["x"])
+    dy = synth.gen_dy(cfg, "cuda")
+    once = layer.backward(dy)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    acc = {k: once[k].clone() for k in ("dw1", "dw3", "dw2", "dw_router", "dws1", "dws3", "dws2")}
+    empty = layer.saved["counts"] == 0
+    assert bool(empty.any())
+    marker = torch.full((int(empty.sum()), cfg.I, cfg.H), 7.0, **f32)
+    acc["dw1"][empty] = marker
+    twice = layer.backward(dy, grads=acc, accumulate=True)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.equal(twice["dx"], once["dx"])
+    full = ~empty
+    assert torch.equal(acc["dw1"][full], 2 * once["dw1"][full])
+    assert torch.equal(acc["dw1"][empty], marker)          # untouched
+    for k in ("dw3", "dw2", "dw_router", "dws1", "dws3", "dws2"):
+        assert torch.equal(acc[k], 2 * once[k]), k
