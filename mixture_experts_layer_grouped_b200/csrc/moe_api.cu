@@ -1025,12 +1025,11 @@ moe_status launch_wgrad(const moe_config& c, const WgDesc* d, int n, bool accumu
   P.offsets = offsets;
   P.E = c.E;
   P.dense_rows = c.T;
-  P.accumulate = accumulate ? 1 : 0;
   P.status = status;
-  MOE_CUDA(cudaFuncSetAttribute(wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                kWgSmemBytes));
+  auto kern = accumulate ? wgrad_kernel<true> : wgrad_kernel<false>;
+  MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWgSmemBytes));
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  MOE_TRY(launch_pdl(wgrad_kernel, dim3(grid), dim3(kWgThreads), kWgSmemBytes, s, P));
+  MOE_TRY(launch_pdl(kern, dim3(grid), dim3(kWgThreads), kWgSmemBytes, s, P));
   return launch_check();
 }
 
