@@ -151,3 +151,41 @@ def test_layer_weight_grads_match_finite_differences():
     for e in range(cfg.E):
         if counts[e] == 0:
             assert not analytic["w1"][e].any() and not analytic["w2"][e].any()
+
+
+def test_backward_closed_forms():
+    """Two closed forms that need no finite differences.
+    (i) Every expert the same (W1, W3, W2): y = rsf * MLP(x) for any routing, so
+        dlogits = 0, dx = the single expert's input gradient for dO = rsf * dy,
+        and the experts' weight gradients sum to that expert's for the same dO.
+    (ii) top_k = 1: the gate is rsf whatever the logits, so dlogits = 0."""
+    rng = np.random.default_rng(11)
+    cfg = synth.MoEShape(name="bwd_same", T=6, H=16, I=8, E=4, n_group=2, topk_group=2,
+                         top_k=2, rsf=2.5, I_shared=0, dtype="bf16", pad_multiple=1,
+                         router_std=0.5)
+    x = rng.normal(size=(cfg.T, cfg.H))
+    wr = rng.normal(size=(cfg.E, cfg.H)) * 0.5
+    bias = rng.uniform(-0.1, 0.1, size=cfg.E)
+    W1 = rng.normal(size=(cfg.I, cfg.H)) * 0.3
+    W3 = rng.normal(size=(cfg.I, cfg.H)) * 0.3
+    W2 = rng.normal(size=(cfg.H, cfg.I)) * 0.3
+    dy = rng.normal(size=(cfg.T, cfg.H))
+    rep = lambda W: np.stack([W] * cfg.E)
+    b = O.backward(cfg, x, wr, bias, rep(W1), rep(W3), rep(W2), dy, rounding=False,
+                   weight_grads=True)
+    assert np.max(np.abs(b["dlogits"])) < 1e-12
+    dX, mid = O.expert_backward(x, W1, W3, W2, cfg.rsf * dy)
+    assert np.allclose(b["dx"], dX, rtol=1e-10, atol=1e-12)
+    d1, d3, d2 = O.expert_weight_grads(x, cfg.rsf * dy, mid, rounding=False)
+    assert np.allclose(sum(b["dw1"].values()), d1, rtol=1e-10, atol=1e-12)
+    assert np.allclose(sum(b["dw3"].values()), d3, rtol=1e-10, atol=1e-12)
+    assert np.allclose(sum(b["dw2"].values()), d2, rtol=1e-10, atol=1e-12)
+    assert np.allclose(b["dw_router"], 0.0, atol=1e-12)
+
+    cfg1 = cfg.scaled(name="bwd_top1", top_k=1, topk_group=1)
+    w1 = rng.normal(size=(cfg.E, cfg.I, cfg.H)) * 0.3
+    w3 = rng.normal(size=(cfg.E, cfg.I, cfg.H)) * 0.3
+    w2 = rng.normal(size=(cfg.E, cfg.H, cfg.I)) * 0.3
+    b1 = O.backward(cfg1, x, wr, bias, w1, w3, w2, dy, rounding=False)
+    assert np.max(np.abs(b1["dlogits"])) < 1e-12
+    assert np.abs(b1["dgate"]).max() > 1e-3   # the gate's own gradient is not zero
