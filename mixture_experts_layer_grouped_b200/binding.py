@@ -444,7 +444,8 @@ class MoETrainLayer(MoELayer):
     plus dlogits and dgate.  ``weights`` are the row-major bf16 tensors (w1, w3,
     w2 and, with a shared expert, ws1, ws3, ws2): they are prepared for the
     forward and transposed for the backward once, here.  Routed weight
-    gradients need cfg.pad_multiple % 64 == 0.
+    gradients need cfg.pad_multiple % 64 == 0.  The forward keeps x by
+    reference: it must not change before the backward that follows.
     """
 
     def __init__(self, cfg: MoEConfig, weights: dict, w_router, bias, device="cuda"):
