@@ -2,8 +2,8 @@
 // backward, and the weight copies the dgrad contractions read.  The
 // contractions run on the grouped GEMM (grouped_gemm.cuh: fc2 mode with
 // transposed weight copies, and fc1's backward form, which recomputes a and u
-// and stores both); the weight gradients in wgrad.cuh; see moe_backward in
-// moe_api.cu.
+// and stores both); the weight gradients in wgrad.cuh; the host steps in
+// backward_api.cuh.
 //
 //   combine backward:  dO[row(t, j)] = bf16(w[t, j] * dy[t]),
 //                      g[t, j] = <dy[t], O[row(t, j)]>  (fp32),
