@@ -172,3 +172,19 @@ def test_backward_weight_sizes(M):
     assert sz["w13t"] == s.E * s.H * 2 * s.I * 2
     assert sz["ws2t"] == s.I_shared * s.H * 2
     assert sz["wdt"] == s.H * (2 * s.I_shared + 64) * 2  # E = 64 columns of W_r^T
+
+
+def test_binding_rejects_host_tensors_for_the_backward(M):
+    """The binding's marshalling checks device, dtype and layout before any C
+    call: host tensors are refused with a ValueError."""
+    import torch
+    s = synth.get_config("tiny_bf16_T64").scaled(pad_multiple=64)
+    c = M.config_from_shape(s)
+    x = torch.zeros(s.T, s.H, dtype=torch.bfloat16)
+    saved = {k: x for k in ("x", "rows", "out_rows")}
+    saved.update({k: torch.zeros(4, dtype=torch.int32) for k in
+                  ("topk_idx", "counts", "offsets", "row_token", "token_row")})
+    saved.update(logits=torch.zeros(4), topk_w=torch.zeros(4))
+    with pytest.raises(ValueError):
+        M.moe_backward(c, M.MoEWeights(), M.MoEBwdWeights(), saved, x, x,
+                       torch.zeros(16, dtype=torch.uint8))
